@@ -1,0 +1,457 @@
+#!/usr/bin/env python
+"""Benchmark of the block-sparse bidirectional attention hot path on B200.
+
+One bench step = one complete denoising run of one attention layer through
+the library's step driver (sparsed_run_steps): dense attention for the warm-up
+steps, pattern selection (dense pass + block mass + top-k) at the switch and at
+anchors, block-sparse attention afterwards. Default workload: c4_64k
+(H=32, L=65536, d=128, bq=bk=128, keep 0.10, T=1024, first 20% dense).
+
+Metric: effective TFLOP/s = attention flops of the run / device time, counting
+4*L*L*d per head for a dense or selecting step and 4*bq*bk*d per kept block for
+a sparse step (the block-mass pass of a selecting step is overhead, not counted).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+With N > 1 (launched by torchrun) every rank runs its own independent layer
+(weak scaling, no data-path collective); the time is the max over ranks.
+--impl reference times the fp64 CPU oracle on this host's cores on a bounded
+sample of the same workload (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from block_sparse_bidirectional_select_b200.inputs import WORKLOADS, make_inputs, to_f64  # noqa: E402
+
+METRIC = "block-sparse attn effective TFLOP/s & ms/step at 64k, % of B200 bf16 peak"
+UNIT = "TFLOP/s"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def log(*a):
+    print(*a, file=sys.stderr, flush=True)
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return p, "measured"
+    except (OSError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ----------------------------------------------------------------- accounting
+
+def run_accounting(wl, kinds, kv_count_sum):
+    """Effective flops of one run and the kernel launches it makes."""
+    dense = 4.0 * wl.H * float(wl.L) * float(wl.L) * wl.d
+    sparse = 4.0 * wl.bq * wl.bk * wl.d * float(kv_count_sum)
+    n_dense = kinds.count(0)
+    n_select = kinds.count(1)
+    n_sparse = kinds.count(2)
+    per_select = 3 + (2 if wl.budget == "entropy" else 0)  # dense, mass, [entropy, budget], top-k
+    return dict(flops=(n_dense + n_select) * dense + n_sparse * sparse, dense_flops=dense,
+                sparse_flops=sparse, n_dense=n_dense, n_select=n_select, n_sparse=n_sparse,
+                launches=n_dense + n_select * per_select + n_sparse)
+
+
+# ----------------------------------------------------------------- clocks
+
+class ClockSampler:
+    FIELDS = ["clocks.sm", "clocks.max.sm", "power.draw", "clocks_event_reasons.hw_slowdown",
+              "clocks_event_reasons.hw_thermal_slowdown", "clocks_event_reasons.sw_thermal_slowdown",
+              "clocks_event_reasons.sw_power_cap"]
+    REASONS = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+
+    def __init__(self, device_index):
+        self.dev = device_index
+        self.proc = None
+        self.lines = []
+        self.thread = None
+
+    def _gpu_id(self):
+        try:
+            uuid = torch.cuda.get_device_properties(self.dev).uuid
+            s = str(uuid)
+            return s if s.startswith("GPU-") else "GPU-" + s
+        except Exception:
+            return str(self.dev)
+
+    def start(self):
+        cmd = ["nvidia-smi", f"--id={self._gpu_id()}", "--query-gpu=" + ",".join(self.FIELDS),
+               "--format=csv,noheader,nounits", "-lms", "200"]
+        try:
+            self.proc = subprocess.Popen(cmd, stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        if self.thread:
+            self.thread.join(timeout=5)
+        sm, smax, reasons = [], [], set()
+        for ln in self.lines:
+            parts = [x.strip() for x in ln.split(",")]
+            if len(parts) != len(self.FIELDS):
+                continue
+            try:
+                sm.append(float(parts[0]))
+                smax.append(float(parts[1]))
+            except ValueError:
+                continue
+            for name, val in zip(self.REASONS, parts[3:]):
+                if val.lower().startswith("active"):
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ----------------------------------------------------------------- CPU oracle
+
+def cpu_oracle_sample(wl, q, k, v, budget_s, rng_seed=0):
+    """Time the fp64 oracle on sampled (head, query block) tiles of this
+    workload: the dense rows of the tile, its block-mass row, its top-k and its
+    block-masked rows; extrapolate to the effective TFLOP/s of a full run."""
+    import oracle as O
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+    except Exception:
+        cores = os.cpu_count() or 1
+    nqb, nkb = -(-wl.L // wl.bq), -(-wl.L // wl.bk)
+    kk = O.uniform_keep(nkb, wl.keep)
+    rng = np.random.default_rng(rng_seed)
+    t_dense = t_mass = t_sparse = 0.0
+    n = 0
+    heads = {}
+    t_start = time.perf_counter()
+    while time.perf_counter() - t_start < budget_s and n < 64:
+        h = int(rng.integers(wl.H))
+        i = int(rng.integers(nqb))
+        if h not in heads:
+            heads.clear()
+            heads[h] = (to_f64(q[h]), to_f64(k[h]), to_f64(v[h]))
+        qh, kh, vh = heads[h]
+        r0, r1 = i * wl.bq, min((i + 1) * wl.bq, wl.L)
+        t0 = time.perf_counter()
+        _, lse = O.dense_attention(qh[r0:r1], kh, vh, wl.scale)
+        t1 = time.perf_counter()
+        lse_full = np.zeros(wl.L)
+        lse_full[r0:r1] = lse
+        mrow = O.block_mass(qh, kh, wl.scale, lse_full, wl.bq, wl.bk, qblocks=[i])[0]
+        sel = O.topk_blocks(mrow, kk)
+        t2 = time.perf_counter()
+        keys = O.kept_keys(sel, wl.bk, wl.L)
+        O.softmax_attention(qh[r0:r1], kh[keys], vh[keys], wl.scale)
+        t3 = time.perf_counter()
+        t_dense += t1 - t0
+        t_mass += t2 - t1
+        t_sparse += t3 - t2
+        n += 1
+    tiles = wl.H * nqb
+    kinds = O.schedule(wl.T, wl.warmup_frac, wl.refresh_every)
+    acc = run_accounting(wl, kinds, wl.H * nqb * kk)
+    step_dense = tiles * t_dense / n
+    step_select = tiles * (t_dense + t_mass) / n
+    step_sparse = tiles * t_sparse / n
+    run_s = acc["n_dense"] * step_dense + acc["n_select"] * step_select + acc["n_sparse"] * step_sparse
+    value = acc["flops"] / run_s / 1e12
+    sample = (f"{n} (head, query-block) tiles of {wl.name}: fp64 dense rows + block-mass row + top-k + "
+              f"masked rows per tile, {t_dense + t_mass + t_sparse:.1f} s of oracle time, "
+              f"extrapolated to a full {wl.T}-step run ({tiles} tiles per step)")
+    return {"value": value, "unit": UNIT, "cores": int(cores), "kind": "oracle", "sample": sample,
+            "ms_per_step_extrapolated": run_s * 1e3}
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return 0
+    wl = WORKLOADS[args.workload]
+    log(f"[reference] generating inputs for {wl.name}")
+    q, k, v = make_inputs(wl)
+    budget = args.cpu_seconds
+    for _ in range(args.warmup):
+        cpu_oracle_sample(wl, q, k, v, min(budget, 5.0), rng_seed=99)
+    vals, base = [], None
+    t0 = time.perf_counter()
+    for s in range(args.steps):
+        base = cpu_oracle_sample(wl, q, k, v, budget, rng_seed=s)
+        vals.append(base["value"])
+    wall = time.perf_counter() - t0
+    value = statistics.median(vals)
+    base = dict(base, value=value)
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": base["ms_per_step_extrapolated"],
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": workload_config(wl),
+            "cpu_baseline": base,
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+            "wall_s_sampling": wall}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ----------------------------------------------------------------- GPU arm
+
+def workload_config(wl):
+    return {"workload": wl.name, "H": wl.H, "L": wl.L, "d": wl.d, "bq": wl.bq, "bk": wl.bk,
+            "keep": wl.keep, "budget": wl.budget, "T": wl.T, "warmup_frac": wl.warmup_frac,
+            "refresh_every": wl.refresh_every, "inputs": wl.structure,
+            "l2": "inputs larger than L2 (Q,K,V %.2f GiB vs 126 MB)" % (3 * wl.H * wl.L * wl.d * 2 / 2**30)}
+
+
+def event_time(fn, stream, n):
+    s = torch.cuda.Event(enable_timing=True)
+    e = torch.cuda.Event(enable_timing=True)
+    s.record(stream)
+    for _ in range(n):
+        fn()
+    e.record(stream)
+    e.synchronize()
+    return s.elapsed_time(e)
+
+
+def median_time(fn, stream, reps):
+    out = []
+    for _ in range(reps):
+        out.append(event_time(fn, stream, 1))
+    return statistics.median(out)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="c4_64k", choices=sorted(WORKLOADS))
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--skip-cpu", action="store_true")
+    ap.add_argument("--skip-e2e", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        return run_reference(args, rank, world)
+
+    import block_sparse_bidirectional_select_b200 as sp
+    import torch.distributed as dist
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", device_id=dev, timeout=datetime.timedelta(seconds=900))
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def max_over_ranks(x):
+        if world == 1:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    wl = WORKLOADS[args.workload]
+    log(f"[rank {rank}] inputs for {wl.name}")
+    q_cpu, k_cpu, v_cpu = make_inputs(wl.scaled(seed=wl.seed + rank))
+    q, k, v = (t.to(dev) for t in (q_cpu, k_cpu, v_cpu))
+    stream = torch.cuda.current_stream()
+    peaks, peak_src = load_peaks()
+
+    H, L, d = wl.H, wl.L, wl.d
+    nqb = -(-L // wl.bq)
+    ws = torch.empty(sp.workspace_bytes(H, L, wl.bq, wl.bk), dtype=torch.uint8, device=dev)
+    o = torch.empty_like(q)
+    lse = torch.empty((H, L), dtype=torch.float32, device=dev)
+
+    def one_run(time_steps=False):
+        return sp.run_steps(q, k, v, wl.T, wl.warmup_frac, keep=wl.keep, budget=wl.budget,
+                            refresh_every=wl.refresh_every, bq=wl.bq, bk=wl.bk, out=o, lse=lse,
+                            workspace=ws, time_steps=time_steps)
+
+    log(f"[rank {rank}] warm-up x{args.warmup}")
+    for _ in range(args.warmup):
+        res = one_run()
+    sp.device_check()
+    kinds = res.kinds
+    kv_sum = int(res.kv_count.sum().item())
+    acc = run_accounting(wl, kinds, kv_sum)
+
+    # ---------------- timed region: K full runs
+    torch.cuda.synchronize()
+    barrier()
+    clocks = ClockSampler(local)
+    clocks.start()
+    step_ms = []
+    s_ev = torch.cuda.Event(enable_timing=True)
+    e_ev = torch.cuda.Event(enable_timing=True)
+    s_ev.record(stream)
+    for _ in range(args.steps):
+        r = one_run(time_steps=True)
+        step_ms.append(r.step_ms)
+    e_ev.record(stream)
+    e_ev.synchronize()
+    torch.cuda.synchronize()
+    barrier()
+    clk = clocks.stop()
+    total_ms = max_over_ranks(s_ev.elapsed_time(e_ev))
+    sp.device_check()
+    ms_per_step = total_ms / args.steps
+    value = acc["flops"] * args.steps * world / (total_ms * 1e-3) / 1e12
+
+    per_kind = {0: [], 1: [], 2: []}
+    for run in step_ms:
+        for kind, ms in zip(kinds, run):
+            per_kind[kind].append(ms)
+    dense_ms = statistics.mean(per_kind[0]) if per_kind[0] else None
+    select_ms = statistics.mean(per_kind[1]) if per_kind[1] else None
+    sparse_ms = statistics.mean(per_kind[2]) if per_kind[2] else None
+
+    peak_tc = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
+    peak_burst = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
+    time_dense = (acc["n_dense"] * (dense_ms or 0.0))
+    time_sparse = (acc["n_sparse"] * (sparse_ms or 0.0))
+    dominant = "dense" if time_dense >= time_sparse else "sparse"
+    d_ach = acc["dense_flops"] / (dense_ms * 1e-3) / 1e12 if dense_ms else None
+    s_ach = acc["sparse_flops"] / (sparse_ms * 1e-3) / 1e12 if sparse_ms else None
+    traffic = load_traffic(wl.name)
+
+    def roof(kernel, ach, units):
+        return {"kernel": kernel, "bound": "tensor", "achieved": ach, "peak": peak_tc, "unit": "TFLOP/s",
+                "frac": (ach / peak_tc) if ach else None,
+                "peak_source": f"{peak_src} bf16_tflops_sustained (kernel timed inside the long run)",
+                "units_per_launch": units, "traffic": traffic.get(kernel)}
+
+    dense_name = f"attn_fwd_kernel<{d},{wl.bk},dense>"
+    sparse_name = f"attn_fwd_kernel<{d},{wl.bk},sparse>"
+    roof_dense = roof(dense_name, d_ach, f"{H}x{L}x{L} score tiles, 4*H*L^2*d flops")
+    roof_sparse = roof(sparse_name, s_ach, f"{kv_sum} kept blocks, 4*bq*bk*d flops each")
+    roofline = roof_dense if dominant == "dense" else roof_sparse
+
+    # ---------------- single-kernel timings (context)
+    extra = {}
+    if res.kv_idx is not None and acc["n_sparse"] > 0:
+        fn = lambda: sp.block_sparse_attn(q, k, v, res.kv_idx, res.kv_count, bq=wl.bq, bk=wl.bk, out=o, lse=lse)
+        fn()
+        ms = median_time(fn, stream, 20)
+        tf = acc["sparse_flops"] / (ms * 1e-3) / 1e12
+        extra["block_sparse_attn"] = {"ms": ms, "tflops": tf, "frac_of_peak_burst": tf / peak_burst,
+                                      "peak_burst": peak_burst, "kept_blocks": kv_sum}
+    fn = lambda: sp.dense_attn(q, k, v, bq=wl.bq, bk=wl.bk, out=o, lse=lse)
+    fn()
+    ms = median_time(fn, stream, 3)
+    extra["dense_attn"] = {"ms": ms, "tflops": acc["dense_flops"] / (ms * 1e-3) / 1e12}
+    try:
+        import torch.nn.functional as F
+        q4, k4, v4 = (t.unsqueeze(0) for t in (q, k, v))
+        fn = lambda: F.scaled_dot_product_attention(q4, k4, v4)
+        fn()
+        ms = median_time(fn, stream, 3)
+        extra["torch_sdpa_dense"] = {"ms": ms, "tflops": acc["dense_flops"] / (ms * 1e-3) / 1e12}
+    except Exception as ex:  # context only
+        extra["torch_sdpa_dense"] = {"error": str(ex)[:200]}
+    sp.device_check()
+
+    # ---------------- end to end through the public API with host buffers
+    e2e = None
+    if not args.skip_e2e:
+        qh, kh, vh = (t.pin_memory() for t in (q_cpu, k_cpu, v_cpu))
+        oh = torch.empty(o.shape, dtype=o.dtype).pin_memory()
+        lh = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
+        qd, kd, vd = (torch.empty_like(t) for t in (q, k, v))
+
+        def e2e_run():
+            qd.copy_(qh, non_blocking=True)
+            kd.copy_(kh, non_blocking=True)
+            vd.copy_(vh, non_blocking=True)
+            sp.run_steps(qd, kd, vd, wl.T, wl.warmup_frac, keep=wl.keep, budget=wl.budget,
+                         refresh_every=wl.refresh_every, bq=wl.bq, bk=wl.bk, out=o, lse=lse, workspace=ws)
+            oh.copy_(o, non_blocking=True)
+            lh.copy_(lse, non_blocking=True)
+
+        torch.cuda.synchronize()
+        barrier()
+        e2e_ms = max_over_ranks(event_time(e2e_run, stream, args.steps))
+        torch.cuda.synchronize()
+        bi = 3 * q.numel() * q.element_size()
+        bo = o.numel() * o.element_size() + lse.numel() * lse.element_size()
+        e2e = {"value": acc["flops"] * args.steps * world / (e2e_ms * 1e-3) / 1e12, "unit": UNIT,
+               "h2d_bytes_per_step": bi, "d2h_bytes_per_step": bo, "ms_per_step": e2e_ms / args.steps}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.skip_cpu:
+        log("[rank 0] timing the CPU oracle on a bounded sample")
+        cpu = cpu_oracle_sample(wl, q_cpu, k_cpu, v_cpu, args.cpu_seconds)
+
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": dict(workload_config(wl), parallelism=f"replicas x{world}" if world > 1 else "single"),
+        "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": acc["launches"] * args.steps,
+        "clocks": clk,
+        "pct_of_peak": {"value_vs_burst": value / world / peak_burst, "value_vs_sustained": value / world / peak_tc,
+                        "peak_source": peak_src},
+        "ms_per_denoise_step": ms_per_step / wl.T,
+        "steps_breakdown": {"dense_ms": dense_ms, "select_ms": select_ms, "sparse_ms": sparse_ms,
+                            "n_dense": acc["n_dense"], "n_select": acc["n_select"], "n_sparse": acc["n_sparse"]},
+        "roofline_sparse": roof_sparse, "roofline_dense": roof_dense,
+        **extra,
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
+def load_traffic(workload):
+    """DRAM bytes per launch from the committed ncu summary, when one exists
+    for the current kernels (profiles/traffic.json)."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            t = json.load(f)
+        return t.get(workload, {})
+    except (OSError, ValueError):
+        return {}
+
+
+if __name__ == "__main__":
+    sys.exit(main())

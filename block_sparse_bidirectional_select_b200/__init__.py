@@ -1,0 +1,212 @@
+"""Block-sparse bidirectional attention for diffusion-LM denoising on B200.
+
+Thin Python binding over the C ABI of libsparsed.so (include/sparsed.h). Each
+function checks and marshals torch tensors (device memory, dtype, contiguity)
+and passes raw pointers plus the current CUDA stream; every step of the
+computation runs in the library's sm_100a kernels. torch is used only for
+device memory and streams.
+
+    dense_attn(q, k, v)                      -> (o, lse)
+    select_pattern(q, k, v, keep, budget)    -> Pattern (o, lse, kv_idx, kv_count, ...)
+    block_sparse_attn(q, k, v, kv_idx, kv_count) -> (o, lse)
+    run_steps(q, k, v, T, warmup_frac, ...)  -> RunResult (o, lse, kinds, step_ms, pattern)
+
+q, k, v are [H, L, d] bf16 CUDA tensors (d in {64, 128}); o is [H, L, d] bf16,
+lse [H, L] fp32 natural log; kv_idx [H, nqb, kv_stride] int32 and kv_count
+[H, nqb] int32 hold the per-(head, query block) kept key blocks, ascending.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+from dataclasses import dataclass
+
+import torch
+
+from . import _lib
+from ._lib import (BUDGET_ENTROPY, BUDGET_UNIFORM, STEP_DENSE, STEP_SELECT,  # noqa: F401
+                   STEP_SPARSE, SparsedError, check)
+
+__all__ = ["dense_attn", "select_pattern", "block_sparse_attn", "run_steps", "workspace_bytes",
+           "uniform_keep", "schedule", "device_check", "version", "SparsedError", "Pattern",
+           "RunResult", "default_scale"]
+
+
+def _ptr(t: torch.Tensor | None):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _check_qkv(q, k, v):
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        if not isinstance(t, torch.Tensor):
+            raise TypeError(f"{name} must be a torch.Tensor")
+        if t.dtype != torch.bfloat16:
+            raise TypeError(f"{name} must be bfloat16, got {t.dtype}")
+        if t.device.type != "cuda":
+            raise ValueError(f"{name} must be a CUDA tensor")
+        if t.dim() != 3 or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous [H, L, d] tensor")
+    if not (q.shape == k.shape == v.shape):
+        raise ValueError(f"q, k, v shapes differ: {tuple(q.shape)} {tuple(k.shape)} {tuple(v.shape)}")
+    if not (q.device == k.device == v.device):
+        raise ValueError("q, k, v must be on the same device")
+    return q.shape
+
+
+def default_scale(d: int) -> float:
+    """1/sqrt(d) rounded to fp32 (the value the C ABI receives)."""
+    return float(torch.tensor(1.0 / math.sqrt(d), dtype=torch.float32))
+
+
+def version() -> int:
+    return _lib.load().sparsed_version()
+
+
+def uniform_keep(L: int, bk: int, keep: float) -> int:
+    k = ctypes.c_int()
+    check(_lib.load().sparsed_uniform_keep(L, bk, keep, ctypes.byref(k)), "sparsed_uniform_keep")
+    return k.value
+
+
+def schedule(T: int, warmup_frac: float, refresh_every: int = 0) -> list[int]:
+    buf = (ctypes.c_int8 * max(T, 1))()
+    check(_lib.load().sparsed_schedule(T, warmup_frac, refresh_every, ctypes.cast(buf, ctypes.c_void_p)),
+          "sparsed_schedule")
+    return list(buf[:T])
+
+
+def workspace_bytes(H: int, L: int, bq: int = 128, bk: int = 128) -> int:
+    n = ctypes.c_size_t()
+    check(_lib.load().sparsed_workspace_bytes(H, L, bq, bk, ctypes.byref(n)), "sparsed_workspace_bytes")
+    return n.value
+
+
+def device_check(stream=None) -> None:
+    """Synchronise the stream and raise if a kernel recorded a device-side fault."""
+    check(_lib.load().sparsed_check(_stream(stream)), "sparsed_check")
+
+
+def _alloc_out(q, out, lse):
+    H, L, _ = q.shape
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((H, L), dtype=torch.float32, device=q.device)
+    return out, lse
+
+
+def _workspace(q, bq, bk, workspace):
+    H, L, _ = q.shape
+    need = workspace_bytes(H, L, bq, bk)
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    return workspace
+
+
+def dense_attn(q, k, v, scale=None, bq=128, bk=128, out=None, lse=None, stream=None):
+    """Dense bidirectional attention: returns (o [H,L,d] bf16, lse [H,L] fp32)."""
+    H, L, d = _check_qkv(q, k, v)
+    scale = default_scale(d) if scale is None else scale
+    out, lse = _alloc_out(q, out, lse)
+    rc = _lib.load().sparsed_dense_attn(_ptr(q), _ptr(k), _ptr(v), H, L, d, scale, bq, bk, _ptr(out),
+                                        _ptr(lse), _stream(stream))
+    check(rc, "sparsed_dense_attn")
+    return out, lse
+
+
+@dataclass
+class Pattern:
+    o: torch.Tensor
+    lse: torch.Tensor
+    kv_idx: torch.Tensor       # [H, nqb, kv_stride] int32
+    kv_count: torch.Tensor     # [H, nqb] int32
+    block_mass: torch.Tensor | None
+    head_k: torch.Tensor       # [H] int32
+
+
+def select_pattern(q, k, v, keep=0.1, budget="uniform", scale=None, bq=128, bk=128, kv_stride=None,
+                   return_mass=False, workspace=None, stream=None) -> Pattern:
+    """Full-attention pass plus block-sparse pattern selection."""
+    H, L, d = _check_qkv(q, k, v)
+    scale = default_scale(d) if scale is None else scale
+    mode = {"uniform": BUDGET_UNIFORM, "entropy": BUDGET_ENTROPY}[budget]
+    nqb, nkb = -(-L // bq), -(-L // bk)
+    if kv_stride is None:
+        kv_stride = uniform_keep(L, bk, keep) if (mode == BUDGET_UNIFORM and L > 0) else max(nkb, 1)
+    dev = q.device
+    out, lse = _alloc_out(q, None, None)
+    kv_idx = torch.full((H, nqb, kv_stride), -1, dtype=torch.int32, device=dev)
+    kv_count = torch.zeros((H, nqb), dtype=torch.int32, device=dev)
+    mass = torch.empty((H, nqb, nkb), dtype=torch.float32, device=dev) if return_mass else None
+    head_k = torch.zeros(H, dtype=torch.int32, device=dev)
+    ws = _workspace(q, bq, bk, workspace)
+    rc = _lib.load().sparsed_select_pattern(
+        _ptr(q), _ptr(k), _ptr(v), H, L, d, scale, bq, bk, keep, mode, _ptr(out), _ptr(lse),
+        _ptr(kv_idx), _ptr(kv_count), kv_stride, _ptr(mass), _ptr(head_k), _ptr(ws), ws.numel(),
+        _stream(stream))
+    check(rc, "sparsed_select_pattern")
+    return Pattern(out, lse, kv_idx, kv_count, mass, head_k)
+
+
+def block_sparse_attn(q, k, v, kv_idx, kv_count, scale=None, bq=128, bk=128, out=None, lse=None,
+                      stream=None):
+    """Block-sparse attention over a cached pattern: returns (o, lse)."""
+    H, L, d = _check_qkv(q, k, v)
+    scale = default_scale(d) if scale is None else scale
+    for name, t in (("kv_idx", kv_idx), ("kv_count", kv_count)):
+        if t.dtype != torch.int32 or not t.is_contiguous() or t.device != q.device:
+            raise ValueError(f"{name} must be a contiguous int32 tensor on {q.device}")
+    nqb = -(-L // bq)
+    if kv_idx.dim() != 3 or kv_idx.shape[:2] != (H, nqb) or kv_count.shape != (H, nqb):
+        raise ValueError(f"pattern shapes must be [H, nqb, stride] and [H, nqb] with nqb={nqb}")
+    out, lse = _alloc_out(q, out, lse)
+    rc = _lib.load().sparsed_block_sparse_attn(
+        _ptr(q), _ptr(k), _ptr(v), H, L, d, scale, bq, bk, _ptr(kv_idx), _ptr(kv_count),
+        kv_idx.shape[2], _ptr(out), _ptr(lse), _stream(stream))
+    check(rc, "sparsed_block_sparse_attn")
+    return out, lse
+
+
+@dataclass
+class RunResult:
+    o: torch.Tensor
+    lse: torch.Tensor
+    kinds: list
+    step_ms: list | None
+    kv_idx: torch.Tensor
+    kv_count: torch.Tensor
+
+
+def run_steps(q, k, v, T, warmup_frac=0.2, keep=0.1, budget="uniform", refresh_every=0, scale=None,
+              bq=128, bk=128, start_step=0, pattern=None, time_steps=False, out=None, lse=None,
+              workspace=None, stream=None) -> RunResult:
+    """The denoising loop over one layer: dense warm-up, pattern selection at
+    the switch (and at anchors), block-sparse attention afterwards."""
+    H, L, d = _check_qkv(q, k, v)
+    scale = default_scale(d) if scale is None else scale
+    mode = {"uniform": BUDGET_UNIFORM, "entropy": BUDGET_ENTROPY}[budget]
+    nqb, nkb = -(-L // bq), -(-L // bk)
+    if pattern is not None:
+        kv_idx, kv_count = pattern
+        have = 1
+    else:
+        stride = uniform_keep(L, bk, keep) if (mode == BUDGET_UNIFORM and L > 0) else max(nkb, 1)
+        kv_idx = torch.full((H, nqb, stride), -1, dtype=torch.int32, device=q.device)
+        kv_count = torch.zeros((H, nqb), dtype=torch.int32, device=q.device)
+        have = 0
+    out, lse = _alloc_out(q, out, lse)
+    ws = _workspace(q, bq, bk, workspace)
+    kinds = (ctypes.c_int8 * max(T, 1))()
+    ms = (ctypes.c_float * max(T, 1))() if time_steps else None
+    rc = _lib.load().sparsed_run_steps(
+        _ptr(q), _ptr(k), _ptr(v), H, L, d, scale, bq, bk, keep, mode, T, warmup_frac, refresh_every,
+        start_step, have, _ptr(kv_idx), _ptr(kv_count), kv_idx.shape[2], _ptr(out), _ptr(lse),
+        ctypes.cast(kinds, ctypes.c_void_p), None if ms is None else ctypes.cast(ms, ctypes.c_void_p),
+        _ptr(ws), ws.numel(), _stream(stream))
+    check(rc, "sparsed_run_steps")
+    return RunResult(out, lse, list(kinds[:T]), None if ms is None else list(ms[:T]), kv_idx, kv_count)

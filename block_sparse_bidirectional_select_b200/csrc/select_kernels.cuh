@@ -1,0 +1,385 @@
+// Pattern selection after the full-attention pass (SparseD abstract: the
+// head-specific sparse pattern is computed once from full attention; Step-dLLM
+// abstract: a block-sparse mask under a uniform or head-adaptive budget).
+//
+//   block_mass_kernel   M[h,i,j] = sum_{r in qblk i, c in kblk j}
+//                                  exp(scale*<q_r,k_c> - LSE_r)
+//                       recomputes S = Q K^T on tcgen05 (fp32 in TMEM) and
+//                       reduces every 128 x BK tile to one fp32 scalar in a
+//                       fixed order (bit-reproducible).
+//   row_entropy_kernel  entropy of each row M[h,i,:] / sum_j M[h,i,j] (fp64)
+//   budget_kernel       per-head k_h from the mean row entropy (fp64, one thread)
+//   topk_kernel         per (h,i): the k_h largest masses, ties to the lower
+//                       block index, written in ascending block order.
+#pragma once
+
+#include "ptx_sm100.cuh"
+
+namespace sparsed {
+
+struct MassArgs {
+  int H, L, bq, nqb, nkb;
+  float scale_log2;
+  const float* lse;   // [H, L]
+  float* mass;        // [H, nqb, nkb]
+  uint64_t timeout_ns;
+};
+
+template <int D, int BK>
+struct MassCfg {
+  static constexpr int M = 128;
+  static constexpr int STAGES = 3;
+  static constexpr int DCH = D / 64;
+  static constexpr int Q_CHUNK = M * 128;
+  static constexpr int KV_CHUNK = BK * 128;
+  static constexpr int Q_BYTES = M * D * 2;
+  static constexpr int K_BYTES = BK * D * 2;
+  static constexpr int OFF_Q = 0;
+  static constexpr int OFF_K = Q_BYTES;
+  static constexpr int OFF_BAR = OFF_K + STAGES * K_BYTES;
+  static constexpr int B_QFULL = 0;
+  static constexpr int B_KFULL = 1;
+  static constexpr int B_KEMPTY = B_KFULL + STAGES;
+  static constexpr int B_SFULL = B_KEMPTY + STAGES;
+  static constexpr int B_SFREE = B_SFULL + 2;
+  static constexpr int B_DRAIN = B_SFREE + 2;
+  static constexpr int NUM_BARS = B_DRAIN + 1;
+  static constexpr int OFF_RED = OFF_BAR + NUM_BARS * 8;     // float red[2][4]
+  static constexpr int OFF_MISC = OFF_RED + 2 * 4 * 4;       // tmem slot, abort flag
+  static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;
+  static constexpr int TM_S0 = 0;
+  static constexpr int TM_S1 = BK;
+  static constexpr int TM_ALLOC = 2 * BK <= 128 ? 128 : 256;
+  static constexpr uint32_t IDESC_S = ptx::idesc_bf16_f32(128, BK, 0, 0);
+  static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+};
+
+template <int D, int BK>
+__global__ void __launch_bounds__(256, 1)
+    block_mass_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                      const MassArgs a) {
+  using C = MassCfg<D, BK>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  const uint32_t sb = ptx::smem_u32(smem);
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int qi = blockIdx.x;
+  const int h = blockIdx.y;
+  const int n = a.nkb;
+  float* red = reinterpret_cast<float*>(smem + C::OFF_RED);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
+  auto bar = [&](int idx) -> uint32_t { return sb + C::OFF_BAR + 8 * idx; };
+
+  if (threadIdx.x == 0) {
+    ptx::mbar_init(bar(C::B_QFULL), 1);
+    for (int s = 0; s < C::STAGES; ++s) {
+      ptx::mbar_init(bar(C::B_KFULL + s), 1);
+      ptx::mbar_init(bar(C::B_KEMPTY + s), 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      ptx::mbar_init(bar(C::B_SFULL + b), 1);
+      ptx::mbar_init(bar(C::B_SFREE + b), 128);
+    }
+    ptx::mbar_init(bar(C::B_DRAIN), 1);
+    *abort_flag = 0;
+    ptx::fence_mbar_init();
+  }
+  if (warp == 1) {
+    ptx::tmem_alloc(ptx::smem_u32(tmem_slot), C::TM_ALLOC);
+    ptx::tmem_relinquish();
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0 && lane == 0) {
+    // ================================================================ producer
+    ptx::mbar_arrive_expect_tx(bar(C::B_QFULL), C::Q_BYTES);
+#pragma unroll
+    for (int c = 0; c < C::DCH; ++c)
+      ptx::tma_load_3d(sb + C::OFF_Q + c * C::Q_CHUNK, &tm_q, bar(C::B_QFULL), c * 64, qi * a.bq, h);
+    int issued = 0;
+    for (int j = 0; j < n; ++j) {
+      const int s = j % C::STAGES;
+      const uint32_t use = static_cast<uint32_t>(j / C::STAGES);
+      if (j >= C::STAGES &&
+          !ptx::mbar_wait(bar(C::B_KEMPTY + s), (use - 1) & 1, abort_flag, a.timeout_ns, kErrTimeout))
+        break;
+      ptx::mbar_arrive_expect_tx(bar(C::B_KFULL + s), C::K_BYTES);
+#pragma unroll
+      for (int c = 0; c < C::DCH; ++c)
+        ptx::tma_load_3d(sb + C::OFF_K + s * C::K_BYTES + c * C::KV_CHUNK, &tm_k, bar(C::B_KFULL + s),
+                         c * 64, j * BK, h);
+      ++issued;
+    }
+    if (*abort_flag) {
+      const uint64_t short_ns = a.timeout_ns / 4;
+      for (int t = (issued > C::STAGES ? issued - C::STAGES : 0); t < issued; ++t) {
+        volatile int dummy = 0;
+        ptx::mbar_wait(bar(C::B_KFULL + t % C::STAGES), (t / C::STAGES) & 1, &dummy, short_ns, 0);
+      }
+    }
+  } else if (warp == 1 && lane == 0) {
+    // ================================================================ MMA issuer
+    bool ok = ptx::mbar_wait(bar(C::B_QFULL), 0, abort_flag, a.timeout_ns, kErrTimeout);
+    ptx::tc_fence_after();
+    for (int j = 0; ok && j < n; ++j) {
+      const int s = j % C::STAGES;
+      const int b = j & 1;
+      if (!ptx::mbar_wait(bar(C::B_KFULL + s), (j / C::STAGES) & 1, abort_flag, a.timeout_ns,
+                          kErrTimeout)) {
+        ok = false;
+        break;
+      }
+      if (j >= 2 && !ptx::mbar_wait(bar(C::B_SFREE + b), ((j - 2) >> 1) & 1, abort_flag, a.timeout_ns,
+                                    kErrTimeout)) {
+        ok = false;
+        break;
+      }
+      ptx::tc_fence_after();
+      const uint32_t s_tmem = tmem + (b ? C::TM_S1 : C::TM_S0);
+      const uint32_t k_base = sb + C::OFF_K + s * C::K_BYTES;
+#pragma unroll
+      for (int kk = 0; kk < D / 16; ++kk) {
+        const uint32_t off = (kk & 3) * 32;
+        const uint64_t adesc = ptx::sdesc_sw128(sb + C::OFF_Q + (kk >> 2) * C::Q_CHUNK + off, 16, 1024);
+        const uint64_t bdesc = ptx::sdesc_sw128(k_base + (kk >> 2) * C::KV_CHUNK + off, 16, 1024);
+        ptx::umma_ss(s_tmem, adesc, bdesc, C::IDESC_S, kk > 0 ? 1u : 0u);
+      }
+      ptx::umma_commit(bar(C::B_SFULL + b));
+      ptx::umma_commit(bar(C::B_KEMPTY + s));
+    }
+    if (!ok) {
+      ptx::umma_commit(bar(C::B_DRAIN));
+      volatile int dummy = 0;
+      ptx::mbar_wait(bar(C::B_DRAIN), 0, &dummy, a.timeout_ns / 4, 0);
+    }
+  } else if (warp >= 4) {
+    // ================================================================ reducers
+    const int wq = warp & 3;
+    const int r = wq * 32 + lane;
+    const uint32_t lane_base = tmem + (static_cast<uint32_t>(wq * 32) << 16);
+    const int grow = qi * a.bq + r;
+    const bool row_valid = (r < a.bq) && (grow < a.L);
+    const float lse2 = row_valid ? a.lse[static_cast<long>(h) * a.L + grow] * 1.44269504088896340736f : 0.f;
+    const float sl2 = a.scale_log2;
+    float* out = a.mass + (static_cast<long>(h) * a.nqb + qi) * a.nkb;
+    for (int j = 0; j < n; ++j) {
+      const int b = j & 1;
+      // after an abort every wait returns at once; the loop still runs to the
+      // end so all 128 reducers take every named barrier
+      const bool ok =
+          ptx::mbar_wait_warp(bar(C::B_SFULL + b), (j >> 1) & 1, abort_flag, a.timeout_ns, kErrTimeout);
+      float acc = 0.f;
+      if (ok) {
+        ptx::tc_fence_after();
+        const int valid = a.L - j * BK < BK ? a.L - j * BK : BK;
+        float part[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int c = 0; c < BK / 32; ++c) {
+          uint32_t raw[32];
+          ptx::tmem_ld32(lane_base + (b ? C::TM_S1 : C::TM_S0) + c * 32, raw);
+          ptx::tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 32; ++e) {
+            const float p = ptx::ex2(fmaf(__uint_as_float(raw[e]), sl2, -lse2));
+            part[e & 3] += (c * 32 + e < valid) ? p : 0.f;
+          }
+        }
+        ptx::tc_fence_before();
+        ptx::mbar_arrive(bar(C::B_SFREE + b));
+        acc = row_valid ? (part[0] + part[1]) + (part[2] + part[3]) : 0.f;
+      }
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+      if (lane == 0) red[b * 4 + wq] = acc;
+      ptx::named_bar_sync(1, 128);
+      if (r == 0 && !*abort_flag) out[j] = (red[b * 4 + 0] + red[b * 4 + 1]) + (red[b * 4 + 2] + red[b * 4 + 3]);
+    }
+  }
+
+  ptx::tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    ptx::tc_fence_after();
+    ptx::tmem_dealloc(tmem, C::TM_ALLOC);
+  }
+}
+
+// ---------------------------------------------------------------- top-k
+
+// One warp per (h, i) row (head_k: per-head k from the entropy budget, else
+// k_uniform for every head). rank(j) = #{j' : M[j'] > M[j] or (M[j'] == M[j] and
+// j' < j)}; block j is kept iff rank(j) < k_h. Kept blocks are written in
+// ascending j by warp-ballot compaction.
+__global__ void __launch_bounds__(256)
+    topk_kernel(const float* __restrict__ mass, int rows, int nqb, int nkb, int k_uniform,
+                const int32_t* __restrict__ head_k, int32_t* __restrict__ head_k_out,
+                int32_t* __restrict__ kv_idx, int32_t* __restrict__ kv_count, int kv_stride) {
+  constexpr int CH = 1024;
+  __shared__ float buf[8][CH];
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const long row = static_cast<long>(blockIdx.x) * 8 + warp;
+  if (row >= rows) return;
+  const int h = static_cast<int>(row / nqb);
+  int k = head_k ? head_k[h] : k_uniform;
+  k = k < 0 ? 0 : (k > nkb ? nkb : k);
+  if (k > kv_stride) k = kv_stride;
+  const float* m = mass + row * nkb;
+  int32_t* dst = kv_idx + row * kv_stride;
+  int written = 0;
+  for (int base = 0; base < nkb; base += 32) {
+    const int j = base + lane;
+    const float mj = j < nkb ? m[j] : 0.f;
+    int rank = 0;
+    for (int c0 = 0; c0 < nkb; c0 += CH) {
+      const int len = nkb - c0 < CH ? nkb - c0 : CH;
+      __syncwarp();
+      for (int t = lane; t < len; t += 32) buf[warp][t] = m[c0 + t];
+      __syncwarp();
+      for (int t = 0; t < len; ++t) {
+        const float x = buf[warp][t];
+        rank += (x > mj) || (x == mj && c0 + t < j);
+      }
+    }
+    const bool keep = j < nkb && rank < k;
+    const unsigned ball = __ballot_sync(0xffffffffu, keep);
+    if (keep) dst[written + __popc(ball & ((1u << lane) - 1u))] = j;
+    written += __popc(ball);
+  }
+  if (lane == 0) {
+    kv_count[row] = k;
+    if (head_k_out && row % nqb == 0) head_k_out[h] = k;  // uniform budget: export k per head
+  }
+}
+
+// ---------------------------------------------------------------- entropy budget
+
+// One warp per (h, i): z = sum_j M, entropy = -sum_j (M/z) ln(M/z) over M > 0 (fp64).
+__global__ void __launch_bounds__(256)
+    row_entropy_kernel(const float* __restrict__ mass, int rows, int nkb, double* __restrict__ ent) {
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const long row = static_cast<long>(blockIdx.x) * 8 + warp;
+  if (row >= rows) return;
+  const float* m = mass + row * nkb;
+  double z = 0.0;
+  for (int j = lane; j < nkb; j += 32) z += static_cast<double>(m[j]);
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) z += __shfl_xor_sync(0xffffffffu, z, off);
+  double e = 0.0;
+  if (z > 0.0) {
+    for (int j = lane; j < nkb; j += 32) {
+      const double x = static_cast<double>(m[j]);
+      if (x > 0.0) {
+        const double p = x / z;
+        e -= p * log(p);
+      }
+    }
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) e += __shfl_xor_sync(0xffffffffu, e, off);
+  if (lane == 0) ent[row] = e;
+}
+
+// One block. E_h = (sum_i ent[h,i]) / nqb (sequential in i). Then one thread
+// allocates B = clamp(ceil(rho*H*nkb - 1e-6), H, H*nkb): one block per head,
+// the extra B-H split in proportion to E_h (evenly if the split heads' E sum to
+// 0), shares above nkb-1 capped and the rest re-split, then largest-remainder
+// rounding with ties to the lower head. Writes k_h = 1 + extra_h.
+// scratch: 4*H doubles (entropy, share, quota, mark).
+__global__ void budget_kernel(const double* __restrict__ ent, int H, int nqb, int nkb, float keep_ratio,
+                              int32_t* __restrict__ head_k, double* __restrict__ scratch) {
+  double* E = scratch;
+  double* extra = scratch + H;      // < 0: not yet decided
+  double* quota = scratch + 2 * H;
+  double* mark = scratch + 3 * H;
+  for (int h = threadIdx.x; h < H; h += blockDim.x) {
+    double s = 0.0;
+    for (int i = 0; i < nqb; ++i) s += ent[static_cast<long>(h) * nqb + i];
+    E[h] = s / nqb;
+    extra[h] = -1.0;
+    mark[h] = 0.0;
+  }
+  __syncthreads();
+  if (threadIdx.x != 0) return;
+  const double rho = static_cast<double>(keep_ratio);
+  long B = static_cast<long>(ceil(rho * H * nkb - 1e-6));
+  if (B < H) B = H;
+  if (B > static_cast<long>(H) * nkb) B = static_cast<long>(H) * nkb;
+  const double cap = nkb - 1;
+  while (true) {
+    int nfree = 0;
+    long fixed = 0;
+    double sE = 0.0;
+    for (int h = 0; h < H; ++h) {
+      if (extra[h] < 0.0) {
+        ++nfree;
+        sE += E[h];
+      } else {
+        fixed += static_cast<long>(extra[h]);
+      }
+    }
+    if (nfree == 0) break;
+    const long Xf = (B - H) - fixed;
+    const bool prop = sE > 0.0;
+    const double sw = prop ? sE : static_cast<double>(nfree);
+    bool over = false;
+    for (int h = 0; h < H; ++h) {
+      if (extra[h] >= 0.0) continue;
+      const double w = prop ? E[h] : 1.0;
+      if (static_cast<double>(Xf) * w / sw > cap) {
+        extra[h] = cap;
+        over = true;
+      }
+    }
+    if (over) continue;
+    long assigned = 0;
+    for (int h = 0; h < H; ++h) {
+      if (extra[h] >= 0.0) {
+        quota[h] = -1.0;
+        continue;
+      }
+      const double w = prop ? E[h] : 1.0;
+      quota[h] = static_cast<double>(Xf) * w / sw;
+      extra[h] = floor(quota[h]);
+      assigned += static_cast<long>(extra[h]);
+    }
+    long rem = Xf - assigned;
+    while (rem > 0) {  // one more unit to the largest fractions, ties to the lower head
+      int best = -1;
+      double bf = -1.0;
+      for (int h = 0; h < H; ++h) {
+        if (quota[h] < 0.0 || mark[h] != 0.0) continue;
+        const double f = quota[h] - floor(quota[h]);
+        if (f > bf) { bf = f; best = h; }
+      }
+      if (best < 0) break;
+      extra[best] += 1.0;
+      mark[best] = 1.0;
+      --rem;
+    }
+    while (rem < 0) {  // only reachable through fp64 rounding of the quotas
+      int best = -1;
+      double bf = 2.0;
+      for (int h = 0; h < H; ++h) {
+        if (quota[h] < 0.0 || mark[h] != 0.0 || extra[h] <= 0.0) continue;
+        const double f = quota[h] - floor(quota[h]);
+        if (f <= bf) { bf = f; best = h; }
+      }
+      if (best < 0) break;
+      extra[best] -= 1.0;
+      mark[best] = 1.0;
+      ++rem;
+    }
+    break;
+  }
+  for (int h = 0; h < H; ++h) head_k[h] = 1 + static_cast<int32_t>(extra[h]);
+}
+
+}  // namespace sparsed

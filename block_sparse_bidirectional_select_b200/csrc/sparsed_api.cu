@@ -1,0 +1,474 @@
+// Host side of the C ABI declared in include/sparsed.h: argument validation,
+// workspace layout, TMA descriptor encoding, kernel launches and the
+// denoising-step driver. Every step of the computation runs in the kernels of
+// attn_kernel.cuh and select_kernels.cuh; nothing here computes attention.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_runtime.h>
+
+#include <atomic>
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+#include <vector>
+
+#include "sparsed.h"
+#include "attn_kernel.cuh"
+#include "select_kernels.cuh"
+
+using namespace sparsed;
+
+namespace {
+
+constexpr uint64_t kWaitTimeoutNs = 2000000000ull;  // 2 s bound on every device wait
+constexpr double kRoundEps = 1e-6;
+
+std::atomic<int> g_last_cuda{0};
+
+int fail_cuda(cudaError_t e) {
+  g_last_cuda.store(static_cast<int>(e));
+  return SPARSED_ERR_CUDA;
+}
+
+#define SP_CUDA(x)                                   \
+  do {                                               \
+    cudaError_t e_ = (x);                            \
+    if (e_ != cudaSuccess) return fail_cuda(e_);     \
+  } while (0)
+
+#define SP_TRY(x)                \
+  do {                           \
+    int rc_ = (x);               \
+    if (rc_ != SPARSED_OK) return rc_; \
+  } while (0)
+
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+std::once_flag g_encode_once;
+cudaError_t g_encode_err = cudaSuccess;
+
+int get_encoder() {
+  std::call_once(g_encode_once, [] {
+    cudaDriverEntryPointQueryResult q;
+    void* fn = nullptr;
+    g_encode_err = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q);
+    if (g_encode_err == cudaSuccess && q == cudaDriverEntryPointSuccess)
+      g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+    else if (g_encode_err == cudaSuccess)
+      g_encode_err = cudaErrorSymbolNotFound;
+  });
+  if (!g_encode) return fail_cuda(g_encode_err);
+  return SPARSED_OK;
+}
+
+int require_sm100() {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e == cudaErrorNoDevice || e == cudaErrorInsufficientDriver) {
+    g_last_cuda.store(static_cast<int>(e));
+    return SPARSED_ERR_NO_DEVICE;
+  }
+  SP_CUDA(e);
+  int major = 0, minor = 0;
+  SP_CUDA(cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev));
+  SP_CUDA(cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev));
+  if (major != 10 || minor != 0) return SPARSED_ERR_NO_DEVICE;
+  return SPARSED_OK;
+}
+
+inline long cdiv(long a, long b) { return (a + b - 1) / b; }
+inline size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int check_shapes(int H, int L, int d, float scale, int bq, int bk) {
+  if (H < 0 || L < 0) return SPARSED_ERR_INVALID_ARG;
+  if (!std::isfinite(scale)) return SPARSED_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return SPARSED_ERR_UNSUPPORTED;
+  if ((bq != 64 && bq != 128) || (bk != 64 && bk != 128)) return SPARSED_ERR_UNSUPPORTED;
+  if (H > 65535) return SPARSED_ERR_UNSUPPORTED;
+  if (static_cast<long long>(H) * L * d >= (1ll << 31)) return SPARSED_ERR_UNSUPPORTED;
+  return SPARSED_OK;
+}
+
+int check_qkvo(const void* Q, const void* K, const void* V, const void* O, const void* LSE) {
+  if (!Q || !K || !V || !O || !LSE) return SPARSED_ERR_INVALID_ARG;
+  if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O)) return SPARSED_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(LSE) & 3u) != 0) return SPARSED_ERR_INVALID_ARG;
+  return SPARSED_OK;
+}
+
+int uniform_k(int nkb, float keep) {
+  const double k = std::ceil(static_cast<double>(keep) * nkb - kRoundEps);
+  long kk = static_cast<long>(k);
+  if (kk < 1) kk = 1;
+  if (kk > nkb) kk = nkb;
+  return static_cast<int>(kk);
+}
+
+// [H, L, d] bf16 viewed as a 3-D tensor (d innermost), boxes of 64 columns x rows.
+int make_map(CUtensorMap* m, const void* ptr, int H, int L, int d, int box_rows) {
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(L),
+                        static_cast<cuuint64_t>(H)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2, static_cast<cuuint64_t>(L) * d * 2};
+  cuuint32_t box[3] = {64, static_cast<cuuint32_t>(box_rows), 1};
+  cuuint32_t es[3] = {1, 1, 1};
+  CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box,
+                        es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail_cuda(cudaErrorInvalidValue);
+  return SPARSED_OK;
+}
+
+struct Problem {
+  const uint16_t *Q, *K, *V;
+  uint16_t* O;
+  float* LSE;
+  int H, L, d, bq, bk, nqb, nkb;
+  float scale;
+};
+
+template <int D, int BK, bool SPARSE>
+int launch_attn_t(const Problem& p, const int32_t* kv_idx, const int32_t* kv_count, int kv_stride,
+                  cudaStream_t st) {
+  using C = AttnCfg<D, BK>;
+  CUtensorMap tq, tk, tv, to;
+  SP_TRY(make_map(&tq, p.Q, p.H, p.L, D, 128));
+  SP_TRY(make_map(&tk, p.K, p.H, p.L, D, BK));
+  SP_TRY(make_map(&tv, p.V, p.H, p.L, D, BK));
+  SP_TRY(make_map(&to, p.O, p.H, p.L, D, p.bq));
+  AttnArgs a;
+  a.H = p.H;
+  a.L = p.L;
+  a.bq = p.bq;
+  a.nqb = p.nqb;
+  a.nkb = p.nkb;
+  a.scale_log2 = p.scale * 1.44269504088896340736f;
+  a.kv_idx = kv_idx;
+  a.kv_count = kv_count;
+  a.kv_stride = kv_stride;
+  a.lse = p.LSE;
+  a.o = p.O;
+  a.timeout_ns = kWaitTimeoutNs;
+  auto kern = attn_fwd_kernel<D, BK, SPARSE>;
+  SP_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES));
+  kern<<<dim3(p.nqb, p.H), 256, C::SMEM_BYTES, st>>>(tq, tk, tv, to, a);
+  SP_CUDA(cudaGetLastError());
+  return SPARSED_OK;
+}
+
+int launch_attn(const Problem& p, bool sparse, const int32_t* kv_idx, const int32_t* kv_count,
+                int kv_stride, cudaStream_t st) {
+#define SP_ATTN(D_, BK_)                                                               \
+  if (p.d == D_ && p.bk == BK_)                                                        \
+    return sparse ? launch_attn_t<D_, BK_, true>(p, kv_idx, kv_count, kv_stride, st)   \
+                  : launch_attn_t<D_, BK_, false>(p, kv_idx, kv_count, kv_stride, st);
+  SP_ATTN(64, 64)
+  SP_ATTN(64, 128)
+  SP_ATTN(128, 64)
+  SP_ATTN(128, 128)
+#undef SP_ATTN
+  return SPARSED_ERR_UNSUPPORTED;
+}
+
+template <int D, int BK>
+int launch_mass_t(const Problem& p, float* mass, cudaStream_t st) {
+  using C = MassCfg<D, BK>;
+  CUtensorMap tq, tk;
+  SP_TRY(make_map(&tq, p.Q, p.H, p.L, D, 128));
+  SP_TRY(make_map(&tk, p.K, p.H, p.L, D, BK));
+  MassArgs a;
+  a.H = p.H;
+  a.L = p.L;
+  a.bq = p.bq;
+  a.nqb = p.nqb;
+  a.nkb = p.nkb;
+  a.scale_log2 = p.scale * 1.44269504088896340736f;
+  a.lse = p.LSE;
+  a.mass = mass;
+  a.timeout_ns = kWaitTimeoutNs;
+  auto kern = block_mass_kernel<D, BK>;
+  SP_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES));
+  kern<<<dim3(p.nqb, p.H), 256, C::SMEM_BYTES, st>>>(tq, tk, a);
+  SP_CUDA(cudaGetLastError());
+  return SPARSED_OK;
+}
+
+int launch_mass(const Problem& p, float* mass, cudaStream_t st) {
+  if (p.d == 64 && p.bk == 64) return launch_mass_t<64, 64>(p, mass, st);
+  if (p.d == 64 && p.bk == 128) return launch_mass_t<64, 128>(p, mass, st);
+  if (p.d == 128 && p.bk == 64) return launch_mass_t<128, 64>(p, mass, st);
+  if (p.d == 128 && p.bk == 128) return launch_mass_t<128, 128>(p, mass, st);
+  return SPARSED_ERR_UNSUPPORTED;
+}
+
+struct Workspace {
+  size_t grid, ent, scratch, headk, total;
+};
+
+Workspace ws_layout(int H, int nqb, int nkb) {
+  Workspace w;
+  w.grid = 0;
+  w.ent = w.grid + align256(static_cast<size_t>(H) * nqb * nkb * sizeof(float));
+  w.scratch = w.ent + align256(static_cast<size_t>(H) * nqb * sizeof(double));
+  w.headk = w.scratch + align256(static_cast<size_t>(H) * 4 * sizeof(double));
+  w.total = w.headk + align256(static_cast<size_t>(H) * sizeof(int32_t));
+  if (w.total == 0) w.total = 256;
+  return w;
+}
+
+// Steps 2-4 of pattern selection, after the dense pass wrote O and LSE.
+int select_after_dense(const Problem& p, float keep_ratio, int budget_mode, int32_t* kv_idx,
+                       int32_t* kv_count, int kv_stride, float* block_mass, int32_t* head_k,
+                       void* workspace, cudaStream_t st) {
+  const Workspace w = ws_layout(p.H, p.nqb, p.nkb);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  float* mass = block_mass ? block_mass : reinterpret_cast<float*>(ws + w.grid);
+  SP_TRY(launch_mass(p, mass, st));
+  const int rows = p.H * p.nqb;
+  const int kblocks = (rows + 7) / 8;
+  int32_t* hk = nullptr;
+  int k_uniform = uniform_k(p.nkb, keep_ratio);
+  if (budget_mode == SPARSED_BUDGET_ENTROPY) {
+    double* ent = reinterpret_cast<double*>(ws + w.ent);
+    double* scratch = reinterpret_cast<double*>(ws + w.scratch);
+    hk = head_k ? head_k : reinterpret_cast<int32_t*>(ws + w.headk);
+    row_entropy_kernel<<<kblocks, 256, 0, st>>>(mass, rows, p.nkb, ent);
+    SP_CUDA(cudaGetLastError());
+    budget_kernel<<<1, 256, 0, st>>>(ent, p.H, p.nqb, p.nkb, keep_ratio, hk, scratch);
+    SP_CUDA(cudaGetLastError());
+  }
+  int32_t* hk_out = (budget_mode == SPARSED_BUDGET_UNIFORM) ? head_k : nullptr;
+  topk_kernel<<<kblocks, 256, 0, st>>>(mass, rows, p.nqb, p.nkb, k_uniform, hk, hk_out, kv_idx,
+                                       kv_count, kv_stride);
+  SP_CUDA(cudaGetLastError());
+  return SPARSED_OK;
+}
+
+int prepare(const uint16_t* Q, const uint16_t* K, const uint16_t* V, int H, int L, int d, float scale,
+            int bq, int bk, uint16_t* O, float* LSE, Problem* p, bool* empty) {
+  SP_TRY(check_shapes(H, L, d, scale, bq, bk));
+  *empty = (static_cast<long>(H) * L == 0);
+  if (*empty) return SPARSED_OK;
+  SP_TRY(check_qkvo(Q, K, V, O, LSE));
+  p->Q = Q;
+  p->K = K;
+  p->V = V;
+  p->O = O;
+  p->LSE = LSE;
+  p->H = H;
+  p->L = L;
+  p->d = d;
+  p->bq = bq;
+  p->bk = bk;
+  p->nqb = static_cast<int>(cdiv(L, bq));
+  p->nkb = static_cast<int>(cdiv(L, bk));
+  p->scale = scale;
+  return SPARSED_OK;
+}
+
+int check_select_args(const Problem& p, float keep_ratio, int budget_mode, int32_t* kv_idx,
+                      int32_t* kv_count, int kv_stride, void* workspace, size_t ws_bytes) {
+  if (!(keep_ratio > 0.f && keep_ratio <= 1.f)) return SPARSED_ERR_INVALID_ARG;
+  if (budget_mode != SPARSED_BUDGET_UNIFORM && budget_mode != SPARSED_BUDGET_ENTROPY)
+    return SPARSED_ERR_INVALID_ARG;
+  if (!kv_idx || !kv_count) return SPARSED_ERR_INVALID_ARG;
+  const int need = budget_mode == SPARSED_BUDGET_UNIFORM ? uniform_k(p.nkb, keep_ratio) : p.nkb;
+  if (kv_stride < need) return SPARSED_ERR_INVALID_ARG;
+  if (static_cast<long long>(p.H) * p.nqb * kv_stride >= (1ll << 31)) return SPARSED_ERR_UNSUPPORTED;
+  if (static_cast<long long>(p.H) * p.nqb * p.nkb >= (1ll << 31)) return SPARSED_ERR_UNSUPPORTED;
+  const Workspace w = ws_layout(p.H, p.nqb, p.nkb);
+  if (!workspace || ws_bytes < w.total) return SPARSED_ERR_WORKSPACE;
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return SPARSED_ERR_WORKSPACE;
+  return SPARSED_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int sparsed_version(void) { return SPARSED_VERSION; }
+
+const char* sparsed_strerror(int status) {
+  switch (status) {
+    case SPARSED_OK: return "ok";
+    case SPARSED_ERR_INVALID_ARG: return "invalid argument (null pointer, negative size, bad value or misaligned buffer)";
+    case SPARSED_ERR_UNSUPPORTED: return "unsupported configuration (d, block size or size limit)";
+    case SPARSED_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
+    case SPARSED_ERR_BAD_PATTERN: return "block pattern entry out of range or not strictly ascending";
+    case SPARSED_ERR_CUDA: return "CUDA runtime error (see sparsed_last_cuda_error)";
+    case SPARSED_ERR_DEVICE_TIMEOUT: return "a bounded device-side wait expired";
+    case SPARSED_ERR_NO_DEVICE: return "no sm_100 (B200) device is current";
+    default: return "unknown status";
+  }
+}
+
+int sparsed_last_cuda_error(void) { return g_last_cuda.load(); }
+
+int sparsed_check(void* stream) {
+  SP_TRY(require_sm100());
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  SP_CUDA(cudaStreamSynchronize(st));
+  int code = 0;
+  SP_CUDA(cudaMemcpyFromSymbol(&code, ptx::g_device_error, sizeof(int)));
+  if (code != 0) {
+    const int zero = 0;
+    SP_CUDA(cudaMemcpyToSymbol(ptx::g_device_error, &zero, sizeof(int)));
+  }
+  return code;
+}
+
+int sparsed_uniform_keep(int L, int bk, float keep_ratio, int* k_out) {
+  if (!k_out || L <= 0 || bk <= 0) return SPARSED_ERR_INVALID_ARG;
+  if (!(keep_ratio > 0.f && keep_ratio <= 1.f)) return SPARSED_ERR_INVALID_ARG;
+  *k_out = uniform_k(static_cast<int>(cdiv(L, bk)), keep_ratio);
+  return SPARSED_OK;
+}
+
+int sparsed_schedule(int T, float warmup_frac, int refresh_every, int8_t* kinds) {
+  if (T < 0 || refresh_every < 0) return SPARSED_ERR_INVALID_ARG;
+  if (!(warmup_frac >= 0.f && warmup_frac <= 1.f)) return SPARSED_ERR_INVALID_ARG;
+  if (T == 0) return SPARSED_OK;
+  if (!kinds) return SPARSED_ERR_INVALID_ARG;
+  long n_dense = static_cast<long>(std::ceil(static_cast<double>(warmup_frac) * T - kRoundEps));
+  if (n_dense < 1) n_dense = 1;
+  if (n_dense > T) n_dense = T;
+  for (int t = 0; t < T; ++t) {
+    int8_t k;
+    if (n_dense == T || t < n_dense - 1)
+      k = SPARSED_STEP_DENSE;
+    else if (t == n_dense - 1)
+      k = SPARSED_STEP_SELECT;
+    else if (refresh_every > 0 && (t - (n_dense - 1)) % refresh_every == 0)
+      k = SPARSED_STEP_SELECT;
+    else
+      k = SPARSED_STEP_SPARSE;
+    kinds[t] = k;
+  }
+  return SPARSED_OK;
+}
+
+int sparsed_workspace_bytes(int H, int L, int bq, int bk, size_t* bytes) {
+  if (!bytes || H < 0 || L < 0) return SPARSED_ERR_INVALID_ARG;
+  if ((bq != 64 && bq != 128) || (bk != 64 && bk != 128)) return SPARSED_ERR_UNSUPPORTED;
+  *bytes = ws_layout(H, static_cast<int>(cdiv(L, bq)), static_cast<int>(cdiv(L, bk))).total;
+  return SPARSED_OK;
+}
+
+int sparsed_dense_attn(const uint16_t* Q, const uint16_t* K, const uint16_t* V, int H, int L, int d,
+                       float scale, int bq, int bk, uint16_t* O, float* LSE, void* stream) {
+  Problem p;
+  bool empty = false;
+  SP_TRY(prepare(Q, K, V, H, L, d, scale, bq, bk, O, LSE, &p, &empty));
+  if (empty) return SPARSED_OK;
+  SP_TRY(require_sm100());
+  SP_TRY(get_encoder());
+  return launch_attn(p, false, nullptr, nullptr, 0, static_cast<cudaStream_t>(stream));
+}
+
+int sparsed_select_pattern(const uint16_t* Q, const uint16_t* K, const uint16_t* V, int H, int L, int d,
+                           float scale, int bq, int bk, float keep_ratio, int budget_mode, uint16_t* O,
+                           float* LSE, int32_t* kv_idx, int32_t* kv_count, int kv_stride,
+                           float* block_mass, int32_t* head_k, void* workspace, size_t workspace_bytes,
+                           void* stream) {
+  Problem p;
+  bool empty = false;
+  SP_TRY(prepare(Q, K, V, H, L, d, scale, bq, bk, O, LSE, &p, &empty));
+  if (empty) return SPARSED_OK;
+  SP_TRY(check_select_args(p, keep_ratio, budget_mode, kv_idx, kv_count, kv_stride, workspace,
+                           workspace_bytes));
+  SP_TRY(require_sm100());
+  SP_TRY(get_encoder());
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  SP_TRY(launch_attn(p, false, nullptr, nullptr, 0, st));
+  return select_after_dense(p, keep_ratio, budget_mode, kv_idx, kv_count, kv_stride, block_mass, head_k,
+                            workspace, st);
+}
+
+int sparsed_block_sparse_attn(const uint16_t* Q, const uint16_t* K, const uint16_t* V, int H, int L, int d,
+                              float scale, int bq, int bk, const int32_t* kv_idx, const int32_t* kv_count,
+                              int kv_stride, uint16_t* O, float* LSE, void* stream) {
+  Problem p;
+  bool empty = false;
+  SP_TRY(prepare(Q, K, V, H, L, d, scale, bq, bk, O, LSE, &p, &empty));
+  if (empty) return SPARSED_OK;
+  if (!kv_idx || !kv_count || kv_stride < 1) return SPARSED_ERR_INVALID_ARG;
+  if (static_cast<long long>(p.H) * p.nqb * kv_stride >= (1ll << 31)) return SPARSED_ERR_UNSUPPORTED;
+  SP_TRY(require_sm100());
+  SP_TRY(get_encoder());
+  return launch_attn(p, true, kv_idx, kv_count, kv_stride, static_cast<cudaStream_t>(stream));
+}
+
+int sparsed_run_steps(const uint16_t* Q, const uint16_t* K, const uint16_t* V, int H, int L, int d,
+                      float scale, int bq, int bk, float keep_ratio, int budget_mode, int T,
+                      float warmup_frac, int refresh_every, int start_step, int have_pattern,
+                      int32_t* kv_idx, int32_t* kv_count, int kv_stride, uint16_t* O, float* LSE,
+                      int8_t* step_kind, float* step_ms, void* workspace, size_t workspace_bytes,
+                      void* stream) {
+  if (T < 0 || start_step < 0 || start_step > T) return SPARSED_ERR_INVALID_ARG;
+  std::vector<int8_t> kinds(static_cast<size_t>(T) + 1);
+  SP_TRY(sparsed_schedule(T, warmup_frac, refresh_every, kinds.data()));
+  if (step_kind && T > 0) std::memcpy(step_kind, kinds.data(), static_cast<size_t>(T));
+  if (step_ms)
+    for (int t = 0; t < T; ++t) step_ms[t] = 0.f;
+  Problem p;
+  bool empty = false;
+  SP_TRY(prepare(Q, K, V, H, L, d, scale, bq, bk, O, LSE, &p, &empty));
+  if (empty) return SPARSED_OK;
+  bool any_select = false, pattern_ready = have_pattern != 0;
+  for (int t = start_step; t < T; ++t) {
+    if (kinds[t] == SPARSED_STEP_SELECT) pattern_ready = any_select = true;
+    if (kinds[t] == SPARSED_STEP_SPARSE && !pattern_ready) return SPARSED_ERR_INVALID_ARG;
+  }
+  if (any_select)
+    SP_TRY(check_select_args(p, keep_ratio, budget_mode, kv_idx, kv_count, kv_stride, workspace,
+                             workspace_bytes));
+  else if (start_step < T && pattern_ready && (!kv_idx || !kv_count || kv_stride < 1))
+    return SPARSED_ERR_INVALID_ARG;
+  SP_TRY(require_sm100());
+  SP_TRY(get_encoder());
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  std::vector<cudaEvent_t> ev;
+  if (step_ms && start_step < T) {
+    ev.resize(static_cast<size_t>(T - start_step) + 1, nullptr);
+    for (auto& e : ev) SP_CUDA(cudaEventCreate(&e));
+    SP_CUDA(cudaEventRecord(ev[0], st));
+  }
+  int rc = SPARSED_OK;
+  for (int t = start_step; t < T && rc == SPARSED_OK; ++t) {
+    switch (kinds[t]) {
+      case SPARSED_STEP_DENSE:
+        rc = launch_attn(p, false, nullptr, nullptr, 0, st);
+        break;
+      case SPARSED_STEP_SELECT:
+        rc = launch_attn(p, false, nullptr, nullptr, 0, st);
+        if (rc == SPARSED_OK)
+          rc = select_after_dense(p, keep_ratio, budget_mode, kv_idx, kv_count, kv_stride, nullptr,
+                                  nullptr, workspace, st);
+        break;
+      default:
+        rc = launch_attn(p, true, kv_idx, kv_count, kv_stride, st);
+        break;
+    }
+    if (!ev.empty() && rc == SPARSED_OK) {
+      cudaError_t e = cudaEventRecord(ev[t - start_step + 1], st);
+      if (e != cudaSuccess) rc = fail_cuda(e);
+    }
+  }
+  if (!ev.empty()) {
+    if (rc == SPARSED_OK) {
+      cudaError_t e = cudaEventSynchronize(ev.back());
+      if (e != cudaSuccess) rc = fail_cuda(e);
+      for (int t = start_step; t < T && rc == SPARSED_OK; ++t) {
+        float ms = 0.f;
+        e = cudaEventElapsedTime(&ms, ev[t - start_step], ev[t - start_step + 1]);
+        if (e != cudaSuccess) rc = fail_cuda(e);
+        step_ms[t] = ms;
+      }
+    }
+    for (auto& e : ev)
+      if (e) cudaEventDestroy(e);
+  }
+  return rc;
+}
+
+}  // extern "C"

@@ -1,0 +1,191 @@
+/*
+ * sparsed.h -- C ABI of the block-sparse bidirectional attention library
+ * (libsparsed.so, built for NVIDIA B200 / sm_100a only).
+ *
+ * What it computes. Multi-head bidirectional (non-causal) attention of a
+ * diffusion language model across its denoising steps, in three parts:
+ *   - dense attention for the early steps
+ *     (SparseD: Sparse Attention for Diffusion Language Models, abstract:
+ *      full attention in the early steps, which are critical for generation);
+ *   - a head-specific block-sparse pattern selected from one full-attention
+ *     pass and reused at later steps
+ *     (SparseD abstract: patterns differ across heads and stay similar across
+ *      steps, so they are pre-computed once and reused; Step-dLLM: Adaptive
+ *      Step-aware Sparse Attention for Efficient Diffusion LLM Inference,
+ *      abstract: the block-sparse mask is refreshed at anchor steps and the
+ *      sparsity budget may be head-adaptive);
+ *   - block-sparse attention that visits only the kept key blocks
+ *     (Step-dLLM abstract: block-sparse attention kernel; PulseCol abstract:
+ *      block-sparse computation in the later iterations).
+ *
+ * Conventions shared by every entry point
+ *   Layout    Q, K, V, O are [H, L, d] bf16 (raw 16-bit patterns), row-major,
+ *             d contiguous, one contiguous buffer each. LSE is [H, L] fp32,
+ *             natural log of the softmax denominator of each query row.
+ *             Query block i covers rows [i*bq, min((i+1)*bq, L)); key block j
+ *             covers keys [j*bk, min((j+1)*bk, L)); nqb = ceil(L/bq),
+ *             nkb = ceil(L/bk). L need not be a multiple of the block sizes.
+ *   Pattern   kv_idx is [H, nqb, kv_stride] int32, kv_count is [H, nqb] int32:
+ *             the kept key blocks of (head h, query block i) are
+ *             kv_idx[(h*nqb+i)*kv_stride + 0 .. kv_count[h*nqb+i]-1], strictly
+ *             ascending, each in [0, nkb). Slots past kv_count are never read
+ *             or written.
+ *   Sizes     d in {64, 128}; bq, bk in {64, 128}; H >= 0, L >= 0 (H*L == 0 is
+ *             a no-op returning SPARSED_OK); H*L*d < 2^31.
+ *   Memory    Every array argument is DEVICE memory owned by the caller; the
+ *             library never allocates, frees or retains user memory. Q, K, V,
+ *             O must be 16-byte aligned. Scratch space comes only from a
+ *             caller-supplied workspace of the size sparsed_workspace_bytes
+ *             reports.
+ *   Streams   `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *             stream). Calls are asynchronous on that stream unless stated.
+ *   Errors    Every call returns an int status: SPARSED_OK (0) or a negative
+ *             SPARSED_ERR_* code; arguments are validated on the host before
+ *             anything is launched, and a failed validation launches nothing.
+ *             Faults found on the device (a bad pattern entry, a bounded wait
+ *             that expired) are recorded in a device error word and returned
+ *             by the next sparsed_check(). No kernel traps or hangs on bad
+ *             input: every device-side wait is bounded.
+ */
+#ifndef SPARSED_H
+#define SPARSED_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define SPARSED_VERSION 100 /* major*10000 + minor*100 + patch: 0.1.0 */
+
+enum {
+  SPARSED_OK = 0,
+  SPARSED_ERR_INVALID_ARG = -1,    /* null pointer, negative size, misaligned buffer */
+  SPARSED_ERR_UNSUPPORTED = -2,    /* d, bq or bk outside the supported set, size limits */
+  SPARSED_ERR_WORKSPACE = -3,      /* workspace missing or smaller than required */
+  SPARSED_ERR_BAD_PATTERN = -4,    /* a pattern entry out of range / not ascending (device) */
+  SPARSED_ERR_CUDA = -5,           /* a CUDA runtime call failed; see sparsed_last_cuda_error */
+  SPARSED_ERR_DEVICE_TIMEOUT = -6, /* a bounded device-side wait expired */
+  SPARSED_ERR_NO_DEVICE = -7       /* no sm_100 device is current */
+};
+
+enum { SPARSED_BUDGET_UNIFORM = 0, SPARSED_BUDGET_ENTROPY = 1 };
+enum { SPARSED_STEP_DENSE = 0, SPARSED_STEP_SELECT = 1, SPARSED_STEP_SPARSE = 2 };
+
+/* Library version (SPARSED_VERSION of the build). Never fails. */
+int sparsed_version(void);
+
+/* Static message for a status code; never NULL. */
+const char* sparsed_strerror(int status);
+
+/* The cudaError_t of the last runtime failure mapped to SPARSED_ERR_CUDA
+ * (0 if none). Host-side, thread-shared, not reset by successful calls. */
+int sparsed_last_cuda_error(void);
+
+/* Synchronises `stream`, then returns and clears the device error word: the
+ * first device-side fault recorded since the previous check
+ * (SPARSED_ERR_BAD_PATTERN or SPARSED_ERR_DEVICE_TIMEOUT), else SPARSED_OK. */
+int sparsed_check(void* stream);
+
+/* Host-only. Kept key blocks per query block under the uniform budget:
+ * k = clamp(ceil(keep_ratio * nkb - 1e-6), 1, nkb), nkb = ceil(L/bk)
+ * (Step-dLLM abstract: a uniform budget across heads; "90% sparsity" keeps
+ * 0.10). keep_ratio must be in (0, 1]. */
+int sparsed_uniform_keep(int L, int bk, float keep_ratio, int* k_out);
+
+/* Host-only. Step kinds of a T-step denoising run, written to kinds[0..T-1]
+ * (host memory) as SPARSED_STEP_*: with n_dense = clamp(ceil(w*T - 1e-6), 1, T),
+ * steps t < n_dense-1 are DENSE, t = n_dense-1 is SELECT, and a later step is
+ * SELECT when refresh_every > 0 and (t - (n_dense-1)) % refresh_every == 0,
+ * else SPARSE; if n_dense == T every step is DENSE (SparseD abstract: full
+ * attention early, pattern computed once and reused; Step-dLLM abstract:
+ * refresh at anchor steps). warmup_frac in [0, 1], refresh_every >= 0. */
+int sparsed_schedule(int T, float warmup_frac, int refresh_every, int8_t* kinds);
+
+/* Host-only. Bytes of workspace sparsed_select_pattern and sparsed_run_steps
+ * need for these sizes (0 < result; layout is private to the library). */
+int sparsed_workspace_bytes(int H, int L, int bq, int bk, size_t* bytes);
+
+/* Dense bidirectional attention (SparseD abstract: attention over all
+ * query-key pairs; Step-dLLM abstract: the full map is recomputed at every
+ * step since bidirectional attention has no KV cache).
+ *   O[h,r,:]  = sum_c softmax_c(scale * <Q[h,r,:], K[h,c,:]>) * V[h,c,:]   (bf16)
+ *   LSE[h,r]  = ln sum_c exp(scale * <Q[h,r,:], K[h,c,:]>)                  (fp32)
+ * Products and the softmax run in fp32 on bf16 tensor cores; P is rounded to
+ * bf16 before the PV product. bq/bk are the tile sizes (results agree across
+ * tile sizes to rounding; sparsed_block_sparse_attn with every block kept and
+ * the same bk is bitwise equal). */
+int sparsed_dense_attn(const uint16_t* Q, const uint16_t* K, const uint16_t* V,
+                       int H, int L, int d, float scale, int bq, int bk,
+                       uint16_t* O, float* LSE, void* stream);
+
+/* One full-attention pass that also selects the block-sparse pattern
+ * (SparseD abstract: head-specific patterns from full attention; Step-dLLM
+ * abstract: block-sparse mask, uniform or head-adaptive budget).
+ *   1. O, LSE as sparsed_dense_attn (this pass's output is the step's output).
+ *   2. block mass M[h,i,j] = sum over rows r of query block i and keys c of key
+ *      block j of exp(scale*<q_r,k_c> - LSE[h,r]), from fp32 scores
+ *      (written to block_mass [H,nqb,nkb] fp32 when non-NULL).
+ *   3. per-head budget k_h: UNIFORM: sparsed_uniform_keep for every head.
+ *      ENTROPY: E_h = mean over i of the entropy of M[h,i,:]/sum_j M[h,i,j];
+ *      B = clamp(ceil(keep_ratio*H*nkb - 1e-6), H, H*nkb); each head keeps one
+ *      block and the extra B-H is split in proportion to E_h (evenly if the
+ *      split heads' entropies sum to 0), capping a head at nkb and re-splitting
+ *      its overflow, then rounded by largest remainder (ties to the lower head);
+ *      sum_h k_h = B. Written to head_k [H] int32 when non-NULL.
+ *   4. per (h, i): the k_h blocks of largest M[h,i,:] (ties to the lower block
+ *      index), written ascending to kv_idx, and kv_count[h*nqb+i] = k_h.
+ * kv_stride >= k (UNIFORM) or >= nkb (ENTROPY). workspace: device memory of at
+ * least sparsed_workspace_bytes(H, L, bq, bk) bytes, 256-byte aligned, owned by
+ * the caller; contents on entry are ignored. */
+int sparsed_select_pattern(const uint16_t* Q, const uint16_t* K, const uint16_t* V,
+                           int H, int L, int d, float scale, int bq, int bk,
+                           float keep_ratio, int budget_mode,
+                           uint16_t* O, float* LSE,
+                           int32_t* kv_idx, int32_t* kv_count, int kv_stride,
+                           float* block_mass, int32_t* head_k,
+                           void* workspace, size_t workspace_bytes, void* stream);
+
+/* Block-sparse attention over a cached pattern (Step-dLLM abstract: the mask
+ * is reused within each interval; SparseD abstract: the precomputed pattern is
+ * reused at all later steps). For each row r of query block i of head h, the
+ * softmax runs over the keys of blocks kv_idx[h,i,0..kv_count[h,i]-1] only:
+ *   O[h,r,:] = sum over kept keys c of softmax(scale*<q_r,k_c>) v_c  (bf16)
+ *   LSE[h,r] = ln sum over kept keys of exp(scale*<q_r,k_c>)          (fp32)
+ * kv_count 0 gives O = 0 and LSE = -inf for that block's rows. A pattern entry
+ * out of range or out of order is clamped (no out-of-bounds access) and
+ * reported as SPARSED_ERR_BAD_PATTERN by the next sparsed_check. */
+int sparsed_block_sparse_attn(const uint16_t* Q, const uint16_t* K, const uint16_t* V,
+                              int H, int L, int d, float scale, int bq, int bk,
+                              const int32_t* kv_idx, const int32_t* kv_count, int kv_stride,
+                              uint16_t* O, float* LSE, void* stream);
+
+/* The denoising loop for one attention layer with fixed inputs: steps
+ * t = start_step .. T-1 run the kind sparsed_schedule(T, warmup_frac,
+ * refresh_every) gives -- DENSE: sparsed_dense_attn; SELECT:
+ * sparsed_select_pattern into kv_idx/kv_count (the pattern cache, caller
+ * memory); SPARSE: sparsed_block_sparse_attn with the cached pattern.
+ * O and LSE hold the last step's output. have_pattern != 0 means kv_idx/
+ * kv_count already hold a pattern (resume after the switch); a SPARSE step
+ * with no pattern yet is SPARSED_ERR_INVALID_ARG (checked before launching).
+ * step_kind (nullable, HOST [T] int8) receives the kinds of all T steps.
+ * step_ms (nullable, HOST [T] fp32) receives each executed step's device time
+ * in ms from CUDA events (0 for skipped steps); when given, the call
+ * synchronises the stream before returning. workspace as in
+ * sparsed_select_pattern. */
+int sparsed_run_steps(const uint16_t* Q, const uint16_t* K, const uint16_t* V,
+                      int H, int L, int d, float scale, int bq, int bk,
+                      float keep_ratio, int budget_mode,
+                      int T, float warmup_frac, int refresh_every,
+                      int start_step, int have_pattern,
+                      int32_t* kv_idx, int32_t* kv_count, int kv_stride,
+                      uint16_t* O, float* LSE,
+                      int8_t* step_kind, float* step_ms,
+                      void* workspace, size_t workspace_bytes, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SPARSED_H */

@@ -178,9 +178,17 @@ def largest_remainder(total, weights):
     quota = [total * x / sw for x in w]
     base = [math.floor(x) for x in quota]
     rem = total - sum(base)
-    order = sorted(range(len(w)), key=lambda a: (-(quota[a] - base[a]), a))
-    for a in order[:rem]:
-        base[a] += 1
+    if rem >= 0:
+        order = sorted(range(len(w)), key=lambda a: (-(quota[a] - base[a]), a))
+        for a in order[:rem]:
+            base[a] += 1
+    else:
+        # only reachable when fp64 rounding pushes a quota across an integer:
+        # take units back from the smallest fractions (ties: higher position)
+        order = sorted((a for a in range(len(w)) if base[a] > 0),
+                       key=lambda a: (quota[a] - base[a], -a))
+        for a in order[:-rem]:
+            base[a] -= 1
     return base, quota
 
 

@@ -1,0 +1,163 @@
+"""The C ABI without a GPU: the library loads, exports every symbol the header
+declares, and its host-side logic (argument validation, budgets, schedule,
+workspace sizing) behaves as documented. No compute call reaches a device."""
+import ctypes
+import os
+import re
+
+import pytest
+import torch
+
+import oracle as O
+import block_sparse_bidirectional_select_b200 as sp
+from block_sparse_bidirectional_select_b200 import _lib
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include", "sparsed.h")
+lib = _lib.load()
+GPU = torch.cuda.is_available()
+P = ctypes.c_void_p(0x10000)          # aligned, never dereferenced by these calls
+MIS = ctypes.c_void_p(0x10008)        # 8-byte aligned only
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(sparsed_\w+)\s*\(", text)))
+
+
+def test_header_symbols_exported():
+    names = declared_functions()
+    assert len(names) >= 10
+    for n in names:
+        assert hasattr(lib, n), f"{n} declared in sparsed.h but not exported"
+    assert set(names) == set(_lib.SIGNATURES)
+
+
+def test_version_and_strerror():
+    assert sp.version() == 100
+    for code in range(-7, 1):
+        msg = lib.sparsed_strerror(code)
+        assert msg and len(msg) > 1
+    assert lib.sparsed_strerror(-99) == b"unknown status"
+
+
+@pytest.mark.parametrize("L,bk", [(8192, 128), (65536, 128), (1000, 64), (1, 128), (130, 64)])
+def test_uniform_keep_matches_oracle(L, bk):
+    nkb = -(-L // bk)
+    for keep in (0.01, 0.1, 0.15, 0.25, 0.3333, 0.5, 0.999, 1.0):
+        assert sp.uniform_keep(L, bk, keep) == O.uniform_keep(nkb, keep)
+
+
+def test_uniform_keep_rejects():
+    k = ctypes.c_int()
+    assert lib.sparsed_uniform_keep(100, 64, 0.0, ctypes.byref(k)) == _lib.ERR_INVALID_ARG
+    assert lib.sparsed_uniform_keep(100, 64, 1.5, ctypes.byref(k)) == _lib.ERR_INVALID_ARG
+    assert lib.sparsed_uniform_keep(0, 64, 0.5, ctypes.byref(k)) == _lib.ERR_INVALID_ARG
+
+
+def test_schedule_matches_oracle():
+    for T in (1, 2, 3, 5, 17, 256, 512, 1024):
+        for w in (0.0, 0.1, 0.2, 0.34, 0.5, 0.99, 1.0):
+            for R in (0, 1, 3, 64):
+                assert sp.schedule(T, w, R) == O.schedule(T, w, R), (T, w, R)
+
+
+def test_schedule_rejects():
+    buf = (ctypes.c_int8 * 4)()
+    assert lib.sparsed_schedule(4, 1.5, 0, ctypes.cast(buf, ctypes.c_void_p)) == _lib.ERR_INVALID_ARG
+    assert lib.sparsed_schedule(4, 0.5, -1, ctypes.cast(buf, ctypes.c_void_p)) == _lib.ERR_INVALID_ARG
+    assert lib.sparsed_schedule(4, 0.5, 0, None) == _lib.ERR_INVALID_ARG
+    assert lib.sparsed_schedule(0, 0.5, 0, None) == _lib.OK
+
+
+def test_workspace_bytes():
+    a = sp.workspace_bytes(32, 8192)
+    b = sp.workspace_bytes(32, 65536)
+    assert 0 < a < b
+    assert a % 256 == 0
+    # grid alone is H * nqb * nkb floats
+    assert b >= 32 * 512 * 512 * 4
+    n = ctypes.c_size_t()
+    assert lib.sparsed_workspace_bytes(4, 100, 96, 64, ctypes.byref(n)) == _lib.ERR_UNSUPPORTED
+
+
+def _dense(Q=P, K=P, V=P, H=2, L=256, d=128, scale=0.088, bq=128, bk=128, O_=P, LSE=P):
+    return lib.sparsed_dense_attn(Q, K, V, H, L, d, scale, bq, bk, O_, LSE, None)
+
+
+def test_dense_validation_before_any_launch():
+    assert _dense(d=96) == _lib.ERR_UNSUPPORTED
+    assert _dense(bq=32) == _lib.ERR_UNSUPPORTED
+    assert _dense(bk=256) == _lib.ERR_UNSUPPORTED
+    assert _dense(H=-1) == _lib.ERR_INVALID_ARG
+    assert _dense(Q=None) == _lib.ERR_INVALID_ARG
+    assert _dense(LSE=None) == _lib.ERR_INVALID_ARG
+    assert _dense(K=MIS) == _lib.ERR_INVALID_ARG
+    assert _dense(scale=float("nan")) == _lib.ERR_INVALID_ARG
+    assert _dense(H=70000) == _lib.ERR_UNSUPPORTED
+    assert _dense(H=64, L=1 << 20) == _lib.ERR_UNSUPPORTED   # H*L*d >= 2^31
+    # empty problems are no-ops even with null pointers
+    assert _dense(Q=None, K=None, V=None, O_=None, LSE=None, H=0) == _lib.OK
+    assert _dense(Q=None, K=None, V=None, O_=None, LSE=None, L=0) == _lib.OK
+
+
+@pytest.mark.skipif(GPU, reason="checks the no-device path")
+def test_valid_call_without_device_reports_no_device():
+    assert _dense() == _lib.ERR_NO_DEVICE
+    assert lib.sparsed_check(None) == _lib.ERR_NO_DEVICE
+
+
+def _select(keep=0.1, mode=0, stride=7, ws=P, ws_bytes=1 << 30, idx=P, cnt=P, L=8192):
+    return lib.sparsed_select_pattern(P, P, P, 2, L, 128, 0.088, 128, 128, keep, mode, P, P, idx, cnt,
+                                      stride, None, None, ws, ws_bytes, None)
+
+
+def test_select_validation():
+    assert _select(keep=0.0) == _lib.ERR_INVALID_ARG
+    assert _select(keep=1.01) == _lib.ERR_INVALID_ARG
+    assert _select(mode=2) == _lib.ERR_INVALID_ARG
+    assert _select(stride=6) == _lib.ERR_INVALID_ARG          # k = 7 at keep 0.1, nkb 64
+    assert _select(mode=1, stride=63) == _lib.ERR_INVALID_ARG  # entropy needs nkb
+    assert _select(idx=None) == _lib.ERR_INVALID_ARG
+    assert _select(ws=None) == _lib.ERR_WORKSPACE
+    assert _select(ws_bytes=1024) == _lib.ERR_WORKSPACE
+    assert _select(ws=ctypes.c_void_p(0x10010)) == _lib.ERR_WORKSPACE  # not 256-aligned
+    if not GPU:
+        assert _select() == _lib.ERR_NO_DEVICE
+
+
+def test_block_sparse_validation():
+    f = lib.sparsed_block_sparse_attn
+    assert f(P, P, P, 2, 256, 128, 0.1, 128, 128, None, P, 4, P, P, None) == _lib.ERR_INVALID_ARG
+    assert f(P, P, P, 2, 256, 128, 0.1, 128, 128, P, P, 0, P, P, None) == _lib.ERR_INVALID_ARG
+    assert f(P, P, P, 2, 256, 80, 0.1, 128, 128, P, P, 4, P, P, None) == _lib.ERR_UNSUPPORTED
+
+
+def test_run_steps_validation():
+    f = lib.sparsed_run_steps
+    args = [P, P, P, 2, 512, 128, 0.088, 128, 128, 0.5, 0, 10, 0.2, 0, 0, 0, P, P, 2, P, P, None, None,
+            P, 1 << 20, None]
+    a = list(args)
+    a[14] = 11                      # start_step > T
+    assert f(*a) == _lib.ERR_INVALID_ARG
+    a = list(args)
+    a[14] = 5                       # resume after the switch without a pattern
+    assert f(*a) == _lib.ERR_INVALID_ARG
+    a = list(args)
+    a[23] = None                    # a SELECT step needs a workspace
+    assert f(*a) == _lib.ERR_WORKSPACE
+    kinds = (ctypes.c_int8 * 10)()
+    a = list(args)
+    a[5] = 96                       # unsupported d: the kinds are still reported
+    a[21] = ctypes.cast(kinds, ctypes.c_void_p)
+    assert f(*a) == _lib.ERR_UNSUPPORTED
+    assert list(kinds) == O.schedule(10, 0.2, 0)
+
+
+def test_python_binding_type_checks():
+    q = torch.zeros((1, 64, 64), dtype=torch.float32)
+    with pytest.raises(TypeError):
+        sp.dense_attn(q, q, q)
+    q = torch.zeros((1, 64, 64), dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        sp.dense_attn(q, q, q)
