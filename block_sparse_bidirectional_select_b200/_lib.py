@@ -42,6 +42,8 @@ SIGNATURES = {
     "sparsed_select_pattern": (_I, [_P, _P, _P, _I, _I, _I, _F, _I, _I, _F, _I, _P, _P, _P, _P, _I,
                                     _P, _P, _P, _SZ, _P]),
     "sparsed_block_sparse_attn": (_I, [_P, _P, _P, _I, _I, _I, _F, _I, _I, _P, _P, _I, _P, _P, _P]),
+    "sparsed_select_pattern_noalloc": (_I, [_P, _P, _P, _I, _I, _I, _F, _I, _I, _F, _I, _P, _P, _P, _P,
+                                            _I, _P, _P, _P]),
     "sparsed_run_steps": (_I, [_P, _P, _P, _I, _I, _I, _F, _I, _I, _F, _I, _I, _F, _I, _I, _I, _P, _P,
                                _I, _P, _P, _P, _P, _P, _SZ, _P]),
 }

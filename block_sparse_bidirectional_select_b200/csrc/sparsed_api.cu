@@ -472,3 +472,72 @@ int sparsed_run_steps(const uint16_t* Q, const uint16_t* K, const uint16_t* V, i
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Allocation-free pattern selection.
+//
+// Some callers may not allocate device memory at all: code that runs inside a
+// host framework which owns the whole device-memory budget through its own pool
+// (a foreign cudaMalloc would bypass its accounting), or latency-critical loops
+// where cudaMalloc/cudaFree would implicitly synchronise the device. For them,
+// sparsed_select_pattern_noalloc takes no workspace: its scratch (block-mass
+// grid, row entropies, budget scratch, per-head k) lives in the fixed-size
+// array below, which every GPU that loads this library holds until exit.
+//
+// The array is shared by every call on a device and keeps the previous call's
+// contents. Each call writes every scratch byte it later reads before reading
+// it, so nothing has to be cleared between calls. Calls that overlap on the
+// GPU (different streams, or several host threads) race on the array.
+// ---------------------------------------------------------------------------
+
+static __device__ __align__(256) unsigned char g_noalloc_scratch[SPARSED_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+
+constexpr int kNoAllocMaxDevices = 64;
+std::mutex g_noalloc_mu;
+void* g_noalloc_addr[kNoAllocMaxDevices] = {};
+
+// Device address of g_noalloc_scratch on the current device. In host code the
+// array's name is only a host-side stand-in, so the address is resolved with
+// cudaGetSymbolAddress once per device (the first call on that device) and
+// cached.
+int noalloc_scratch_address(void** out) {
+  int dev = 0;
+  SP_CUDA(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= kNoAllocMaxDevices) return SPARSED_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (g_noalloc_addr[dev] == nullptr) {
+    void* addr = nullptr;
+    SP_CUDA(cudaGetSymbolAddress(&addr, g_noalloc_scratch));
+    g_noalloc_addr[dev] = addr;
+  }
+  *out = g_noalloc_addr[dev];
+  return SPARSED_OK;
+}
+
+}  // namespace
+
+extern "C" int sparsed_select_pattern_noalloc(const uint16_t* Q, const uint16_t* K, const uint16_t* V,
+                                              int H, int L, int d, float scale, int bq, int bk,
+                                              float keep_ratio, int budget_mode, uint16_t* O, float* LSE,
+                                              int32_t* kv_idx, int32_t* kv_count, int kv_stride,
+                                              float* block_mass, int32_t* head_k, void* stream) {
+  Problem p;
+  bool empty = false;
+  SP_TRY(prepare(Q, K, V, H, L, d, scale, bq, bk, O, LSE, &p, &empty));
+  if (empty) return SPARSED_OK;
+  // The whole scratch layout of these sizes must fit in the built-in array.
+  if (ws_layout(p.H, p.nqb, p.nkb).total > static_cast<size_t>(SPARSED_NOALLOC_SCRATCH_BYTES))
+    return SPARSED_ERR_WORKSPACE;
+  SP_TRY(require_sm100());
+  void* scratch = nullptr;
+  SP_TRY(noalloc_scratch_address(&scratch));
+  SP_TRY(check_select_args(p, keep_ratio, budget_mode, kv_idx, kv_count, kv_stride, scratch,
+                           static_cast<size_t>(SPARSED_NOALLOC_SCRATCH_BYTES)));
+  SP_TRY(get_encoder());
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  SP_TRY(launch_attn(p, false, nullptr, nullptr, 0, st));
+  return select_after_dense(p, keep_ratio, budget_mode, kv_idx, kv_count, kv_stride, block_mass, head_k,
+                            scratch, st);
+}

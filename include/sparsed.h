@@ -184,6 +184,38 @@ int sparsed_run_steps(const uint16_t* Q, const uint16_t* K, const uint16_t* V,
                       int8_t* step_kind, float* step_ms,
                       void* workspace, size_t workspace_bytes, void* stream);
 
+/* Bytes of the library's built-in scratch array used by
+ * sparsed_select_pattern_noalloc (16 MiB, held by every GPU that loads the
+ * library until the process exits). */
+#define SPARSED_NOALLOC_SCRATCH_BYTES (16u << 20)
+
+/* sparsed_select_pattern without a workspace, for callers that may not
+ * allocate device memory -- for example code running inside a host framework
+ * that owns the whole device-memory budget through its own pool, or
+ * latency-critical loops where cudaMalloc/cudaFree would implicitly
+ * synchronise the device. The pages describe no such entry point; it has no
+ * counterpart there. Arguments, outputs and results are those of
+ * sparsed_select_pattern (the caller still passes every input and output);
+ * the scratch comes from a fixed array inside the library instead of a
+ * workspace, and no cudaMalloc, cudaFree or other allocating routine is called.
+ *   - Returns SPARSED_ERR_WORKSPACE, launching nothing, when these sizes need
+ *     more than SPARSED_NOALLOC_SCRATCH_BYTES of scratch
+ *     (sparsed_workspace_bytes(H, L, bq, bk) > SPARSED_NOALLOC_SCRATCH_BYTES;
+ *     e.g. H=32, L=32768, bq=bk=128 fits, L=65536 does not).
+ *   - The first call on each device looks up the array's device address
+ *     (cudaGetSymbolAddress) with that device current and caches it; make that
+ *     first call before any stream capture.
+ *   - Every call on a device shares the one array, which keeps the previous
+ *     call's contents; each call overwrites all scratch it reads, so nothing
+ *     needs clearing. Calls that overlap on the GPU race on the array: issue
+ *     them on one stream (or otherwise order them). */
+int sparsed_select_pattern_noalloc(const uint16_t* Q, const uint16_t* K, const uint16_t* V,
+                                   int H, int L, int d, float scale, int bq, int bk,
+                                   float keep_ratio, int budget_mode,
+                                   uint16_t* O, float* LSE,
+                                   int32_t* kv_idx, int32_t* kv_count, int kv_stride,
+                                   float* block_mass, int32_t* head_k, void* stream);
+
 #ifdef __cplusplus
 }
 #endif
