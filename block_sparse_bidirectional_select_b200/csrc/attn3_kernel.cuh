@@ -1,0 +1,495 @@
+// Flash-style bidirectional attention for sm_100a, dense or block-sparse.
+//
+// One CTA computes one (head h, query block i) tile of up to 128 rows:
+//   O = softmax(scale * Q_i K^T) V over the key blocks of its list, and the
+//   fp32 natural-log LSE of every row.
+// Dense mode walks key blocks 0..nkb-1 (SparseD abstract: full attention in the
+// early denoising steps; Step-dLLM abstract: the full map is recomputed at every
+// step). Sparse mode walks kv_idx[h,i,0..kv_count) (Step-dLLM abstract:
+// block-sparse attention over a reused mask). Both modes share every line of
+// the arithmetic, so a sparse call that keeps every block in ascending order is
+// bitwise equal to the dense call.
+//
+// Warp roles (384 threads):
+//   warps 0-3   softmax, columns [0, BK/2) of every S tile (thread r: row r)
+//   warps 4-7   softmax, columns [BK/2, BK)
+//   warp 8      TMA producer: Q once, then K_j / V_j into KS- and VS-deep rings
+//   warp 9      TMEM owner; its lane 0 issues the S = Q K^T MMAs
+//   warp 10     lane 0 issues the O += P V MMAs
+//   warp 11     idle (donates its registers)
+// TMEM (128 lanes): [S0 | S1 | O | P0 | P1] = 2*BK + D + BK fp32 columns. S is
+// double-buffered, so S(j+1) is computed while the softmax works on S(j); P has
+// its own two buffers, so the two issuers never touch the same columns and can
+// run independently (a commit from one thread tracks only its own MMAs):
+//   S issuer : S_b(j) after the softmax released S_b(j-2)        (SFREE)
+//   softmax  : reads S_b(j), exchanges the half-row maxima, writes P_b(j) after
+//              PV(j-2) released P_b                              (PVDONE)
+//   PV issuer: O += P_b(j) V_j                                   (PFULL)
+// Both softmax halves of a row compute the same row max, so the lazy rescale
+// (O and the running sum keep a stale max until a row's max grows by more than
+// 2^8) takes the same decision in both; each half rescales its half of O.
+// Every wait is bounded; the in-loop exchange uses an mbarrier (bounded), never
+// a named barrier, so a timed-out warp cannot strand the others.
+#pragma once
+
+#include "ptx_sm100.cuh"
+
+namespace sparsed {
+
+struct AttnArgs {
+  int H, L, bq, nqb, nkb;
+  float scale_log2;          // scale * log2(e)
+  const int32_t* kv_idx;     // sparse mode only
+  const int32_t* kv_count;   // sparse mode only
+  int kv_stride;
+  float* lse;                // [H, L]
+  uint16_t* o;               // [H, L, D] (used only for kv_count == 0 rows)
+  uint64_t timeout_ns;       // bound of every device-side wait
+};
+
+__device__ __forceinline__ void setmaxnreg_inc_224() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 224;" ::: "memory");
+}
+__device__ __forceinline__ void setmaxnreg_dec_56() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 56;" ::: "memory");
+}
+
+template <int D, int BK>
+struct Attn3Cfg {
+  static constexpr int M = 128;
+  static constexpr int HALF = BK / 2;  // S columns per softmax thread
+  static constexpr int DCH = D / 64;
+  static constexpr int Q_CHUNK = M * 128;
+  static constexpr int KV_CHUNK = BK * 128;
+  static constexpr int Q_BYTES = M * D * 2;
+  static constexpr int KV_BYTES = BK * D * 2;
+  static constexpr int KS = 3;
+  // a third V stage when it fits next to Q, three K stages and ~4 KB of
+  // barriers / exchange buffers
+  static constexpr int VS = (Q_BYTES + 6 * KV_BYTES + 6144) <= 232448 ? 3 : 2;
+  static constexpr int OFF_Q = 0;
+  static constexpr int OFF_K = Q_BYTES;
+  static constexpr int OFF_V = OFF_K + KS * KV_BYTES;
+  static constexpr int OFF_BAR = OFF_V + VS * KV_BYTES;
+  static constexpr int B_QFULL = 0;
+  static constexpr int B_KFULL = 1;
+  static constexpr int B_KEMPTY = B_KFULL + KS;
+  static constexpr int B_VFULL = B_KEMPTY + KS;
+  static constexpr int B_VEMPTY = B_VFULL + VS;
+  static constexpr int B_SFULL = B_VEMPTY + VS;  // [2]
+  static constexpr int B_SFREE = B_SFULL + 2;    // [2] 256 arrivals
+  static constexpr int B_PFULL = B_SFREE + 2;    // [2] 256 arrivals
+  static constexpr int B_PVDONE = B_PFULL + 2;   // [2]
+  static constexpr int B_XCHG = B_PVDONE + 2;    // [2] half-row maxima exchanged (8 warps)
+  static constexpr int B_EPI = B_XCHG + 2;       // epilogue: sums exchanged / O staged (8 warps)
+  static constexpr int B_DRAIN = B_EPI + 2;      // [2] per issuer
+  static constexpr int NUM_BARS = B_DRAIN + 2;
+  static constexpr int OFF_XCHG = OFF_BAR + NUM_BARS * 8;  // float [2 bufs][2 halves][128]
+  static constexpr int OFF_LSUM = OFF_XCHG + 2 * 2 * 128 * 4;  // float [2 halves][128]
+  static constexpr int OFF_MISC = OFF_LSUM + 2 * 128 * 4;      // tmem slot, abort flag
+  static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;
+  static constexpr int TM_S0 = 0;
+  static constexpr int TM_S1 = BK;
+  static constexpr int TM_O = 2 * BK;
+  static constexpr int TM_P0 = 2 * BK + D;
+  static constexpr int TM_P1 = TM_P0 + BK / 2;
+  static constexpr int TM_USED = TM_P1 + BK / 2;
+  static constexpr int TM_ALLOC = TM_USED <= 256 ? 256 : 512;
+  static constexpr uint32_t IDESC_S = ptx::idesc_bf16_f32(128, BK, 0, 0);
+  static constexpr uint32_t IDESC_PV = ptx::idesc_bf16_f32(128, D, 0, 1);
+  static constexpr int THREADS = 384;
+  static constexpr int REGS_SOFTMAX = 224;
+  static constexpr int REGS_OTHER = 56;
+  static_assert(TM_USED <= 512, "TMEM budget");
+  static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+};
+
+// The exp pass of one half row: P = bf16(2^(s*sl2 - m)) for HALF columns into
+// TMEM at p_taddr (two columns per 32-bit cell, even column in the low half),
+// returning the fp32 sum. Column pairs go through packed fp32x2 FMA/ADD.
+template <int HALF>
+__device__ __forceinline__ float softmax_half_exp(const float (&s)[HALF], float sl2, float m, uint32_t p_taddr) {
+  const uint64_t scale2 = ptx::f32x2(sl2, sl2);
+  const uint64_t negm2 = ptx::f32x2(-m, -m);
+  uint64_t acc0 = ptx::f32x2(0.f, 0.f), acc1 = acc0;
+#pragma unroll
+  for (int c = 0; c < HALF / 64 + (HALF % 64 ? 1 : 0); ++c) {
+    constexpr int W = HALF < 64 ? HALF / 2 : 32;  // packed cells per store
+    uint32_t pk[32];
+#pragma unroll
+    for (int e = 0; e < W; ++e) {
+      const int i0 = c * 64 + 2 * e;
+      float x0, x1;
+      ptx::f32x2_split(ptx::fma_f32x2(ptx::f32x2(s[i0], s[i0 + 1]), scale2, negm2), x0, x1);
+      const float p0 = ptx::ex2(x0);
+      const float p1 = ptx::ex2(x1);
+      if (e & 1)
+        acc1 = ptx::add_f32x2(acc1, ptx::f32x2(p0, p1));
+      else
+        acc0 = ptx::add_f32x2(acc0, ptx::f32x2(p0, p1));
+      pk[e] = ptx::pack_bf16x2(p0, p1);
+    }
+    if constexpr (W == 32) {
+      ptx::tmem_st32(p_taddr + c * 32, pk);
+    } else {
+      ptx::tmem_st16(p_taddr + c * 32, pk);
+    }
+  }
+  float a0, a1, b0, b1;
+  ptx::f32x2_split(acc0, a0, a1);
+  ptx::f32x2_split(acc1, b0, b1);
+  return (a0 + b0) + (a1 + b1);
+}
+
+template <int D, int BK, bool SPARSE>
+__global__ void __launch_bounds__(384, 1)
+    attn3_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
+                     const AttnArgs a) {
+  using C = Attn3Cfg<D, BK>;
+  constexpr int HALF = C::HALF;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  const uint32_t sb = ptx::smem_u32(smem);
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int qi = blockIdx.x;
+  const int h = blockIdx.y;
+  float* xchg = reinterpret_cast<float*>(smem + C::OFF_XCHG);
+  float* lsum_x = reinterpret_cast<float*>(smem + C::OFF_LSUM);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
+  auto bar = [&](int idx) -> uint32_t { return sb + C::OFF_BAR + 8 * idx; };
+
+  // ---- work list
+  int n = a.nkb;
+  const int32_t* list = nullptr;
+  if constexpr (SPARSE) {
+    const long row = static_cast<long>(h) * a.nqb + qi;
+    n = a.kv_count[row];
+    const int cap = a.kv_stride < a.nkb ? a.kv_stride : a.nkb;
+    if (n < 0 || n > cap) {
+      if (threadIdx.x == 0) ptx::record_error(kErrBadPattern);
+      n = n < 0 ? 0 : cap;
+    }
+    list = a.kv_idx + row * a.kv_stride;
+  }
+  auto kv_block = [&](int jj) -> int {
+    if constexpr (SPARSE) {
+      const int j = list[jj];
+      return (j >= 0 && j < a.nkb) ? j : 0;
+    } else {
+      return jj;
+    }
+  };
+
+  // ---- setup
+  if (threadIdx.x == 0) {
+    ptx::mbar_init(bar(C::B_QFULL), 1);
+    for (int s = 0; s < C::KS; ++s) {
+      ptx::mbar_init(bar(C::B_KFULL + s), 1);
+      ptx::mbar_init(bar(C::B_KEMPTY + s), 1);
+    }
+    for (int s = 0; s < C::VS; ++s) {
+      ptx::mbar_init(bar(C::B_VFULL + s), 1);
+      ptx::mbar_init(bar(C::B_VEMPTY + s), 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      ptx::mbar_init(bar(C::B_SFULL + b), 1);
+      ptx::mbar_init(bar(C::B_SFREE + b), 256);
+      ptx::mbar_init(bar(C::B_PFULL + b), 256);
+      ptx::mbar_init(bar(C::B_PVDONE + b), 1);
+      ptx::mbar_init(bar(C::B_XCHG + b), 8);
+      ptx::mbar_init(bar(C::B_EPI + b), 8);
+      ptx::mbar_init(bar(C::B_DRAIN + b), 1);
+    }
+    *abort_flag = 0;
+    ptx::fence_mbar_init();
+  }
+  if (warp == 9) {
+    ptx::tmem_alloc(ptx::smem_u32(tmem_slot), C::TM_ALLOC);
+    ptx::tmem_relinquish();
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp >= 8) {
+    setmaxnreg_dec_56();
+    if (warp == 8 && lane == 0 && n > 0) {
+      // ============================================================ producer
+      ptx::tma_prefetch_desc(&tm_q);
+      ptx::tma_prefetch_desc(&tm_k);
+      ptx::tma_prefetch_desc(&tm_v);
+      ptx::mbar_arrive_expect_tx(bar(C::B_QFULL), C::Q_BYTES);
+#pragma unroll
+      for (int c = 0; c < C::DCH; ++c)
+        ptx::tma_load_3d(sb + C::OFF_Q + c * C::Q_CHUNK, &tm_q, bar(C::B_QFULL), c * 64, qi * a.bq, h);
+      int prev = -1, issued_k = 0, issued_v = 0;
+      for (int jj = 0; jj < n; ++jj) {
+        int j = jj;
+        if constexpr (SPARSE) {
+          j = list[jj];
+          if (j < 0 || j >= a.nkb || j <= prev) ptx::record_error(kErrBadPattern);
+          prev = j;
+          j = kv_block(jj);
+        }
+        const int ks = jj % C::KS;
+        if (jj >= C::KS &&
+            !ptx::mbar_wait(bar(C::B_KEMPTY + ks), (jj / C::KS - 1) & 1, abort_flag, a.timeout_ns, kErrTimeout))
+          break;
+        ptx::mbar_arrive_expect_tx(bar(C::B_KFULL + ks), C::KV_BYTES);
+#pragma unroll
+        for (int c = 0; c < C::DCH; ++c)
+          ptx::tma_load_3d(sb + C::OFF_K + ks * C::KV_BYTES + c * C::KV_CHUNK, &tm_k, bar(C::B_KFULL + ks),
+                           c * 64, j * BK, h);
+        issued_k = jj + 1;
+        const int vs = jj % C::VS;
+        if (jj >= C::VS &&
+            !ptx::mbar_wait(bar(C::B_VEMPTY + vs), (jj / C::VS - 1) & 1, abort_flag, a.timeout_ns, kErrTimeout))
+          break;
+        ptx::mbar_arrive_expect_tx(bar(C::B_VFULL + vs), C::KV_BYTES);
+#pragma unroll
+        for (int c = 0; c < C::DCH; ++c)
+          ptx::tma_load_3d(sb + C::OFF_V + vs * C::KV_BYTES + c * C::KV_CHUNK, &tm_v, bar(C::B_VFULL + vs),
+                           c * 64, j * BK, h);
+        issued_v = jj + 1;
+      }
+      if (*abort_flag) {
+        const uint64_t short_ns = a.timeout_ns / 4;
+        volatile int dummy = 0;
+        for (int u = (issued_k > C::KS ? issued_k - C::KS : 0); u < issued_k; ++u)
+          ptx::mbar_wait(bar(C::B_KFULL + u % C::KS), (u / C::KS) & 1, &dummy, short_ns, 0);
+        for (int u = (issued_v > C::VS ? issued_v - C::VS : 0); u < issued_v; ++u)
+          ptx::mbar_wait(bar(C::B_VFULL + u % C::VS), (u / C::VS) & 1, &dummy, short_ns, 0);
+      }
+    } else if (warp == 9 && lane == 0 && n > 0) {
+      // ============================================================ S issuer
+      constexpr uint32_t HI = ptx::sdesc_sw128_hi(1024);
+      const uint32_t qlo = ptx::sdesc_sw128_lo(sb + C::OFF_Q, 16);
+      const uint32_t klo = ptx::sdesc_sw128_lo(sb + C::OFF_K, 16);
+      bool ok = ptx::mbar_wait(bar(C::B_QFULL), 0, abort_flag, a.timeout_ns, kErrTimeout);
+      for (int jj = 0; ok && jj < n; ++jj) {
+        const int b = jj & 1;
+        const int ks = jj % C::KS;
+        if (!ptx::mbar_wait(bar(C::B_KFULL + ks), (jj / C::KS) & 1, abort_flag, a.timeout_ns, kErrTimeout) ||
+            (jj >= 2 &&
+             !ptx::mbar_wait(bar(C::B_SFREE + b), ((jj - 2) >> 1) & 1, abort_flag, a.timeout_ns, kErrTimeout))) {
+          ok = false;
+          break;
+        }
+        ptx::tc_fence_after();
+        const uint32_t b0 = klo + static_cast<uint32_t>(ks * C::KV_BYTES >> 4);
+        const uint32_t s_tmem = tmem + (b ? C::TM_S1 : C::TM_S0);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t ao = (kk >> 2) * (C::Q_CHUNK >> 4) + (kk & 3) * 2;
+          const uint32_t bo = (kk >> 2) * (C::KV_CHUNK >> 4) + (kk & 3) * 2;
+          ptx::umma_ss_lohi(s_tmem, qlo + ao, b0 + bo, HI, C::IDESC_S, kk > 0 ? 1u : 0u);
+        }
+        ptx::umma_commit(bar(C::B_SFULL + b));
+        ptx::umma_commit(bar(C::B_KEMPTY + ks));
+      }
+      if (!ok) {
+        ptx::umma_commit(bar(C::B_DRAIN));
+        volatile int dummy = 0;
+        ptx::mbar_wait(bar(C::B_DRAIN), 0, &dummy, a.timeout_ns / 4, 0);
+      }
+    } else if (warp == 10 && lane == 0 && n > 0) {
+      // ============================================================ PV issuer
+      constexpr uint32_t HI = ptx::sdesc_sw128_hi(1024);
+      const uint32_t vlo = ptx::sdesc_sw128_lo(sb + C::OFF_V, C::KV_CHUNK);
+      bool ok = true;
+      for (int jj = 0; jj < n; ++jj) {
+        const int b = jj & 1;
+        const int vs = jj % C::VS;
+        if (!ptx::mbar_wait(bar(C::B_PFULL + b), (jj >> 1) & 1, abort_flag, a.timeout_ns, kErrTimeout) ||
+            !ptx::mbar_wait(bar(C::B_VFULL + vs), (jj / C::VS) & 1, abort_flag, a.timeout_ns, kErrTimeout)) {
+          ok = false;
+          break;
+        }
+        ptx::tc_fence_after();
+        const uint32_t b0 = vlo + static_cast<uint32_t>(vs * C::KV_BYTES >> 4);
+        const uint32_t p_tmem = tmem + (b ? C::TM_P1 : C::TM_P0);
+#pragma unroll
+        for (int kk = 0; kk < BK / 16; ++kk)
+          ptx::umma_ts_lohi(tmem + C::TM_O, p_tmem + kk * 8, b0 + kk * (2048 >> 4), HI, C::IDESC_PV,
+                            (jj > 0 || kk > 0) ? 1u : 0u);
+        ptx::umma_commit(bar(C::B_VEMPTY + vs));
+        ptx::umma_commit(bar(C::B_PVDONE + b));
+      }
+      if (!ok) {
+        ptx::umma_commit(bar(C::B_DRAIN + 1));
+        volatile int dummy = 0;
+        ptx::mbar_wait(bar(C::B_DRAIN + 1), 0, &dummy, a.timeout_ns / 4, 0);
+      }
+    }
+  } else {
+    // ================================================================ softmax
+    setmaxnreg_inc_224();
+    const int half = warp >> 2;                  // which half of the S columns
+    const int wq = warp & 3;
+    const int r = wq * 32 + lane;                // row within the tile == TMEM lane
+    const uint32_t lane_base = tmem + (static_cast<uint32_t>(wq * 32) << 16);
+    const int grow = qi * a.bq + r;
+    const bool row_valid = (r < a.bq) && (grow < a.L);
+    const float sl2 = a.scale_log2;
+    const uint32_t s_off = static_cast<uint32_t>(half * HALF);        // my S columns
+    const uint32_t p_off = static_cast<uint32_t>(half * (HALF / 2));  // my P cells
+    const uint32_t o_off = static_cast<uint32_t>(half * (D / 2));     // my O columns
+    if (n == 0) {
+      if (row_valid) {
+        uint4* dst = reinterpret_cast<uint4*>(a.o + (static_cast<long>(h) * a.L + grow) * D) + half * (D / 16);
+#pragma unroll
+        for (int c = 0; c < D / 16; ++c) dst[c] = make_uint4(0, 0, 0, 0);
+        if (half == 0) a.lse[static_cast<long>(h) * a.L + grow] = -__int_as_float(0x7f800000);
+      }
+    } else {
+      float m = -__int_as_float(0x7f800000);  // running row max, log2 units (scaled)
+      float l = 0.f;                          // running sum of my half row
+      bool ok = true;
+      for (int jj = 0; jj < n; ++jj) {
+        const int b = jj & 1;
+        if (!ptx::mbar_wait_warp(bar(C::B_SFULL + b), (jj >> 1) & 1, abort_flag, a.timeout_ns, kErrTimeout)) {
+          ok = false;
+          break;
+        }
+        ptx::tc_fence_after();
+        float s[HALF];
+        {
+          uint32_t raw[HALF / 32 > 0 ? HALF / 32 : 1][32];
+#pragma unroll
+          for (int c = 0; c < HALF / 32; ++c)
+            ptx::tmem_ld32(lane_base + (b ? C::TM_S1 : C::TM_S0) + s_off + c * 32, raw[c]);
+          ptx::tmem_wait_ld();
+#pragma unroll
+          for (int c = 0; c < HALF / 32; ++c) {
+            ptx::reg_fence32(raw[c]);
+#pragma unroll
+            for (int e = 0; e < 32; ++e) s[c * 32 + e] = __uint_as_float(raw[c][e]);
+          }
+        }
+        ptx::tc_fence_before();
+        ptx::mbar_arrive(bar(C::B_SFREE + b));
+        // ragged last key block: keys past L do not exist
+        const int valid = a.L - kv_block(jj) * BK - static_cast<int>(s_off);
+        if (valid < HALF) {
+#pragma unroll
+          for (int c = 0; c < HALF; ++c)
+            if (c >= valid) s[c] = -__int_as_float(0x7f800000);
+        }
+        float mx0 = s[0], mx1 = s[1];
+#pragma unroll
+        for (int c = 2; c < HALF; c += 4) {
+          mx0 = ptx::max3(mx0, s[c], s[c + 1]);
+          if (c + 3 < HALF) mx1 = ptx::max3(mx1, s[c + 2], s[c + 3]);
+        }
+        // exchange the half-row maxima (mbarrier: 8 warp arrivals, bounded wait)
+        xchg[(b * 2 + half) * 128 + r] = fmaxf(mx0, mx1);
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive(bar(C::B_XCHG + b));
+        if (!ptx::mbar_wait_warp(bar(C::B_XCHG + b), (jj >> 1) & 1, abort_flag, a.timeout_ns, kErrTimeout)) {
+          ok = false;
+          break;
+        }
+        const float mx = fmaxf(xchg[(b * 2) * 128 + r], xchg[(b * 2 + 1) * 128 + r]);
+        const float m_new = fmaxf(m, mx * sl2);
+        if (jj == 0) {
+          m = m_new;
+        } else if (__any_sync(0xffffffffu, m_new > m + 8.0f)) {
+          // O holds tiles < jj-1 plus PV(jj-1): wait for it, rescale my half
+          if (!ptx::mbar_wait_warp(bar(C::B_PVDONE + ((jj - 1) & 1)), ((jj - 1) >> 1) & 1, abort_flag,
+                                   a.timeout_ns, kErrTimeout)) {
+            ok = false;
+            break;
+          }
+          ptx::tc_fence_after();
+          const float alpha = ptx::ex2(m - m_new);
+#pragma unroll
+          for (int c = 0; c < D / 64; ++c) {
+            uint32_t raw[32];
+            ptx::tmem_ld32(lane_base + C::TM_O + o_off + c * 32, raw);
+            ptx::tmem_wait_ld();
+            ptx::reg_fence32(raw);
+#pragma unroll
+            for (int e = 0; e < 32; ++e) raw[e] = __float_as_uint(__uint_as_float(raw[e]) * alpha);
+            ptx::tmem_st32(lane_base + C::TM_O + o_off + c * 32, raw);
+          }
+          ptx::tmem_wait_st();
+          l *= alpha;
+          m = m_new;
+        }
+        // P_b is free once PV(jj-2) has consumed it
+        if (jj >= 2 && !ptx::mbar_wait_warp(bar(C::B_PVDONE + b), ((jj - 2) >> 1) & 1, abort_flag,
+                                            a.timeout_ns, kErrTimeout)) {
+          ok = false;
+          break;
+        }
+        ptx::tc_fence_after();
+        l += softmax_half_exp<HALF>(s, sl2, m, lane_base + (b ? C::TM_P1 : C::TM_P0) + p_off);
+        ptx::tmem_wait_st();
+        ptx::tc_fence_before();
+        ptx::mbar_arrive(bar(C::B_PFULL + b));
+      }
+      if (ok)
+        ok = ptx::mbar_wait_warp(bar(C::B_PVDONE + ((n - 1) & 1)), ((n - 1) >> 1) & 1, abort_flag,
+                                 a.timeout_ns, kErrTimeout);
+      // ---- epilogue: combine the two half-row sums, O / l -> bf16 -> swizzled
+      // smem (the Q tile, no longer read by any MMA) -> TMA store; LSE.
+      if (ok) {
+        lsum_x[half * 128 + r] = l;
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive(bar(C::B_EPI));
+        ok = ptx::mbar_wait_warp(bar(C::B_EPI), 0, abort_flag, a.timeout_ns, kErrTimeout);
+      }
+      if (ok) {
+        ptx::tc_fence_after();
+        const float lt = lsum_x[r] + lsum_x[128 + r];
+        const float inv_l = 1.0f / lt;
+#pragma unroll
+        for (int c = 0; c < D / 64; ++c) {
+          uint32_t raw[32];
+          ptx::tmem_ld32(lane_base + C::TM_O + o_off + c * 32, raw);
+          ptx::tmem_wait_ld();
+          ptx::reg_fence32(raw);
+          uint32_t pk[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e)
+            pk[e] = ptx::pack_bf16x2(__uint_as_float(raw[2 * e]) * inv_l, __uint_as_float(raw[2 * e + 1]) * inv_l);
+          const int col32 = static_cast<int>(o_off) / 32 + c;  // 32-column group of O
+          uint8_t* chunk = smem + C::OFF_Q + (col32 >> 1) * C::Q_CHUNK + r * 128;
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const int unit = ((col32 & 1) * 4 + u) ^ (r & 7);
+            *reinterpret_cast<uint4*>(chunk + unit * 16) =
+                make_uint4(pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
+          }
+        }
+        if (row_valid && half == 0)
+          a.lse[static_cast<long>(h) * a.L + grow] = (m + ptx::lg2(lt)) * 0.69314718055994530942f;
+        ptx::fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive(bar(C::B_EPI + 1));
+        ok = ptx::mbar_wait_warp(bar(C::B_EPI + 1), 0, abort_flag, a.timeout_ns, kErrTimeout);
+      }
+      if (ok && threadIdx.x == 0 && !*abort_flag) {
+#pragma unroll
+        for (int c = 0; c < C::DCH; ++c)
+          ptx::tma_store_3d(&tm_o, sb + C::OFF_Q + c * C::Q_CHUNK, c * 64, qi * a.bq, h);
+        ptx::bulk_commit();
+        ptx::bulk_wait0();
+      }
+    }
+  }
+
+  ptx::tc_fence_before();
+  __syncthreads();
+  if (warp == 9) {
+    ptx::tc_fence_after();
+    ptx::tmem_dealloc(tmem, C::TM_ALLOC);
+  }
+}
+
+}  // namespace sparsed

@@ -14,7 +14,7 @@
 #include <vector>
 
 #include "sparsed.h"
-#include "attn_kernel.cuh"
+#include "attn3_kernel.cuh"
 #include "select_kernels.cuh"
 
 using namespace sparsed;
@@ -127,10 +127,21 @@ struct Problem {
   float scale;
 };
 
+// The register split of the kernel (setmaxnreg) must be funded by its launch
+// register count; checked once per kernel before the first launch, so a raise
+// can never wait forever.
 template <int D, int BK, bool SPARSE>
 int launch_attn_t(const Problem& p, const int32_t* kv_idx, const int32_t* kv_count, int kv_stride,
                   cudaStream_t st) {
-  using C = AttnCfg<D, BK>;
+  using C = Attn3Cfg<D, BK>;
+  auto kern = attn3_fwd_kernel<D, BK, SPARSE>;
+  static int regs = -1;
+  if (regs < 0) {
+    cudaFuncAttributes fa;
+    SP_CUDA(cudaFuncGetAttributes(&fa, kern));
+    regs = fa.numRegs;
+  }
+  if (regs * C::THREADS < C::REGS_SOFTMAX * 256 + C::REGS_OTHER * 128) return SPARSED_ERR_UNSUPPORTED;
   CUtensorMap tq, tk, tv, to;
   SP_TRY(make_map(&tq, p.Q, p.H, p.L, D, 128));
   SP_TRY(make_map(&tk, p.K, p.H, p.L, D, BK));
@@ -149,9 +160,8 @@ int launch_attn_t(const Problem& p, const int32_t* kv_idx, const int32_t* kv_cou
   a.lse = p.LSE;
   a.o = p.O;
   a.timeout_ns = kWaitTimeoutNs;
-  auto kern = attn_fwd_kernel<D, BK, SPARSE>;
   SP_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES));
-  kern<<<dim3(p.nqb, p.H), 256, C::SMEM_BYTES, st>>>(tq, tk, tv, to, a);
+  kern<<<dim3(p.nqb, p.H), C::THREADS, C::SMEM_BYTES, st>>>(tq, tk, tv, to, a);
   SP_CUDA(cudaGetLastError());
   return SPARSED_OK;
 }
