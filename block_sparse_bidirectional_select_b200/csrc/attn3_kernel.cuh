@@ -11,8 +11,10 @@
 // bitwise equal to the dense call.
 //
 // Warp roles (384 threads):
-//   warps 0-3   softmax, columns [0, BK/2) of every S tile (thread r: row r)
-//   warps 4-7   softmax, columns [BK/2, BK)
+//   warps 0-7   softmax. Warp w covers the 16 rows 32*(w%4) + 16*(w/4) + 0..15
+//               of the tile with the "16x32bx2" TMEM access: thread t holds row
+//               t%16 and the column half t/16 of every S tile, so the two
+//               halves of a row meet in one warp (row max / sum by shuffle).
 //   warp 8      TMA producer: Q once, then K_j / V_j into KS- and VS-deep rings
 //   warp 9      TMEM owner; its lane 0 issues the S = Q K^T MMAs
 //   warp 10     lane 0 issues the O += P V MMAs
@@ -21,15 +23,15 @@
 // double-buffered, so S(j+1) is computed while the softmax works on S(j); P has
 // its own two buffers, so the two issuers never touch the same columns and can
 // run independently (a commit from one thread tracks only its own MMAs):
-//   S issuer : S_b(j) after the softmax released S_b(j-2)        (SFREE)
-//   softmax  : reads S_b(j), exchanges the half-row maxima, writes P_b(j) after
-//              PV(j-2) released P_b                              (PVDONE)
-//   PV issuer: O += P_b(j) V_j                                   (PFULL)
-// Both softmax halves of a row compute the same row max, so the lazy rescale
-// (O and the running sum keep a stale max until a row's max grows by more than
-// 2^8) takes the same decision in both; each half rescales its half of O.
-// Every wait is bounded; the in-loop exchange uses an mbarrier (bounded), never
-// a named barrier, so a timed-out warp cannot strand the others.
+//   S issuer : S_b(j) once PV(j-2) is done (which also means the softmax has
+//              read S_b(j-2) and that P_b is free again)       (PVDONE)
+//   softmax  : reads S_b(j), writes P_b(j)                      (SFULL -> PFULL)
+//   PV issuer: O += P_b(j) V_j                                  (PFULL -> PVDONE)
+// The lazy rescale keeps O and the running sum on a stale row max until a
+// row's max grows by more than 2^8; both halves of a row see the same max, so
+// they take the same decision, and each rescales its half of O.
+// Every wait is bounded (mbarriers only, no named barriers), so a timed-out
+// warp cannot strand the others.
 #pragma once
 
 #include "ptx_sm100.cuh"
@@ -66,7 +68,7 @@ struct Attn3Cfg {
   static constexpr int KS = 3;
   // a third V stage when it fits next to Q, three K stages and ~4 KB of
   // barriers / exchange buffers
-  static constexpr int VS = (Q_BYTES + 6 * KV_BYTES + 6144) <= 232448 ? 3 : 2;
+  static constexpr int VS = (Q_BYTES + 6 * KV_BYTES + 2048) <= 232448 ? 3 : 2;
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_K = Q_BYTES;
   static constexpr int OFF_V = OFF_K + KS * KV_BYTES;
@@ -77,16 +79,12 @@ struct Attn3Cfg {
   static constexpr int B_VFULL = B_KEMPTY + KS;
   static constexpr int B_VEMPTY = B_VFULL + VS;
   static constexpr int B_SFULL = B_VEMPTY + VS;  // [2]
-  static constexpr int B_SFREE = B_SFULL + 2;    // [2] 256 arrivals
-  static constexpr int B_PFULL = B_SFREE + 2;    // [2] 256 arrivals
+  static constexpr int B_PFULL = B_SFULL + 2;    // [2] 8 warp arrivals
   static constexpr int B_PVDONE = B_PFULL + 2;   // [2]
-  static constexpr int B_XCHG = B_PVDONE + 2;    // [2] half-row maxima exchanged (8 warps)
-  static constexpr int B_EPI = B_XCHG + 2;       // epilogue: sums exchanged / O staged (8 warps)
-  static constexpr int B_DRAIN = B_EPI + 2;      // [2] per issuer
+  static constexpr int B_EPI = B_PVDONE + 2;     // O staged in smem (8 warp arrivals)
+  static constexpr int B_DRAIN = B_EPI + 1;      // [2] per issuer
   static constexpr int NUM_BARS = B_DRAIN + 2;
-  static constexpr int OFF_XCHG = OFF_BAR + NUM_BARS * 8;  // float [2 bufs][2 halves][128]
-  static constexpr int OFF_LSUM = OFF_XCHG + 2 * 2 * 128 * 4;  // float [2 halves][128]
-  static constexpr int OFF_MISC = OFF_LSUM + 2 * 128 * 4;      // tmem slot, abort flag
+  static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;  // tmem slot, abort flag
   static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;
   static constexpr int TM_S0 = 0;
   static constexpr int TM_S1 = BK;
@@ -105,10 +103,13 @@ struct Attn3Cfg {
 };
 
 // The exp pass of one half row: P = bf16(2^(s*sl2 - m)) for HALF columns into
-// TMEM at p_taddr (two columns per 32-bit cell, even column in the low half),
-// returning the fp32 sum. Column pairs go through packed fp32x2 FMA/ADD.
+// TMEM at p_taddr through the 16x32bx2 access (two columns per 32-bit cell,
+// even column in the low half; the other half row's cells HALF/2 further on),
+// returning the fp32 sum. Column pairs go through packed fp32x2 FMA/ADD, and
+// one column in four takes its exponential on the FMA pipe (exp2_fma).
 template <int HALF>
 __device__ __forceinline__ float softmax_half_exp(const float (&s)[HALF], float sl2, float m, uint32_t p_taddr) {
+  static_assert(HALF == 32 || HALF == 64, "half row of 32 or 64 columns");
   const uint64_t scale2 = ptx::f32x2(sl2, sl2);
   const uint64_t negm2 = ptx::f32x2(-m, -m);
   uint64_t acc0 = ptx::f32x2(0.f, 0.f), acc1 = acc0;
@@ -121,24 +122,34 @@ __device__ __forceinline__ float softmax_half_exp(const float (&s)[HALF], float 
       const int i0 = c * 64 + 2 * e;
       float x0, x1;
       ptx::f32x2_split(ptx::fma_f32x2(ptx::f32x2(s[i0], s[i0 + 1]), scale2, negm2), x0, x1);
+      // every fourth column's exponential on the FMA pipe: MUFU (16 per
+      // clock per SM) is the softmax's binding unit
       const float p0 = ptx::ex2(x0);
-      const float p1 = ptx::ex2(x1);
+      const float p1 = (e & 1) ? ptx::exp2_fma(x1) : ptx::ex2(x1);
       if (e & 1)
         acc1 = ptx::add_f32x2(acc1, ptx::f32x2(p0, p1));
       else
         acc0 = ptx::add_f32x2(acc0, ptx::f32x2(p0, p1));
       pk[e] = ptx::pack_bf16x2(p0, p1);
     }
+    // thread t's cells go to column half t/16 of the tile's P cells
     if constexpr (W == 32) {
-      ptx::tmem_st32(p_taddr + c * 32, pk);
+      ptx::tmem_st16x2_32<HALF / 2>(p_taddr, pk);
     } else {
-      ptx::tmem_st16(p_taddr + c * 32, pk);
+      ptx::tmem_st16x2_16<HALF / 2>(p_taddr, pk);
     }
   }
   float a0, a1, b0, b1;
   ptx::f32x2_split(acc0, a0, a1);
   ptx::f32x2_split(acc1, b0, b1);
   return (a0 + b0) + (a1 + b1);
+}
+
+// Store 32 O columns of my row half through the 16x32bx2 access (the other
+// half of the row's O columns D/2 further on).
+template <int D>
+__device__ __forceinline__ void tmem_st16x2_o(uint32_t taddr, const uint32_t (&r)[32]) {
+  ptx::tmem_st16x2_32<D / 2>(taddr, r);
 }
 
 template <int D, int BK, bool SPARSE>
@@ -156,8 +167,6 @@ __global__ void __launch_bounds__(384, 1)
   const int lane = threadIdx.x & 31;
   const int qi = blockIdx.x;
   const int h = blockIdx.y;
-  float* xchg = reinterpret_cast<float*>(smem + C::OFF_XCHG);
-  float* lsum_x = reinterpret_cast<float*>(smem + C::OFF_LSUM);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
   auto bar = [&](int idx) -> uint32_t { return sb + C::OFF_BAR + 8 * idx; };
@@ -197,13 +206,11 @@ __global__ void __launch_bounds__(384, 1)
     }
     for (int b = 0; b < 2; ++b) {
       ptx::mbar_init(bar(C::B_SFULL + b), 1);
-      ptx::mbar_init(bar(C::B_SFREE + b), 256);
-      ptx::mbar_init(bar(C::B_PFULL + b), 256);
+      ptx::mbar_init(bar(C::B_PFULL + b), 8);  // one arrival per softmax warp
       ptx::mbar_init(bar(C::B_PVDONE + b), 1);
-      ptx::mbar_init(bar(C::B_XCHG + b), 8);
-      ptx::mbar_init(bar(C::B_EPI + b), 8);
       ptx::mbar_init(bar(C::B_DRAIN + b), 1);
     }
+    ptx::mbar_init(bar(C::B_EPI), 8);
     *abort_flag = 0;
     ptx::fence_mbar_init();
   }
@@ -276,7 +283,7 @@ __global__ void __launch_bounds__(384, 1)
         const int ks = jj % C::KS;
         if (!ptx::mbar_wait(bar(C::B_KFULL + ks), (jj / C::KS) & 1, abort_flag, a.timeout_ns, kErrTimeout) ||
             (jj >= 2 &&
-             !ptx::mbar_wait(bar(C::B_SFREE + b), ((jj - 2) >> 1) & 1, abort_flag, a.timeout_ns, kErrTimeout))) {
+             !ptx::mbar_wait(bar(C::B_PVDONE + b), ((jj - 2) >> 1) & 1, abort_flag, a.timeout_ns, kErrTimeout))) {
           ok = false;
           break;
         }
@@ -329,16 +336,13 @@ __global__ void __launch_bounds__(384, 1)
   } else {
     // ================================================================ softmax
     setmaxnreg_inc_224();
-    const int half = warp >> 2;                  // which half of the S columns
-    const int wq = warp & 3;
-    const int r = wq * 32 + lane;                // row within the tile == TMEM lane
-    const uint32_t lane_base = tmem + (static_cast<uint32_t>(wq * 32) << 16);
+    const int half = lane >> 4;                             // column half of my row
+    const int r = (warp & 3) * 32 + (warp >> 2) * 16 + (lane & 15);  // row == TMEM lane
+    const uint32_t lane_base = tmem + (static_cast<uint32_t>((warp & 3) * 32 + (warp >> 2) * 16) << 16);
     const int grow = qi * a.bq + r;
     const bool row_valid = (r < a.bq) && (grow < a.L);
     const float sl2 = a.scale_log2;
-    const uint32_t s_off = static_cast<uint32_t>(half * HALF);        // my S columns
-    const uint32_t p_off = static_cast<uint32_t>(half * (HALF / 2));  // my P cells
-    const uint32_t o_off = static_cast<uint32_t>(half * (D / 2));     // my O columns
+    const int s_off = half * HALF;   // first S column of my half row
     if (n == 0) {
       if (row_valid) {
         uint4* dst = reinterpret_cast<uint4*>(a.o + (static_cast<long>(h) * a.L + grow) * D) + half * (D / 16);
@@ -359,10 +363,10 @@ __global__ void __launch_bounds__(384, 1)
         ptx::tc_fence_after();
         float s[HALF];
         {
-          uint32_t raw[HALF / 32 > 0 ? HALF / 32 : 1][32];
+          uint32_t raw[HALF / 32][32];
 #pragma unroll
           for (int c = 0; c < HALF / 32; ++c)
-            ptx::tmem_ld32(lane_base + (b ? C::TM_S1 : C::TM_S0) + s_off + c * 32, raw[c]);
+            ptx::tmem_ld16x2_32<HALF>(lane_base + (b ? C::TM_S1 : C::TM_S0) + c * 32, raw[c]);
           ptx::tmem_wait_ld();
 #pragma unroll
           for (int c = 0; c < HALF / 32; ++c) {
@@ -371,10 +375,8 @@ __global__ void __launch_bounds__(384, 1)
             for (int e = 0; e < 32; ++e) s[c * 32 + e] = __uint_as_float(raw[c][e]);
           }
         }
-        ptx::tc_fence_before();
-        ptx::mbar_arrive(bar(C::B_SFREE + b));
         // ragged last key block: keys past L do not exist
-        const int valid = a.L - kv_block(jj) * BK - static_cast<int>(s_off);
+        const int valid = a.L - kv_block(jj) * BK - s_off;
         if (valid < HALF) {
 #pragma unroll
           for (int c = 0; c < HALF; ++c)
@@ -386,15 +388,8 @@ __global__ void __launch_bounds__(384, 1)
           mx0 = ptx::max3(mx0, s[c], s[c + 1]);
           if (c + 3 < HALF) mx1 = ptx::max3(mx1, s[c + 2], s[c + 3]);
         }
-        // exchange the half-row maxima (mbarrier: 8 warp arrivals, bounded wait)
-        xchg[(b * 2 + half) * 128 + r] = fmaxf(mx0, mx1);
-        __syncwarp();
-        if (lane == 0) ptx::mbar_arrive(bar(C::B_XCHG + b));
-        if (!ptx::mbar_wait_warp(bar(C::B_XCHG + b), (jj >> 1) & 1, abort_flag, a.timeout_ns, kErrTimeout)) {
-          ok = false;
-          break;
-        }
-        const float mx = fmaxf(xchg[(b * 2) * 128 + r], xchg[(b * 2 + 1) * 128 + r]);
+        float mx = fmaxf(mx0, mx1);
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));  // the other half of my row
         const float m_new = fmaxf(m, mx * sl2);
         if (jj == 0) {
           m = m_new;
@@ -410,55 +405,44 @@ __global__ void __launch_bounds__(384, 1)
 #pragma unroll
           for (int c = 0; c < D / 64; ++c) {
             uint32_t raw[32];
-            ptx::tmem_ld32(lane_base + C::TM_O + o_off + c * 32, raw);
+            ptx::tmem_ld16x2_32<D / 2>(lane_base + C::TM_O + c * 32, raw);
             ptx::tmem_wait_ld();
             ptx::reg_fence32(raw);
 #pragma unroll
             for (int e = 0; e < 32; ++e) raw[e] = __float_as_uint(__uint_as_float(raw[e]) * alpha);
-            ptx::tmem_st32(lane_base + C::TM_O + o_off + c * 32, raw);
+            tmem_st16x2_o<D>(lane_base + C::TM_O + c * 32, raw);
           }
           ptx::tmem_wait_st();
           l *= alpha;
           m = m_new;
         }
-        // P_b is free once PV(jj-2) has consumed it
-        if (jj >= 2 && !ptx::mbar_wait_warp(bar(C::B_PVDONE + b), ((jj - 2) >> 1) & 1, abort_flag,
-                                            a.timeout_ns, kErrTimeout)) {
-          ok = false;
-          break;
-        }
-        ptx::tc_fence_after();
-        l += softmax_half_exp<HALF>(s, sl2, m, lane_base + (b ? C::TM_P1 : C::TM_P0) + p_off);
+        // P_b is free: S_b(jj) was issued only after PV(jj-2) completed
+        l += softmax_half_exp<HALF>(s, sl2, m, lane_base + (b ? C::TM_P1 : C::TM_P0));
         ptx::tmem_wait_st();
         ptx::tc_fence_before();
-        ptx::mbar_arrive(bar(C::B_PFULL + b));
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive(bar(C::B_PFULL + b));
       }
       if (ok)
         ok = ptx::mbar_wait_warp(bar(C::B_PVDONE + ((n - 1) & 1)), ((n - 1) >> 1) & 1, abort_flag,
                                  a.timeout_ns, kErrTimeout);
-      // ---- epilogue: combine the two half-row sums, O / l -> bf16 -> swizzled
-      // smem (the Q tile, no longer read by any MMA) -> TMA store; LSE.
-      if (ok) {
-        lsum_x[half * 128 + r] = l;
-        __syncwarp();
-        if (lane == 0) ptx::mbar_arrive(bar(C::B_EPI));
-        ok = ptx::mbar_wait_warp(bar(C::B_EPI), 0, abort_flag, a.timeout_ns, kErrTimeout);
-      }
+      // ---- epilogue: O / l -> bf16 -> swizzled smem (the Q tile, no longer
+      // read by any MMA) -> TMA store; LSE.
       if (ok) {
         ptx::tc_fence_after();
-        const float lt = lsum_x[r] + lsum_x[128 + r];
+        const float lt = l + __shfl_xor_sync(0xffffffffu, l, 16);
         const float inv_l = 1.0f / lt;
 #pragma unroll
         for (int c = 0; c < D / 64; ++c) {
           uint32_t raw[32];
-          ptx::tmem_ld32(lane_base + C::TM_O + o_off + c * 32, raw);
+          ptx::tmem_ld16x2_32<D / 2>(lane_base + C::TM_O + c * 32, raw);
           ptx::tmem_wait_ld();
           ptx::reg_fence32(raw);
           uint32_t pk[16];
 #pragma unroll
           for (int e = 0; e < 16; ++e)
             pk[e] = ptx::pack_bf16x2(__uint_as_float(raw[2 * e]) * inv_l, __uint_as_float(raw[2 * e + 1]) * inv_l);
-          const int col32 = static_cast<int>(o_off) / 32 + c;  // 32-column group of O
+          const int col32 = half * (D / 64) + c;  // 32-column group of O this thread holds
           uint8_t* chunk = smem + C::OFF_Q + (col32 >> 1) * C::Q_CHUNK + r * 128;
 #pragma unroll
           for (int u = 0; u < 4; ++u) {
@@ -471,8 +455,8 @@ __global__ void __launch_bounds__(384, 1)
           a.lse[static_cast<long>(h) * a.L + grow] = (m + ptx::lg2(lt)) * 0.69314718055994530942f;
         ptx::fence_proxy_async_smem();
         __syncwarp();
-        if (lane == 0) ptx::mbar_arrive(bar(C::B_EPI + 1));
-        ok = ptx::mbar_wait_warp(bar(C::B_EPI + 1), 0, abort_flag, a.timeout_ns, kErrTimeout);
+        if (lane == 0) ptx::mbar_arrive(bar(C::B_EPI));
+        ok = ptx::mbar_wait_warp(bar(C::B_EPI), 0, abort_flag, a.timeout_ns, kErrTimeout);
       }
       if (ok && threadIdx.x == 0 && !*abort_flag) {
 #pragma unroll
