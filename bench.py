@@ -260,6 +260,9 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--skip-cpu", action="store_true")
     ap.add_argument("--skip-e2e", action="store_true")
+    ap.add_argument("--op", choices=["run", "dense", "sparse", "select"], default="run",
+                    help="run: the full denoising run (the benchmark); dense/sparse/select: time one "
+                         "library call alone, K launches after W warm-up launches (for profiling)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     rank = int(os.environ.get("RANK", "0"))
@@ -288,6 +291,8 @@ def main():
         return float(t.item())
 
     wl = WORKLOADS[args.workload]
+    if args.op != "run":
+        return time_one_op(args, wl, dev, rank)
     log(f"[rank {rank}] inputs for {wl.name}")
     q_cpu, k_cpu, v_cpu = make_inputs(wl.scaled(seed=wl.seed + rank))
     q, k, v = (t.to(dev) for t in (q_cpu, k_cpu, v_cpu))
@@ -438,6 +443,43 @@ def main():
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.destroy_process_group()
+    return 0
+
+
+def time_one_op(args, wl, dev, rank):
+    """Time one library call alone (dense_attn, block_sparse_attn with the
+    pattern select_pattern picks, or select_pattern) on one GPU."""
+    import block_sparse_bidirectional_select_b200 as sp
+    q, k, v = (t.to(dev) for t in make_inputs(wl))
+    stream = torch.cuda.current_stream()
+    o = torch.empty_like(q)
+    lse = torch.empty((wl.H, wl.L), dtype=torch.float32, device=dev)
+    dense_flops = 4.0 * wl.H * float(wl.L) * float(wl.L) * wl.d
+    if args.op == "dense":
+        fn = lambda: sp.dense_attn(q, k, v, bq=wl.bq, bk=wl.bk, out=o, lse=lse)
+        flops = dense_flops
+    elif args.op == "select":
+        ws = torch.empty(sp.workspace_bytes(wl.H, wl.L, wl.bq, wl.bk), dtype=torch.uint8, device=dev)
+        fn = lambda: sp.select_pattern(q, k, v, keep=wl.keep, budget=wl.budget, bq=wl.bq, bk=wl.bk,
+                                       workspace=ws)
+        flops = dense_flops
+    else:
+        pat = sp.select_pattern(q, k, v, keep=wl.keep, budget=wl.budget, bq=wl.bq, bk=wl.bk)
+        fn = lambda: sp.block_sparse_attn(q, k, v, pat.kv_idx, pat.kv_count, bq=wl.bq, bk=wl.bk, out=o, lse=lse)
+        flops = 4.0 * wl.bq * wl.bk * wl.d * float(pat.kv_count.sum().item())
+    for _ in range(args.warmup):
+        fn()
+    sp.device_check()
+    torch.cuda.synchronize()
+    clocks = ClockSampler(dev.index or 0)
+    clocks.start()
+    times = [event_time(fn, stream, 1) for _ in range(args.steps)]
+    clk = clocks.stop()
+    sp.device_check()
+    ms = statistics.median(times)
+    if rank == 0:
+        print(json.dumps({"op": args.op, "workload": wl.name, "launches": args.steps, "ms_median": ms,
+                          "ms_all": times, "tflops": flops / (ms * 1e-3) / 1e12, "clocks": clk}), flush=True)
     return 0
 
 
