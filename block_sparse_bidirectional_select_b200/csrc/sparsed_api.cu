@@ -14,7 +14,7 @@
 #include <vector>
 
 #include "sparsed.h"
-#include "attn3_kernel.cuh"
+#include "attn_kernel.cuh"
 #include "select_kernels.cuh"
 
 using namespace sparsed;
@@ -76,6 +76,14 @@ int require_sm100() {
   return SPARSED_OK;
 }
 
+// Number of SMs of the current device (the persistent grid size).
+int sm_count(int* out) {
+  int dev = 0;
+  SP_CUDA(cudaGetDevice(&dev));
+  SP_CUDA(cudaDeviceGetAttribute(out, cudaDevAttrMultiProcessorCount, dev));
+  return SPARSED_OK;
+}
+
 inline long cdiv(long a, long b) { return (a + b - 1) / b; }
 inline size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -133,8 +141,8 @@ struct Problem {
 template <int D, int BK, bool SPARSE>
 int launch_attn_t(const Problem& p, const int32_t* kv_idx, const int32_t* kv_count, int kv_stride,
                   cudaStream_t st) {
-  using C = Attn3Cfg<D, BK>;
-  auto kern = attn3_fwd_kernel<D, BK, SPARSE>;
+  using C = AttnCfg<D, BK>;
+  auto kern = attn_fwd_kernel<D, BK, SPARSE>;
   static int regs = -1;
   if (regs < 0) {
     cudaFuncAttributes fa;
@@ -142,11 +150,10 @@ int launch_attn_t(const Problem& p, const int32_t* kv_idx, const int32_t* kv_cou
     regs = fa.numRegs;
   }
   if (regs * C::THREADS < C::REGS_SOFTMAX * 256 + C::REGS_OTHER * 128) return SPARSED_ERR_UNSUPPORTED;
-  CUtensorMap tq, tk, tv, to;
+  CUtensorMap tq, tk, tv;
   SP_TRY(make_map(&tq, p.Q, p.H, p.L, D, 128));
   SP_TRY(make_map(&tk, p.K, p.H, p.L, D, BK));
   SP_TRY(make_map(&tv, p.V, p.H, p.L, D, BK));
-  SP_TRY(make_map(&to, p.O, p.H, p.L, D, p.bq));
   AttnArgs a;
   a.H = p.H;
   a.L = p.L;
@@ -160,8 +167,14 @@ int launch_attn_t(const Problem& p, const int32_t* kv_idx, const int32_t* kv_cou
   a.lse = p.LSE;
   a.o = p.O;
   a.timeout_ns = kWaitTimeoutNs;
+  int sms = 0;
+  SP_TRY(sm_count(&sms));
   SP_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES));
-  kern<<<dim3(p.nqb, p.H), C::THREADS, C::SMEM_BYTES, st>>>(tq, tk, tv, to, a);
+  // persistent: one CTA per SM (shared memory admits one), each walking items
+  // blockIdx.x, blockIdx.x + gridDim.x, ...
+  const long items = static_cast<long>(p.H) * p.nqb;
+  const int grid = static_cast<int>(items < sms ? items : sms);
+  kern<<<grid, C::THREADS, C::SMEM_BYTES, st>>>(tq, tk, tv, a);
   SP_CUDA(cudaGetLastError());
   return SPARSED_OK;
 }
