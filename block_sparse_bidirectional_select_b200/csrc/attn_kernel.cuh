@@ -169,18 +169,23 @@ struct ItemList {
   }
 };
 
+// kv_count of work item w (row h*nqb + i of the [H, nqb] count array); every
+// role reads the next item's count one item ahead, off its critical path
 template <bool SPARSE>
-__device__ __forceinline__ ItemList<SPARSE> item_list(const AttnArgs& a, int h, int qi) {
+__device__ __forceinline__ int raw_count(const AttnArgs& a, int w) {
+  if constexpr (SPARSE) return w < a.H * a.nqb ? a.kv_count[w] : 0;
+  else return a.nkb;
+}
+
+template <bool SPARSE>
+__device__ __forceinline__ ItemList<SPARSE> item_list(const AttnArgs& a, int w, int n_raw) {
   ItemList<SPARSE> it;
   it.nkb = a.nkb;
   it.n = a.nkb;
   if constexpr (SPARSE) {
-    const long row = static_cast<long>(h) * a.nqb + qi;
-    int n = a.kv_count[row];
     const int cap = a.kv_stride < a.nkb ? a.kv_stride : a.nkb;
-    if (n < 0 || n > cap) n = n < 0 ? 0 : cap;  // reported by the producer
-    it.n = n;
-    it.list = a.kv_idx + row * a.kv_stride;
+    it.n = n_raw < 0 ? 0 : (n_raw > cap ? cap : n_raw);  // a bad count is reported by the producer
+    it.list = a.kv_idx + static_cast<long>(w) * a.kv_stride;
   }
   return it;
 }
@@ -242,13 +247,12 @@ __global__ void __launch_bounds__(384, 1)
       int g = 0, iq = 0;  // tile counter, Q tiles loaded so far
       int issued_k = 0, issued_v = 0;
       bool ok = true;
-      for (int w = blockIdx.x; ok && w < n_items; w += gridDim.x) {
+      int n_raw = raw_count<SPARSE>(a, blockIdx.x), n_raw_next = 0;
+      for (int w = blockIdx.x; ok && w < n_items; w += gridDim.x, n_raw = n_raw_next) {
+        n_raw_next = raw_count<SPARSE>(a, w + gridDim.x);
         const int h = w / a.nqb, qi = w - h * a.nqb;
-        const ItemList<SPARSE> it = item_list<SPARSE>(a, h, qi);
-        if constexpr (SPARSE) {
-          const int n_raw = a.kv_count[static_cast<long>(h) * a.nqb + qi];
-          if (n_raw != it.n) ptx::record_error(kErrBadPattern);
-        }
+        const ItemList<SPARSE> it = item_list<SPARSE>(a, w, n_raw);
+        if (SPARSE && n_raw != it.n) ptx::record_error(kErrBadPattern);
         if (it.n == 0) continue;
         // Q of this item once every S MMA of the previous item is complete
         if (iq > 0 && !ptx::mbar_wait(bar(C::B_QEMPTY), (iq - 1) & 1, abort_flag, a.timeout_ns, kErrTimeout)) {
@@ -312,9 +316,10 @@ __global__ void __launch_bounds__(384, 1)
       const uint32_t klo = ptx::sdesc_sw128_lo(sb + C::OFF_K, 16);
       int g = 0, iq = 0;
       bool ok = true;
-      for (int w = blockIdx.x; ok && w < n_items; w += gridDim.x) {
-        const int h = w / a.nqb, qi = w - h * a.nqb;
-        const ItemList<SPARSE> it = item_list<SPARSE>(a, h, qi);
+      int n_raw = raw_count<SPARSE>(a, blockIdx.x), n_raw_next = 0;
+      for (int w = blockIdx.x; ok && w < n_items; w += gridDim.x, n_raw = n_raw_next) {
+        n_raw_next = raw_count<SPARSE>(a, w + gridDim.x);
+        const ItemList<SPARSE> it = item_list<SPARSE>(a, w, n_raw);
         if (it.n == 0) continue;
         if (!ptx::mbar_wait(bar(C::B_QFULL), iq & 1, abort_flag, a.timeout_ns, kErrTimeout)) {
           ok = false;
@@ -357,9 +362,10 @@ __global__ void __launch_bounds__(384, 1)
       const uint32_t vlo = ptx::sdesc_sw128_lo(sb + C::OFF_V, C::KV_CHUNK);
       int g = 0;
       bool ok = true;
-      for (int w = blockIdx.x; ok && w < n_items; w += gridDim.x) {
-        const int h = w / a.nqb, qi = w - h * a.nqb;
-        const ItemList<SPARSE> it = item_list<SPARSE>(a, h, qi);
+      int n_raw = raw_count<SPARSE>(a, blockIdx.x), n_raw_next = 0;
+      for (int w = blockIdx.x; ok && w < n_items; w += gridDim.x, n_raw = n_raw_next) {
+        n_raw_next = raw_count<SPARSE>(a, w + gridDim.x);
+        const ItemList<SPARSE> it = item_list<SPARSE>(a, w, n_raw);
         for (int jj = 0; jj < it.n; ++jj, ++g) {
           const int b = g & 1;
           const int vs = g % C::VS;
@@ -395,9 +401,11 @@ __global__ void __launch_bounds__(384, 1)
     const int s_off = half * HALF;  // first S column of my half row
     int g = 0;
     bool ok = true;
-    for (int w = blockIdx.x; ok && w < n_items; w += gridDim.x) {
+    int n_raw = raw_count<SPARSE>(a, blockIdx.x), n_raw_next = 0;
+    for (int w = blockIdx.x; ok && w < n_items; w += gridDim.x, n_raw = n_raw_next) {
+      n_raw_next = raw_count<SPARSE>(a, w + gridDim.x);
       const int h = w / a.nqb, qi = w - h * a.nqb;
-      const ItemList<SPARSE> it = item_list<SPARSE>(a, h, qi);
+      const ItemList<SPARSE> it = item_list<SPARSE>(a, w, n_raw);
       const int grow = qi * a.bq + r;
       const bool row_valid = (r < a.bq) && (grow < a.L);
       // my contiguous half row of O: D/2 bf16 = D bytes
