@@ -264,14 +264,16 @@ __global__ void __launch_bounds__(384, 1)
         for (int c = 0; c < C::DCH; ++c)
           ptx::tma_load_3d(sb + C::OFF_Q + c * C::Q_CHUNK, &tm_q, bar(C::B_QFULL), c * 64, qi * a.bq, h);
         ++iq;
-        int prev = -1;
+        // list entries are read one tile ahead, off the copy-issue path
+        int prev = -1, raw_next = it.raw(0);
         for (int jj = 0; jj < it.n; ++jj, ++g) {
+          const int raw = raw_next;
+          if (jj + 1 < it.n) raw_next = it.raw(jj + 1);
           if constexpr (SPARSE) {
-            const int j = it.raw(jj);
-            if (j < 0 || j >= a.nkb || j <= prev) ptx::record_error(kErrBadPattern);
-            prev = j;
+            if (raw < 0 || raw >= a.nkb || raw <= prev) ptx::record_error(kErrBadPattern);
+            prev = raw;
           }
-          const int j = it.block(jj);
+          const int j = (raw >= 0 && raw < a.nkb) ? raw : 0;
           const int ks = g % C::KS;
           if (g >= C::KS &&
               !ptx::mbar_wait(bar(C::B_KEMPTY + ks), (g / C::KS - 1) & 1, abort_flag, a.timeout_ns, kErrTimeout)) {
