@@ -484,15 +484,21 @@ def time_one_op(args, wl, dev, rank):
 
 
 def load_traffic(workload):
-    """DRAM bytes per launch from the committed ncu summary, when one exists
-    for the current kernels (profiles/traffic.json)."""
+    """DRAM bytes per launch from the committed ncu capture (profiles/traffic.json),
+    used only while the attention kernel source is the one that was captured."""
+    import hashlib
     path = os.path.join(ROOT, "profiles", "traffic.json")
+    src = os.path.join(ROOT, "block_sparse_bidirectional_select_b200", "csrc", "attn_kernel.cuh")
     try:
         with open(path) as f:
             t = json.load(f)
-        return t.get(workload, {})
+        with open(src, "rb") as f:
+            sha = hashlib.sha256(f.read()).hexdigest()
     except (OSError, ValueError):
         return {}
+    if t.get("attn_kernel_sha256") != sha:
+        return {}
+    return t.get(workload, {})
 
 
 if __name__ == "__main__":
