@@ -195,6 +195,29 @@ def cpu_oracle_sample(wl, q, k, v, budget_s, rng_seed=0):
             "ms_per_step_extrapolated": run_s * 1e3}
 
 
+# ----------------------------------------------------------------- ranks
+
+def rank_workload(wl, rank):
+    """Each rank runs its own independent layer: same shapes, its own seed."""
+    return wl.scaled(seed=wl.seed + rank)
+
+
+def reduce_max(x, world, device):
+    """Max of a host float over all ranks (identity for one rank)."""
+    if world == 1:
+        return float(x)
+    import torch.distributed as dist
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_value(flops_per_step, steps, world, total_ms):
+    """Whole-job throughput in TFLOP/s: every rank's steps over the slowest
+    rank's time (weak scaling: each rank does the same work)."""
+    return flops_per_step * steps * world / (total_ms * 1e-3) / 1e12
+
+
 def run_reference(args, rank, world):
     if rank != 0:
         return 0
@@ -277,24 +300,20 @@ def main():
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
     if world > 1:
-        dist.init_process_group("nccl", device_id=dev, timeout=datetime.timedelta(seconds=900))
+        dist.init_process_group("nccl", device_id=dev, timeout=datetime.timedelta(seconds=300))
 
     def barrier():
         if world > 1:
             dist.barrier()
 
     def max_over_ranks(x):
-        if world == 1:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+        return reduce_max(x, world, dev)
 
     wl = WORKLOADS[args.workload]
     if args.op != "run":
         return time_one_op(args, wl, dev, rank)
     log(f"[rank {rank}] inputs for {wl.name}")
-    q_cpu, k_cpu, v_cpu = make_inputs(wl.scaled(seed=wl.seed + rank))
+    q_cpu, k_cpu, v_cpu = make_inputs(rank_workload(wl, rank))
     q, k, v = (t.to(dev) for t in (q_cpu, k_cpu, v_cpu))
     stream = torch.cuda.current_stream()
     peaks, peak_src = load_peaks()
@@ -338,7 +357,7 @@ def main():
     total_ms = max_over_ranks(s_ev.elapsed_time(e_ev))
     sp.device_check()
     ms_per_step = total_ms / args.steps
-    value = acc["flops"] * args.steps * world / (total_ms * 1e-3) / 1e12
+    value = job_value(acc["flops"], args.steps, world, total_ms)
 
     per_kind = {0: [], 1: [], 2: []}
     for run in step_ms:
@@ -416,7 +435,7 @@ def main():
         torch.cuda.synchronize()
         bi = 3 * q.numel() * q.element_size()
         bo = o.numel() * o.element_size() + lse.numel() * lse.element_size()
-        e2e = {"value": acc["flops"] * args.steps * world / (e2e_ms * 1e-3) / 1e12, "unit": UNIT,
+        e2e = {"value": job_value(acc["flops"], args.steps, world, e2e_ms), "unit": UNIT,
                "h2d_bytes_per_step": bi, "d2h_bytes_per_step": bo, "ms_per_step": e2e_ms / args.steps}
 
     cpu = None

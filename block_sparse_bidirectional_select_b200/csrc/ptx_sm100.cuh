@@ -372,29 +372,6 @@ __device__ __forceinline__ float ex2(float x) {
   return y;
 }
 
-// 2^x evaluated on the FMA pipe instead of MUFU, for x <= 127 (smaller x is
-// clamped to -125, i.e. results below 2^-125 are returned as ~2^-125).
-// Cody-Waite range reduction: adding 1.5*2^23 rounds x to the nearest integer
-// n, which then sits in the low mantissa bits of t; f = x - n is in
-// [-0.5, 0.5]. 2^f comes from a cubic fitted here by iteratively reweighted
-// least squares on Chebyshev nodes (maximum relative error 7.5e-5 on
-// [-0.5, 0.5], evaluated in fp32), and 2^n is applied by adding n to the
-// exponent field: the low bits of t shifted left by 23 are exactly n << 23.
-constexpr float kExp2C0 = 0.9999280571937561f;
-constexpr float kExp2C1 = 0.6932609677314758f;
-constexpr float kExp2C2 = 0.2426111251115799f;
-constexpr float kExp2C3 = 0.0551716648042202f;
-__device__ __forceinline__ float exp2_fma(float x) {
-  x = fmaxf(x, -125.0f);
-  const float t = x + 12582912.0f;
-  const float n = t - 12582912.0f;
-  const float f = x - n;
-  float p = fmaf(kExp2C3, f, kExp2C2);
-  p = fmaf(p, f, kExp2C1);
-  p = fmaf(p, f, kExp2C0);
-  return __uint_as_float(__float_as_uint(p) + (__float_as_uint(t) << 23));
-}
-
 // Hardware base-2 logarithm (MUFU).
 __device__ __forceinline__ float lg2(float x) {
   float y;
