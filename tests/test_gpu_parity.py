@@ -85,6 +85,33 @@ def test_sparse_parity_given_pattern(d, bq, bk):
         assert torch.isneginf(lse[h, rows]).all()
 
 
+@pytest.mark.parametrize("d,bq,bk", [(64, 64, 64), (128, 128, 128)])
+def test_many_items_per_persistent_cta(d, bq, bk):
+    """More work items than SMs, so every CTA walks several (head, query
+    block) items and its pipelines cross item boundaries: ragged L, random
+    list lengths including empty lists between non-empty ones, then a dense
+    pass over the same shape."""
+    H, L = 8, 4000
+    q, k, v, scale = _inputs(H, L, d, seed=77 + d)
+    nqb, nkb = -(-L // bq), -(-L // bk)
+    assert H * nqb > 148 * (2 if bq == 64 else 1)
+    rng = np.random.default_rng(4242 + d)
+    kv_idx, kv_count = _random_pattern(H, nqb, nkb, nkb, rng)
+    qc, kc, vc = _cuda(q, k, v)
+    o, lse = sp.block_sparse_attn(qc, kc, vc, kv_idx, kv_count, bq=bq, bk=bk)
+    od, ld = sp.dense_attn(qc, kc, vc, bq=bq, bk=bk)
+    sp.device_check()
+    lists, cnt = pattern_lists(kv_idx, kv_count)
+    qh, kh, vh = f64(q), f64(k), f64(v)
+    o_ref = np.empty(qh.shape)
+    l_ref = np.empty(qh.shape[:2])
+    for h in range(H):
+        o_ref[h], l_ref[h] = O.masked_attention(qh[h], kh[h], vh[h], scale, lists[h], cnt[h], bq, bk)
+    assert_o_lse(o, lse, o_ref, l_ref, f"sparse, many items, d={d} bq={bq}")
+    od_ref, ld_ref = oracle_dense_heads(q, k, v, scale)
+    assert_o_lse(od, ld, od_ref, ld_ref, f"dense, many items, d={d} bq={bq}")
+
+
 @pytest.mark.parametrize("d,bk", [(64, 64), (128, 128), (128, 64)])
 def test_keep_all_bitwise_equals_dense(d, bk):
     H, L, bq = 2, 1024 + 64, 128
