@@ -19,7 +19,8 @@ the pages define (citations name the page title and the part of the page):
   a head-adaptive global budget compresses concentrated heads harder;
   "90% sparsity" means a keep ratio of 0.10.
 * PulseCol: Periodically Refreshed Column-Sparse Attention for Accelerating
-  Diffusion Language Models, abstract -- the same periodic-refresh schedule.
+  Diffusion Language Models, abstract -- the same periodic-refresh schedule,
+  and column-level (per key position) instead of block-level sparsity.
 
 Where the pages leave a step open, the reading taken is stated in the function
 docstring (rule for what is scored, rounding of k, tie-break, list order, the
@@ -390,6 +391,102 @@ def run_steps(q, k, v, scale, bq, bk, keep_ratio, budget, T, warmup_frac,
                 o[h], lse[h] = masked_attention(q[h], k[h], v[h], scale,
                                                 pattern["kv_idx"][h],
                                                 pattern["kv_count"][h], bq, bk)
+    return o, lse, kinds, pattern
+
+
+# --------------------------------------------------------------------------
+# O7  column-sparse attention (PulseCol)
+# --------------------------------------------------------------------------
+
+
+def column_keep(L, keep_ratio):
+    """Number of key columns kept per head: clamp(ceil(rho*L), 1, L).
+
+    PulseCol abstract: column-level sparsity instead of block-level. Reading
+    taken (the page gives no count rule): the keep ratio rho applies to the
+    L key columns of a head, rounded up as for blocks (``uniform_keep``)."""
+    rho = float(np.float32(keep_ratio))
+    return min(max(math.ceil(rho * L - ROUND_EPS), 1), L)
+
+
+def column_mass(q, k, scale, lse, chunk=1024):
+    """Full-attention probability mass of every key column of one head:
+        A[c] = sum over all rows r of p_rc,  p_rc = exp(scale*<q_r,k_c> - lse_r).
+
+    PulseCol abstract: important attention interactions are kept at column
+    granularity, identified from an early full pass. Reading taken for what is
+    scored: the column analogue of the block mass, i.e. the post-softmax mass a
+    key receives from all queries of the head. Rows are summed in ascending
+    order, ``chunk`` rows at a time. Returns [Lk]."""
+    q = np.asarray(q, dtype=np.float64)
+    k = np.asarray(k, dtype=np.float64)
+    lse = np.asarray(lse, dtype=np.float64)
+    out = np.zeros(k.shape[0])
+    for r0 in range(0, q.shape[0], chunk):
+        r1 = min(r0 + chunk, q.shape[0])
+        s = float(scale) * (q[r0:r1] @ k.T)
+        out += np.exp(s - lse[r0:r1, None]).sum(axis=0)
+    return out
+
+
+def topk_columns(col_mass, k):
+    """The k key columns of largest mass of one head, ties to the lower
+    column index, emitted in ascending index order (the block rule of
+    ``topk_blocks`` at column granularity)."""
+    m = np.asarray(col_mass, dtype=np.float64)
+    order = np.lexsort((np.arange(len(m)), -m))
+    return np.sort(order[:k]).astype(np.int32)
+
+
+def column_sparse_attention(q, k, v, scale, cols):
+    """Every query row of one head attends to the kept key columns only, in
+    ascending column order: softmax attention over k[cols], v[cols]."""
+    cols = np.asarray(cols, dtype=np.int64)
+    return softmax_attention(q, np.asarray(k)[cols], np.asarray(v)[cols], scale)
+
+
+def select_columns(q, k, v, scale, keep_ratio):
+    """One full-attention pass that also yields the per-head column pattern
+    (PulseCol abstract: the sparse pattern is identified at an early denoising
+    step). q, k, v are [H, L, d]. Returns dict with o [H,L,d], lse [H,L],
+    col_mass [H,L], cols [H, kc] (ascending per head)."""
+    H, L, _ = q.shape
+    kc = column_keep(L, keep_ratio)
+    o = np.empty(q.shape)
+    lse = np.empty((H, L))
+    mass = np.empty((H, L))
+    cols = np.empty((H, kc), dtype=np.int32)
+    for h in range(H):
+        o[h], lse[h] = dense_attention(q[h], k[h], v[h], scale)
+        mass[h] = column_mass(q[h], k[h], scale, lse[h])
+        cols[h] = topk_columns(mass[h], kc)
+    return dict(o=o, lse=lse, col_mass=mass, cols=cols)
+
+
+def run_steps_columns(q, k, v, scale, keep_ratio, T, warmup_frac, refresh_every=0):
+    """The denoising loop with the column-sparse pattern (PulseCol abstract:
+    the pattern is identified early, reused, and refreshed at a few
+    intermediate steps): the step kinds of ``schedule``; SELECT runs
+    ``select_columns``, SPARSE ``column_sparse_attention`` with the cached
+    columns. Returns (o, lse, kinds, pattern) of the last step."""
+    kinds = schedule(T, warmup_frac, refresh_every)
+    H, L, _ = q.shape
+    pattern = None
+    o = lse = None
+    for t in range(T):
+        if kinds[t] == DENSE:
+            o = np.empty(q.shape)
+            lse = np.empty((H, L))
+            for h in range(H):
+                o[h], lse[h] = dense_attention(q[h], k[h], v[h], scale)
+        elif kinds[t] == SELECT:
+            pattern = select_columns(q, k, v, scale, keep_ratio)
+            o, lse = pattern["o"], pattern["lse"]
+        else:
+            o = np.empty(q.shape)
+            lse = np.empty((H, L))
+            for h in range(H):
+                o[h], lse[h] = column_sparse_attention(q[h], k[h], v[h], scale, pattern["cols"][h])
     return o, lse, kinds, pattern
 
 
