@@ -11,6 +11,12 @@ device memory and streams.
     block_sparse_attn(q, k, v, kv_idx, kv_count) -> (o, lse)
     run_steps(q, k, v, T, warmup_frac, ...)  -> RunResult (o, lse, kinds, step_ms, pattern)
 
+Column-sparse path (per-head kept key columns shared by all queries):
+
+    select_columns(q, k, v, keep)            -> ColumnPattern (o, lse, cols, col_mass)
+    column_sparse_attn(q, k, v, cols)        -> (o, lse)
+    run_steps_columns(q, k, v, T, warmup_frac, ...) -> RunResult (kv_idx holds cols [H, kc])
+
 q, k, v are [H, L, d] bf16 CUDA tensors (d in {64, 128}); o is [H, L, d] bf16,
 lse [H, L] fp32 natural log; kv_idx [H, nqb, kv_stride] int32 and kv_count
 [H, nqb] int32 hold the per-(head, query block) kept key blocks, ascending.
@@ -29,7 +35,8 @@ from ._lib import (BUDGET_ENTROPY, BUDGET_UNIFORM, STEP_DENSE, STEP_SELECT,  # n
 
 __all__ = ["dense_attn", "select_pattern", "block_sparse_attn", "run_steps", "workspace_bytes",
            "uniform_keep", "schedule", "device_check", "version", "SparsedError", "Pattern",
-           "RunResult", "default_scale"]
+           "RunResult", "default_scale", "column_keep", "column_workspace_bytes", "select_columns",
+           "column_sparse_attn", "run_steps_columns", "ColumnPattern"]
 
 
 def _ptr(t: torch.Tensor | None):
@@ -210,3 +217,93 @@ def run_steps(q, k, v, T, warmup_frac=0.2, keep=0.1, budget="uniform", refresh_e
         _ptr(ws), ws.numel(), _stream(stream))
     check(rc, "sparsed_run_steps")
     return RunResult(out, lse, list(kinds[:T]), None if ms is None else list(ms[:T]), kv_idx, kv_count)
+
+
+# ---------------------------------------------------------------- column path
+
+def column_keep(L: int, keep: float) -> int:
+    kc = ctypes.c_int()
+    check(_lib.load().sparsed_column_keep(L, keep, ctypes.byref(kc)), "sparsed_column_keep")
+    return kc.value
+
+
+def column_workspace_bytes(H: int, L: int, d: int, kc: int) -> int:
+    n = ctypes.c_size_t()
+    check(_lib.load().sparsed_column_workspace_bytes(H, L, d, kc, ctypes.byref(n)),
+          "sparsed_column_workspace_bytes")
+    return n.value
+
+
+def _col_workspace(q, kc, workspace):
+    H, L, d = q.shape
+    need = column_workspace_bytes(H, L, d, kc)
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    return workspace
+
+
+@dataclass
+class ColumnPattern:
+    o: torch.Tensor
+    lse: torch.Tensor
+    cols: torch.Tensor              # [H, kc] int32, ascending per head
+    col_mass: torch.Tensor | None   # [H, L] fp32
+
+
+def select_columns(q, k, v, keep=0.1, scale=None, bq=128, bk=128, return_mass=False, workspace=None,
+                   stream=None) -> ColumnPattern:
+    """Full-attention pass plus per-head column selection (column mass, top-k)."""
+    H, L, d = _check_qkv(q, k, v)
+    scale = default_scale(d) if scale is None else scale
+    kc = column_keep(L, keep) if L > 0 else 1
+    out, lse = _alloc_out(q, None, None)
+    cols = torch.full((H, kc), -1, dtype=torch.int32, device=q.device)
+    mass = torch.empty((H, L), dtype=torch.float32, device=q.device) if return_mass else None
+    ws = _col_workspace(q, kc, workspace)
+    rc = _lib.load().sparsed_select_columns(
+        _ptr(q), _ptr(k), _ptr(v), H, L, d, scale, bq, bk, keep, _ptr(out), _ptr(lse), _ptr(cols), kc,
+        _ptr(mass), _ptr(ws), ws.numel(), _stream(stream))
+    check(rc, "sparsed_select_columns")
+    return ColumnPattern(out, lse, cols, mass)
+
+
+def column_sparse_attn(q, k, v, cols, scale=None, bq=128, bk=128, out=None, lse=None, workspace=None,
+                       stream=None):
+    """Attention of every query over its head's kept columns: returns (o, lse)."""
+    H, L, d = _check_qkv(q, k, v)
+    scale = default_scale(d) if scale is None else scale
+    if cols.dtype != torch.int32 or not cols.is_contiguous() or cols.device != q.device or cols.dim() != 2 \
+            or cols.shape[0] != H:
+        raise ValueError(f"cols must be a contiguous [H, kc] int32 tensor on {q.device}")
+    kc = cols.shape[1]
+    out, lse = _alloc_out(q, out, lse)
+    ws = _col_workspace(q, kc, workspace)
+    rc = _lib.load().sparsed_column_sparse_attn(
+        _ptr(q), _ptr(k), _ptr(v), H, L, d, scale, bq, bk, _ptr(cols), kc, kc, _ptr(out), _ptr(lse),
+        _ptr(ws), ws.numel(), _stream(stream))
+    check(rc, "sparsed_column_sparse_attn")
+    return out, lse
+
+
+def run_steps_columns(q, k, v, T, warmup_frac=0.2, keep=0.1, refresh_every=0, scale=None, bq=128, bk=128,
+                      start_step=0, cols=None, time_steps=False, out=None, lse=None, workspace=None,
+                      stream=None) -> RunResult:
+    """The denoising loop with the column pattern: dense warm-up, column
+    selection at the switch (and at refreshes), column-sparse attention
+    afterwards. The result's kv_idx holds the columns [H, kc]."""
+    H, L, d = _check_qkv(q, k, v)
+    scale = default_scale(d) if scale is None else scale
+    kc = column_keep(L, keep) if L > 0 else 1
+    have = 1 if cols is not None else 0
+    if cols is None:
+        cols = torch.full((H, kc), -1, dtype=torch.int32, device=q.device)
+    out, lse = _alloc_out(q, out, lse)
+    ws = _col_workspace(q, kc, workspace)
+    kinds = (ctypes.c_int8 * max(T, 1))()
+    ms = (ctypes.c_float * max(T, 1))() if time_steps else None
+    rc = _lib.load().sparsed_run_steps_columns(
+        _ptr(q), _ptr(k), _ptr(v), H, L, d, scale, bq, bk, keep, T, warmup_frac, refresh_every, start_step,
+        have, _ptr(cols), cols.shape[1], _ptr(out), _ptr(lse), ctypes.cast(kinds, ctypes.c_void_p),
+        None if ms is None else ctypes.cast(ms, ctypes.c_void_p), _ptr(ws), ws.numel(), _stream(stream))
+    check(rc, "sparsed_run_steps_columns")
+    return RunResult(out, lse, list(kinds[:T]), None if ms is None else list(ms[:T]), cols, None)

@@ -46,6 +46,12 @@ SIGNATURES = {
                                             _I, _P, _P, _P]),
     "sparsed_run_steps": (_I, [_P, _P, _P, _I, _I, _I, _F, _I, _I, _F, _I, _I, _F, _I, _I, _I, _P, _P,
                                _I, _P, _P, _P, _P, _P, _SZ, _P]),
+    "sparsed_column_keep": (_I, [_I, _F, ctypes.POINTER(_I)]),
+    "sparsed_column_workspace_bytes": (_I, [_I, _I, _I, _I, ctypes.POINTER(_SZ)]),
+    "sparsed_select_columns": (_I, [_P, _P, _P, _I, _I, _I, _F, _I, _I, _F, _P, _P, _P, _I, _P, _P, _SZ, _P]),
+    "sparsed_column_sparse_attn": (_I, [_P, _P, _P, _I, _I, _I, _F, _I, _I, _P, _I, _I, _P, _P, _P, _SZ, _P]),
+    "sparsed_run_steps_columns": (_I, [_P, _P, _P, _I, _I, _I, _F, _I, _I, _F, _I, _F, _I, _I, _I, _P, _I,
+                                       _P, _P, _P, _P, _P, _SZ, _P]),
 }
 
 _lib = None

@@ -55,6 +55,7 @@ namespace sparsed {
 
 struct AttnArgs {
   int H, L, bq, nqb, nkb;
+  int Lk;                    // keys (== L, except over the gathered columns of a column pattern)
   float scale_log2;          // scale * log2(e)
   const int32_t* kv_idx;     // sparse mode only
   const int32_t* kv_count;   // sparse mode only
@@ -424,7 +425,7 @@ __global__ void __launch_bounds__(384, 1)
       float l = 0.f;                          // running sum of my half row
       // only a list that can hold the ragged last key block needs its entries
       // here; they are read one tile ahead, off the critical path
-      const bool ragged = SPARSE && (a.L % BK) != 0;
+      const bool ragged = SPARSE && (a.Lk % BK) != 0;
       int blk_next = ragged ? it.block(0) : 0;
       for (int jj = 0; jj < it.n; ++jj, ++g) {
         int blk = jj;
@@ -453,7 +454,7 @@ __global__ void __launch_bounds__(384, 1)
           }
         }
         // ragged last key block: keys past L do not exist
-        const int valid = a.L - blk * BK - s_off;
+        const int valid = a.Lk - blk * BK - s_off;
         if (valid < HALF) {
 #pragma unroll
           for (int c = 0; c < HALF; ++c)

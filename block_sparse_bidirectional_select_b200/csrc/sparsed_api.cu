@@ -16,6 +16,7 @@
 #include "sparsed.h"
 #include "attn_kernel.cuh"
 #include "select_kernels.cuh"
+#include "column_kernels.cuh"
 
 using namespace sparsed;
 
@@ -132,6 +133,7 @@ struct Problem {
   uint16_t* O;
   float* LSE;
   int H, L, d, bq, bk, nqb, nkb;
+  int Lk;  // rows of K and V: L, or the kept columns of a column pattern
   float scale;
 };
 
@@ -152,11 +154,12 @@ int launch_attn_t(const Problem& p, const int32_t* kv_idx, const int32_t* kv_cou
   if (regs * C::THREADS < C::REGS_SOFTMAX * 256 + C::REGS_OTHER * 128) return SPARSED_ERR_UNSUPPORTED;
   CUtensorMap tq, tk, tv;
   SP_TRY(make_map(&tq, p.Q, p.H, p.L, D, 128));
-  SP_TRY(make_map(&tk, p.K, p.H, p.L, D, BK));
-  SP_TRY(make_map(&tv, p.V, p.H, p.L, D, BK));
+  SP_TRY(make_map(&tk, p.K, p.H, p.Lk, D, BK));
+  SP_TRY(make_map(&tv, p.V, p.H, p.Lk, D, BK));
   AttnArgs a;
   a.H = p.H;
   a.L = p.L;
+  a.Lk = p.Lk;
   a.bq = p.bq;
   a.nqb = p.nqb;
   a.nkb = p.nkb;
@@ -224,6 +227,91 @@ int launch_mass(const Problem& p, float* mass, cudaStream_t st) {
   return SPARSED_ERR_UNSUPPORTED;
 }
 
+// ---- column path (PulseCol abstract): column mass, top-k columns, gather,
+// then the dense attention kernel over the gathered keys
+
+template <int D>
+int launch_col_mass_t(const Problem& p, float* mass, cudaStream_t st) {
+  using C = ColMassCfg<D>;
+  CUtensorMap tq, tk;
+  SP_TRY(make_map(&tq, p.Q, p.H, p.L, D, C::N));
+  SP_TRY(make_map(&tk, p.K, p.H, p.L, D, C::M));
+  ColMassArgs a;
+  a.H = p.H;
+  a.L = p.L;
+  a.Lk = p.L;
+  a.scale_log2 = p.scale * 1.44269504088896340736f;
+  a.lse = p.LSE;
+  a.mass = mass;
+  a.timeout_ns = kWaitTimeoutNs;
+  auto kern = column_mass_kernel<D>;
+  SP_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES));
+  kern<<<dim3(static_cast<unsigned>(cdiv(p.L, C::M)), p.H), 256, C::SMEM_BYTES, st>>>(tq, tk, a);
+  SP_CUDA(cudaGetLastError());
+  return SPARSED_OK;
+}
+
+int launch_col_mass(const Problem& p, float* mass, cudaStream_t st) {
+  if (p.d == 64) return launch_col_mass_t<64>(p, mass, st);
+  if (p.d == 128) return launch_col_mass_t<128>(p, mass, st);
+  return SPARSED_ERR_UNSUPPORTED;
+}
+
+struct ColWorkspace {
+  size_t mass, ksel, vsel, total;
+};
+
+ColWorkspace col_ws_layout(int H, int L, int d, int kc) {
+  ColWorkspace w;
+  w.mass = 0;
+  w.ksel = align256(static_cast<size_t>(H) * L * sizeof(float));
+  w.vsel = w.ksel + align256(static_cast<size_t>(H) * kc * d * 2);
+  w.total = w.vsel + align256(static_cast<size_t>(H) * kc * d * 2);
+  return w;
+}
+
+int check_column_args(const Problem& p, int kc, const int32_t* cols, int col_stride, const void* workspace,
+                      size_t ws_bytes) {
+  if (!cols || kc < 1 || kc > p.L || col_stride < kc) return SPARSED_ERR_INVALID_ARG;
+  if (static_cast<long long>(p.H) * col_stride >= (1ll << 31)) return SPARSED_ERR_UNSUPPORTED;
+  if (!workspace || ws_bytes < col_ws_layout(p.H, p.L, p.d, kc).total) return SPARSED_ERR_WORKSPACE;
+  if (reinterpret_cast<uintptr_t>(workspace) % 256 != 0) return SPARSED_ERR_INVALID_ARG;
+  return SPARSED_OK;
+}
+
+// After the dense pass wrote O and LSE: column mass -> the kc columns per head.
+int select_columns_after_dense(const Problem& p, int kc, int32_t* cols, int col_stride, float* mass_out,
+                               void* workspace, cudaStream_t st) {
+  float* mass = mass_out ? mass_out
+                         : reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) +
+                                                    col_ws_layout(p.H, p.L, p.d, kc).mass);
+  SP_TRY(launch_col_mass(p, mass, st));
+  topk_columns_kernel<<<p.H, 1024, 0, st>>>(mass, p.L, kc, cols, col_stride);
+  SP_CUDA(cudaGetLastError());
+  return SPARSED_OK;
+}
+
+// Attention of every query over the head's kc kept columns: gather them, then
+// run the dense kernel with kc keys.
+int column_attn(const Problem& p, const int32_t* cols, int kc, int col_stride, void* workspace, cudaStream_t st) {
+  const ColWorkspace w = col_ws_layout(p.H, p.L, p.d, kc);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  uint16_t* ksel = reinterpret_cast<uint16_t*>(ws + w.ksel);
+  uint16_t* vsel = reinterpret_cast<uint16_t*>(ws + w.vsel);
+  const int row_u4 = p.d * 2 / 16;
+  const long per_head = static_cast<long>(kc) * row_u4;
+  gather_rows_kernel<<<dim3(static_cast<unsigned>(cdiv(per_head, 256)), p.H), 256, 0, st>>>(
+      reinterpret_cast<const uint4*>(p.K), reinterpret_cast<const uint4*>(p.V), cols, p.L, kc, col_stride, row_u4,
+      reinterpret_cast<uint4*>(ksel), reinterpret_cast<uint4*>(vsel));
+  SP_CUDA(cudaGetLastError());
+  Problem g = p;
+  g.K = ksel;
+  g.V = vsel;
+  g.Lk = kc;
+  g.nkb = static_cast<int>(cdiv(kc, p.bk));
+  return launch_attn(g, false, nullptr, nullptr, 0, st);
+}
+
 struct Workspace {
   size_t grid, ent, scratch, headk, total;
 };
@@ -285,6 +373,7 @@ int prepare(const uint16_t* Q, const uint16_t* K, const uint16_t* V, int H, int 
   p->bk = bk;
   p->nqb = static_cast<int>(cdiv(L, bq));
   p->nkb = static_cast<int>(cdiv(L, bk));
+  p->Lk = L;
   p->scale = scale;
   return SPARSED_OK;
 }
@@ -470,6 +559,117 @@ int sparsed_run_steps(const uint16_t* Q, const uint16_t* K, const uint16_t* V, i
         break;
       default:
         rc = launch_attn(p, true, kv_idx, kv_count, kv_stride, st);
+        break;
+    }
+    if (!ev.empty() && rc == SPARSED_OK) {
+      cudaError_t e = cudaEventRecord(ev[t - start_step + 1], st);
+      if (e != cudaSuccess) rc = fail_cuda(e);
+    }
+  }
+  if (!ev.empty()) {
+    if (rc == SPARSED_OK) {
+      cudaError_t e = cudaEventSynchronize(ev.back());
+      if (e != cudaSuccess) rc = fail_cuda(e);
+      for (int t = start_step; t < T && rc == SPARSED_OK; ++t) {
+        float ms = 0.f;
+        e = cudaEventElapsedTime(&ms, ev[t - start_step], ev[t - start_step + 1]);
+        if (e != cudaSuccess) rc = fail_cuda(e);
+        step_ms[t] = ms;
+      }
+    }
+    for (auto& e : ev)
+      if (e) cudaEventDestroy(e);
+  }
+  return rc;
+}
+
+int sparsed_column_keep(int L, float keep_ratio, int* kc) {
+  if (!kc || L < 1 || !(keep_ratio > 0.f && keep_ratio <= 1.f)) return SPARSED_ERR_INVALID_ARG;
+  *kc = uniform_k(L, keep_ratio);
+  return SPARSED_OK;
+}
+
+int sparsed_column_workspace_bytes(int H, int L, int d, int kc, size_t* bytes) {
+  if (!bytes || H < 0 || L < 0 || kc < 0 || kc > L) return SPARSED_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return SPARSED_ERR_UNSUPPORTED;
+  *bytes = col_ws_layout(H, L, d, kc).total;
+  return SPARSED_OK;
+}
+
+int sparsed_select_columns(const uint16_t* Q, const uint16_t* K, const uint16_t* V, int H, int L, int d,
+                           float scale, int bq, int bk, float keep_ratio, uint16_t* O, float* LSE, int32_t* cols,
+                           int col_stride, float* col_mass, void* workspace, size_t workspace_bytes, void* stream) {
+  Problem p;
+  bool empty = false;
+  SP_TRY(prepare(Q, K, V, H, L, d, scale, bq, bk, O, LSE, &p, &empty));
+  if (empty) return SPARSED_OK;
+  if (!(keep_ratio > 0.f && keep_ratio <= 1.f)) return SPARSED_ERR_INVALID_ARG;
+  const int kc = uniform_k(L, keep_ratio);
+  SP_TRY(check_column_args(p, kc, cols, col_stride, workspace, workspace_bytes));
+  SP_TRY(require_sm100());
+  SP_TRY(get_encoder());
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  SP_TRY(launch_attn(p, false, nullptr, nullptr, 0, st));
+  return select_columns_after_dense(p, kc, cols, col_stride, col_mass, workspace, st);
+}
+
+int sparsed_column_sparse_attn(const uint16_t* Q, const uint16_t* K, const uint16_t* V, int H, int L, int d,
+                               float scale, int bq, int bk, const int32_t* cols, int kc, int col_stride,
+                               uint16_t* O, float* LSE, void* workspace, size_t workspace_bytes, void* stream) {
+  Problem p;
+  bool empty = false;
+  SP_TRY(prepare(Q, K, V, H, L, d, scale, bq, bk, O, LSE, &p, &empty));
+  if (empty) return SPARSED_OK;
+  SP_TRY(check_column_args(p, kc, cols, col_stride, workspace, workspace_bytes));
+  SP_TRY(require_sm100());
+  SP_TRY(get_encoder());
+  return column_attn(p, cols, kc, col_stride, workspace, static_cast<cudaStream_t>(stream));
+}
+
+int sparsed_run_steps_columns(const uint16_t* Q, const uint16_t* K, const uint16_t* V, int H, int L, int d,
+                              float scale, int bq, int bk, float keep_ratio, int T, float warmup_frac,
+                              int refresh_every, int start_step, int have_pattern, int32_t* cols, int col_stride,
+                              uint16_t* O, float* LSE, int8_t* step_kind, float* step_ms, void* workspace,
+                              size_t workspace_bytes, void* stream) {
+  if (T < 0 || start_step < 0 || start_step > T) return SPARSED_ERR_INVALID_ARG;
+  if (!(keep_ratio > 0.f && keep_ratio <= 1.f)) return SPARSED_ERR_INVALID_ARG;
+  std::vector<int8_t> kinds(static_cast<size_t>(T) + 1);
+  SP_TRY(sparsed_schedule(T, warmup_frac, refresh_every, kinds.data()));
+  if (step_kind && T > 0) std::memcpy(step_kind, kinds.data(), static_cast<size_t>(T));
+  if (step_ms)
+    for (int t = 0; t < T; ++t) step_ms[t] = 0.f;
+  Problem p;
+  bool empty = false;
+  SP_TRY(prepare(Q, K, V, H, L, d, scale, bq, bk, O, LSE, &p, &empty));
+  if (empty) return SPARSED_OK;
+  bool pattern_ready = have_pattern != 0;
+  for (int t = start_step; t < T; ++t) {
+    if (kinds[t] == SPARSED_STEP_SELECT) pattern_ready = true;
+    if (kinds[t] == SPARSED_STEP_SPARSE && !pattern_ready) return SPARSED_ERR_INVALID_ARG;
+  }
+  const int kc = uniform_k(L, keep_ratio);
+  if (start_step < T) SP_TRY(check_column_args(p, kc, cols, col_stride, workspace, workspace_bytes));
+  SP_TRY(require_sm100());
+  SP_TRY(get_encoder());
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  std::vector<cudaEvent_t> ev;
+  if (step_ms && start_step < T) {
+    ev.resize(static_cast<size_t>(T - start_step) + 1, nullptr);
+    for (auto& e : ev) SP_CUDA(cudaEventCreate(&e));
+    SP_CUDA(cudaEventRecord(ev[0], st));
+  }
+  int rc = SPARSED_OK;
+  for (int t = start_step; t < T && rc == SPARSED_OK; ++t) {
+    switch (kinds[t]) {
+      case SPARSED_STEP_DENSE:
+        rc = launch_attn(p, false, nullptr, nullptr, 0, st);
+        break;
+      case SPARSED_STEP_SELECT:
+        rc = launch_attn(p, false, nullptr, nullptr, 0, st);
+        if (rc == SPARSED_OK) rc = select_columns_after_dense(p, kc, cols, col_stride, nullptr, workspace, st);
+        break;
+      default:
+        rc = column_attn(p, cols, kc, col_stride, workspace, st);
         break;
     }
     if (!ev.empty() && rc == SPARSED_OK) {

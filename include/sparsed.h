@@ -184,6 +184,62 @@ int sparsed_run_steps(const uint16_t* Q, const uint16_t* K, const uint16_t* V,
                       int8_t* step_kind, float* step_ms,
                       void* workspace, size_t workspace_bytes, void* stream);
 
+/* ---- Column-sparse path (PulseCol: Periodically Refreshed Column-Sparse
+ * Attention for Accelerating Diffusion Language Models, abstract: the sparse
+ * pattern is a set of key columns of the attention map instead of blocks,
+ * identified at an early denoising step, reused, and refreshed at a few
+ * intermediate steps). A column pattern keeps, per head h, kc key positions
+ * cols[h*col_stride + 0..kc-1] (strictly ascending) shared by every query of
+ * that head; kc = clamp(ceil(keep_ratio*L - 1e-6), 1, L). The block size
+ * arguments bq, bk only choose the tiles of the attention kernel. */
+
+/* kc for a sequence of L keys (as sparsed_uniform_keep with nkb = L). */
+int sparsed_column_keep(int L, float keep_ratio, int* kc);
+
+/* Workspace bytes of the column path for H heads, L tokens, head dim d and kc
+ * kept columns: the column-mass array [H, L] fp32 and the gathered K and V
+ * columns [H, kc, d] bf16 each, every part 256-byte aligned. */
+int sparsed_column_workspace_bytes(int H, int L, int d, int kc, size_t* bytes);
+
+/* One full-attention pass that also selects the column pattern:
+ *   1. O, LSE as sparsed_dense_attn (this pass's output is the step's output).
+ *   2. column mass A[h,c] = sum over every row r of exp(scale*<q_r,k_c> - LSE[h,r])
+ *      from fp32 scores (written to col_mass [H, L] fp32 when non-NULL).
+ *   3. per head: the kc columns of largest A (ties to the lower column),
+ *      written ascending to cols [H, col_stride], col_stride >= kc.
+ * workspace: device memory of at least sparsed_column_workspace_bytes(H, L, d,
+ * kc) bytes, 256-byte aligned, owned by the caller; contents on entry are
+ * ignored. */
+int sparsed_select_columns(const uint16_t* Q, const uint16_t* K, const uint16_t* V,
+                           int H, int L, int d, float scale, int bq, int bk, float keep_ratio,
+                           uint16_t* O, float* LSE, int32_t* cols, int col_stride,
+                           float* col_mass, void* workspace, size_t workspace_bytes, void* stream);
+
+/* Attention of every query over its head's kc kept columns:
+ *   O[h,r,:] = sum over c in cols[h] of softmax(scale*<q_r,k_c>) v_c  (bf16)
+ *   LSE[h,r] = ln sum over c in cols[h] of exp(scale*<q_r,k_c>)       (fp32)
+ * The kept K and V rows are first gathered into the workspace (as in
+ * sparsed_select_columns). An entry outside [0, L) or not above its predecessor
+ * reads row 0 and is reported as SPARSED_ERR_BAD_PATTERN by the next
+ * sparsed_check. */
+int sparsed_column_sparse_attn(const uint16_t* Q, const uint16_t* K, const uint16_t* V,
+                               int H, int L, int d, float scale, int bq, int bk,
+                               const int32_t* cols, int kc, int col_stride,
+                               uint16_t* O, float* LSE, void* workspace, size_t workspace_bytes,
+                               void* stream);
+
+/* The denoising loop with the column pattern: the step kinds of
+ * sparsed_schedule(T, warmup_frac, refresh_every); DENSE: sparsed_dense_attn;
+ * SELECT: sparsed_select_columns into cols (the pattern cache, caller memory);
+ * SPARSE: sparsed_column_sparse_attn with the cached columns. Arguments and
+ * outputs otherwise as sparsed_run_steps. */
+int sparsed_run_steps_columns(const uint16_t* Q, const uint16_t* K, const uint16_t* V,
+                              int H, int L, int d, float scale, int bq, int bk, float keep_ratio,
+                              int T, float warmup_frac, int refresh_every,
+                              int start_step, int have_pattern, int32_t* cols, int col_stride,
+                              uint16_t* O, float* LSE, int8_t* step_kind, float* step_ms,
+                              void* workspace, size_t workspace_bytes, void* stream);
+
 /* Bytes of the library's built-in scratch array used by
  * sparsed_select_pattern_noalloc (16 MiB, held by every GPU that loads the
  * library until the process exits). */
