@@ -283,9 +283,14 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--skip-cpu", action="store_true")
     ap.add_argument("--skip-e2e", action="store_true")
-    ap.add_argument("--op", choices=["run", "dense", "sparse", "select"], default="run",
-                    help="run: the full denoising run (the benchmark); dense/sparse/select: time one "
-                         "library call alone, K launches after W warm-up launches (for profiling)")
+    ap.add_argument("--op", choices=["run", "dense", "sparse", "select", "col_sparse", "col_select"],
+                    default="run",
+                    help="run: the full denoising run (the benchmark); dense/sparse/select and the column "
+                         "path's col_sparse/col_select: time one library call alone, K launches after W "
+                         "warm-up launches (for profiling)")
+    ap.add_argument("--path", choices=["blocks", "columns"], default="blocks",
+                    help="blocks: the block-sparse path (the benchmark); columns: the same denoising run "
+                         "with the column-sparse pattern")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     rank = int(os.environ.get("RANK", "0"))
@@ -312,6 +317,8 @@ def main():
     wl = WORKLOADS[args.workload]
     if args.op != "run":
         return time_one_op(args, wl, dev, rank)
+    if args.path == "columns":
+        return run_columns(args, wl, dev, rank, world, barrier, max_over_ranks)
     log(f"[rank {rank}] inputs for {wl.name}")
     q_cpu, k_cpu, v_cpu = make_inputs(rank_workload(wl, rank))
     q, k, v = (t.to(dev) for t in (q_cpu, k_cpu, v_cpu))
@@ -482,6 +489,17 @@ def time_one_op(args, wl, dev, rank):
         fn = lambda: sp.select_pattern(q, k, v, keep=wl.keep, budget=wl.budget, bq=wl.bq, bk=wl.bk,
                                        workspace=ws)
         flops = dense_flops
+    elif args.op == "col_select":
+        kc = sp.column_keep(wl.L, wl.keep)
+        ws = torch.empty(sp.column_workspace_bytes(wl.H, wl.L, wl.d, kc), dtype=torch.uint8, device=dev)
+        fn = lambda: sp.select_columns(q, k, v, keep=wl.keep, bq=wl.bq, bk=wl.bk, workspace=ws)
+        flops = dense_flops
+    elif args.op == "col_sparse":
+        pat = sp.select_columns(q, k, v, keep=wl.keep, bq=wl.bq, bk=wl.bk)
+        kc = pat.cols.shape[1]
+        ws = torch.empty(sp.column_workspace_bytes(wl.H, wl.L, wl.d, kc), dtype=torch.uint8, device=dev)
+        fn = lambda: sp.column_sparse_attn(q, k, v, pat.cols, bq=wl.bq, bk=wl.bk, out=o, lse=lse, workspace=ws)
+        flops = 4.0 * wl.H * float(wl.L) * kc * wl.d
     else:
         pat = sp.select_pattern(q, k, v, keep=wl.keep, budget=wl.budget, bq=wl.bq, bk=wl.bk)
         fn = lambda: sp.block_sparse_attn(q, k, v, pat.kv_idx, pat.kv_count, bq=wl.bq, bk=wl.bk, out=o, lse=lse)
@@ -499,6 +517,76 @@ def time_one_op(args, wl, dev, rank):
     if rank == 0:
         print(json.dumps({"op": args.op, "workload": wl.name, "launches": args.steps, "ms_median": ms,
                           "ms_all": times, "tflops": flops / (ms * 1e-3) / 1e12, "clocks": clk}), flush=True)
+    return 0
+
+
+def run_columns(args, wl, dev, rank, world, barrier, max_over_ranks):
+    """The same denoising run with the column-sparse pattern (PulseCol): dense
+    warm-up, column selection at the switch, attention over the kept columns.
+    Effective flops count 4*L*kc*d per head for a sparse step."""
+    import block_sparse_bidirectional_select_b200 as sp
+    q, k, v = (t.to(dev) for t in make_inputs(rank_workload(wl, rank)))
+    stream = torch.cuda.current_stream()
+    H, L, d = wl.H, wl.L, wl.d
+    kc = sp.column_keep(L, wl.keep)
+    ws = torch.empty(sp.column_workspace_bytes(H, L, d, kc), dtype=torch.uint8, device=dev)
+    o = torch.empty_like(q)
+    lse = torch.empty((H, L), dtype=torch.float32, device=dev)
+
+    def one_run(time_steps=False):
+        return sp.run_steps_columns(q, k, v, wl.T, wl.warmup_frac, keep=wl.keep,
+                                    refresh_every=wl.refresh_every, bq=wl.bq, bk=wl.bk, out=o, lse=lse,
+                                    workspace=ws, time_steps=time_steps)
+
+    for _ in range(args.warmup):
+        res = one_run()
+    sp.device_check()
+    kinds = res.kinds
+    n_dense, n_select, n_sparse = kinds.count(0), kinds.count(1), kinds.count(2)
+    dense = 4.0 * H * float(L) * float(L) * d
+    sparse = 4.0 * H * float(L) * kc * d
+    flops = (n_dense + n_select) * dense + n_sparse * sparse
+    torch.cuda.synchronize()
+    barrier()
+    clocks = ClockSampler(dev.index or 0)
+    clocks.start()
+    s_ev = torch.cuda.Event(enable_timing=True)
+    e_ev = torch.cuda.Event(enable_timing=True)
+    step_ms = []
+    s_ev.record(stream)
+    for _ in range(args.steps):
+        step_ms.append(one_run(time_steps=True).step_ms)
+    e_ev.record(stream)
+    e_ev.synchronize()
+    barrier()
+    clk = clocks.stop()
+    total_ms = max_over_ranks(s_ev.elapsed_time(e_ev))
+    sp.device_check()
+    per_kind = {0: [], 1: [], 2: []}
+    for run in step_ms:
+        for kind, ms in zip(kinds, run):
+            per_kind[kind].append(ms)
+    mean = lambda x: statistics.mean(x) if x else None
+    fn = lambda: sp.column_sparse_attn(q, k, v, res.kv_idx, bq=wl.bq, bk=wl.bk, out=o, lse=lse, workspace=ws)
+    fn()
+    ms_alone = median_time(fn, stream, 20)
+    peaks, peak_src = load_peaks()
+    peak_burst = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
+    line = {"metric": "column-sparse attn effective TFLOP/s & ms/step at 64k", "value":
+            job_value(flops, args.steps, world, total_ms), "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": dict(workload_config(wl), path="columns", kept_columns_per_head=kc),
+            "ms_per_denoise_step": total_ms / args.steps / wl.T,
+            "steps_breakdown": {"dense_ms": mean(per_kind[0]), "select_ms": mean(per_kind[1]),
+                                "sparse_ms": mean(per_kind[2]), "n_dense": n_dense, "n_select": n_select,
+                                "n_sparse": n_sparse},
+            "column_sparse_attn": {"ms": ms_alone, "tflops": sparse / (ms_alone * 1e-3) / 1e12,
+                                   "frac_of_peak_burst": sparse / (ms_alone * 1e-3) / 1e12 / peak_burst,
+                                   "peak_source": peak_src},
+            "gpu_launches": (n_dense + 3 * n_select + 2 * n_sparse) * args.steps, "clocks": clk}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
     return 0
 
 
