@@ -327,7 +327,7 @@ def main():
 
     H, L, d = wl.H, wl.L, wl.d
     nqb = -(-L // wl.bq)
-    ws = torch.empty(sp.workspace_bytes(H, L, wl.bq, wl.bk), dtype=torch.uint8, device=dev)
+    ws = torch.empty(sp.run_steps_workspace_bytes(H, L, wl.bq, wl.bk), dtype=torch.uint8, device=dev)
     o = torch.empty_like(q)
     lse = torch.empty((H, L), dtype=torch.float32, device=dev)
 

@@ -34,6 +34,7 @@ from ._lib import (BUDGET_ENTROPY, BUDGET_UNIFORM, STEP_DENSE, STEP_SELECT,  # n
                    STEP_SPARSE, SparsedError, check)
 
 __all__ = ["dense_attn", "select_pattern", "block_sparse_attn", "run_steps", "workspace_bytes",
+           "run_steps_workspace_bytes",
            "uniform_keep", "schedule", "device_check", "version", "SparsedError", "Pattern",
            "RunResult", "default_scale", "column_keep", "column_workspace_bytes", "select_columns",
            "column_sparse_attn", "run_steps_columns", "ColumnPattern"]
@@ -90,6 +91,14 @@ def schedule(T: int, warmup_frac: float, refresh_every: int = 0) -> list[int]:
 def workspace_bytes(H: int, L: int, bq: int = 128, bk: int = 128) -> int:
     n = ctypes.c_size_t()
     check(_lib.load().sparsed_workspace_bytes(H, L, bq, bk, ctypes.byref(n)), "sparsed_workspace_bytes")
+    return n.value
+
+
+def run_steps_workspace_bytes(H: int, L: int, bq: int = 128, bk: int = 128) -> int:
+    """Workspace with which run_steps fuses the block mass into its selecting passes."""
+    n = ctypes.c_size_t()
+    check(_lib.load().sparsed_run_steps_workspace_bytes(H, L, bq, bk, ctypes.byref(n)),
+          "sparsed_run_steps_workspace_bytes")
     return n.value
 
 
@@ -207,7 +216,9 @@ def run_steps(q, k, v, T, warmup_frac=0.2, keep=0.1, budget="uniform", refresh_e
         kv_count = torch.zeros((H, nqb), dtype=torch.int32, device=q.device)
         have = 0
     out, lse = _alloc_out(q, out, lse)
-    ws = _workspace(q, bq, bk, workspace)
+    if workspace is None:
+        workspace = torch.empty(run_steps_workspace_bytes(H, L, bq, bk), dtype=torch.uint8, device=q.device)
+    ws = workspace
     kinds = (ctypes.c_int8 * max(T, 1))()
     ms = (ctypes.c_float * max(T, 1))() if time_steps else None
     rc = _lib.load().sparsed_run_steps(

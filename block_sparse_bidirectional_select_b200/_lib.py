@@ -46,6 +46,7 @@ SIGNATURES = {
                                             _I, _P, _P, _P]),
     "sparsed_run_steps": (_I, [_P, _P, _P, _I, _I, _I, _F, _I, _I, _F, _I, _I, _F, _I, _I, _I, _P, _P,
                                _I, _P, _P, _P, _P, _P, _SZ, _P]),
+    "sparsed_run_steps_workspace_bytes": (_I, [_I, _I, _I, _I, ctypes.POINTER(_SZ)]),
     "sparsed_column_keep": (_I, [_I, _F, ctypes.POINTER(_I)]),
     "sparsed_column_workspace_bytes": (_I, [_I, _I, _I, _I, ctypes.POINTER(_SZ)]),
     "sparsed_select_columns": (_I, [_P, _P, _P, _I, _I, _I, _F, _I, _I, _F, _P, _P, _P, _I, _P, _P, _SZ, _P]),

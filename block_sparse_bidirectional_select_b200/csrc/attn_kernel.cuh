@@ -62,6 +62,11 @@ struct AttnArgs {
   int kv_stride;
   float* lse;                // [H, L]
   uint16_t* o;               // [H, L, D]
+  // block mass from this pass (MASS variant): the LSE of an earlier full pass
+  // of the same inputs, and per (head, query block, key block) one partial sum
+  // per softmax warp, [H, nqb, nkb, 8]
+  const float* lse_prev;
+  float* mass_part;
   uint64_t timeout_ns;       // bound of every device-side wait
 };
 
@@ -191,12 +196,13 @@ __device__ __forceinline__ ItemList<SPARSE> item_list(const AttnArgs& a, int w, 
   return it;
 }
 
-template <int D, int BK, bool SPARSE>
+template <int D, int BK, bool SPARSE, bool MASS = false>
 __global__ void __launch_bounds__(384, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const AttnArgs a) {
   using C = AttnCfg<D, BK>;
   constexpr int HALF = C::HALF;
+  static_assert(!(MASS && SPARSE), "the block mass comes from a full pass");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -423,6 +429,10 @@ __global__ void __launch_bounds__(384, 1)
       }
       float m = -__int_as_float(0x7f800000);  // running row max, log2 units (scaled)
       float l = 0.f;                          // running sum of my half row
+      // MASS: my row's LSE (log2 units) from the earlier full pass
+      float lse2_prev = 0.f;
+      if constexpr (MASS)
+        lse2_prev = row_valid ? a.lse_prev[static_cast<long>(h) * a.L + grow] * 1.44269504088896340736f : 0.f;
       // only a list that can hold the ragged last key block needs its entries
       // here; they are read one tile ahead, off the critical path
       const bool ragged = SPARSE && (a.Lk % BK) != 0;
@@ -496,7 +506,16 @@ __global__ void __launch_bounds__(384, 1)
           m = m_new;
         }
         // P_b is free: S_b(g) was issued only after PV(g-2) completed
-        l += softmax_half_exp<HALF>(s, sl2, m, lane_base + (b ? C::TM_P1 : C::TM_P0));
+        const float ps = softmax_half_exp<HALF>(s, sl2, m, lane_base + (b ? C::TM_P1 : C::TM_P0));
+        l += ps;
+        if constexpr (MASS) {
+          // this tile's probability mass of my half row is ps * 2^(m - lse2);
+          // the warp's 16 rows x 2 halves summed by a fixed shuffle tree
+          float c = row_valid ? ps * ptx::ex2(m - lse2_prev) : 0.f;
+#pragma unroll
+          for (int off = 16; off > 0; off >>= 1) c += __shfl_xor_sync(0xffffffffu, c, off);
+          if (lane == 0) a.mass_part[((static_cast<long>(h) * a.nqb + qi) * a.nkb + jj) * 8 + warp] = c;
+        }
         ptx::tmem_wait_st();
         ptx::tc_fence_before();
         __syncwarp();

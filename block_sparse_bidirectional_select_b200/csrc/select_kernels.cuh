@@ -2,6 +2,8 @@
 // head-specific sparse pattern is computed once from full attention; Step-dLLM
 // abstract: a block-sparse mask under a uniform or head-adaptive budget).
 //
+//   mass_from_parts_kernel  the same M from per-warp partial sums the
+//                       attention kernel's fused variant wrote in its pass
 //   block_mass_kernel   M[h,i,j] = sum_{r in qblk i, c in kblk j}
 //                                  exp(scale*<q_r,k_c> - LSE_r)
 //                       recomputes S = Q K^T on tcgen05 (fp32 in TMEM) and
@@ -208,6 +210,19 @@ __global__ void __launch_bounds__(256, 1)
     ptx::tc_fence_after();
     ptx::tmem_dealloc(tmem, C::TM_ALLOC);
   }
+}
+
+// ---------------------------------------------------------------- fused mass
+
+// Block mass from the partial sums the attention kernel's MASS variant wrote
+// during its full pass: mass[e] = sum of the 8 softmax warps' partials of tile
+// e = (h, i, j), in a fixed order.
+__global__ void __launch_bounds__(256)
+    mass_from_parts_kernel(const float4* __restrict__ part, long n, float* __restrict__ mass) {
+  const long e = static_cast<long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (e >= n) return;
+  const float4 a = part[2 * e], b = part[2 * e + 1];
+  mass[e] = ((a.x + a.y) + (a.z + a.w)) + ((b.x + b.y) + (b.z + b.w));
 }
 
 // ---------------------------------------------------------------- top-k

@@ -140,11 +140,11 @@ struct Problem {
 // The register split of the kernel (setmaxnreg) must be funded by its launch
 // register count; checked once per kernel before the first launch, so a raise
 // can never wait forever.
-template <int D, int BK, bool SPARSE>
+template <int D, int BK, bool SPARSE, bool MASS>
 int launch_attn_t(const Problem& p, const int32_t* kv_idx, const int32_t* kv_count, int kv_stride,
-                  cudaStream_t st) {
+                  const float* lse_prev, float* mass_part, cudaStream_t st) {
   using C = AttnCfg<D, BK>;
-  auto kern = attn_fwd_kernel<D, BK, SPARSE>;
+  auto kern = attn_fwd_kernel<D, BK, SPARSE, MASS>;
   static int regs = -1;
   if (regs < 0) {
     cudaFuncAttributes fa;
@@ -169,6 +169,8 @@ int launch_attn_t(const Problem& p, const int32_t* kv_idx, const int32_t* kv_cou
   a.kv_stride = kv_stride;
   a.lse = p.LSE;
   a.o = p.O;
+  a.lse_prev = lse_prev;
+  a.mass_part = mass_part;
   a.timeout_ns = kWaitTimeoutNs;
   int sms = 0;
   SP_TRY(sm_count(&sms));
@@ -182,12 +184,16 @@ int launch_attn_t(const Problem& p, const int32_t* kv_idx, const int32_t* kv_cou
   return SPARSED_OK;
 }
 
+// mass_part != nullptr selects the fused variant (dense only): the pass also
+// writes the block-mass partials, using lse_prev as every row's LSE.
 int launch_attn(const Problem& p, bool sparse, const int32_t* kv_idx, const int32_t* kv_count,
-                int kv_stride, cudaStream_t st) {
-#define SP_ATTN(D_, BK_)                                                               \
-  if (p.d == D_ && p.bk == BK_)                                                        \
-    return sparse ? launch_attn_t<D_, BK_, true>(p, kv_idx, kv_count, kv_stride, st)   \
-                  : launch_attn_t<D_, BK_, false>(p, kv_idx, kv_count, kv_stride, st);
+                int kv_stride, cudaStream_t st, const float* lse_prev = nullptr, float* mass_part = nullptr) {
+#define SP_ATTN(D_, BK_)                                                                                  \
+  if (p.d == D_ && p.bk == BK_) {                                                                         \
+    if (sparse) return launch_attn_t<D_, BK_, true, false>(p, kv_idx, kv_count, kv_stride, nullptr, nullptr, st); \
+    if (mass_part) return launch_attn_t<D_, BK_, false, true>(p, nullptr, nullptr, 0, lse_prev, mass_part, st);   \
+    return launch_attn_t<D_, BK_, false, false>(p, nullptr, nullptr, 0, nullptr, nullptr, st);           \
+  }
   SP_ATTN(64, 64)
   SP_ATTN(64, 128)
   SP_ATTN(128, 64)
@@ -327,14 +333,11 @@ Workspace ws_layout(int H, int nqb, int nkb) {
   return w;
 }
 
-// Steps 2-4 of pattern selection, after the dense pass wrote O and LSE.
-int select_after_dense(const Problem& p, float keep_ratio, int budget_mode, int32_t* kv_idx,
-                       int32_t* kv_count, int kv_stride, float* block_mass, int32_t* head_k,
-                       void* workspace, cudaStream_t st) {
+// Steps 3-4 of pattern selection from a block-mass grid: budget and top-k.
+int select_from_mass(const Problem& p, const float* mass, float keep_ratio, int budget_mode, int32_t* kv_idx,
+                     int32_t* kv_count, int kv_stride, int32_t* head_k, void* workspace, cudaStream_t st) {
   const Workspace w = ws_layout(p.H, p.nqb, p.nkb);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
-  float* mass = block_mass ? block_mass : reinterpret_cast<float*>(ws + w.grid);
-  SP_TRY(launch_mass(p, mass, st));
   const int rows = p.H * p.nqb;
   const int kblocks = (rows + 7) / 8;
   int32_t* hk = nullptr;
@@ -352,6 +355,56 @@ int select_after_dense(const Problem& p, float keep_ratio, int budget_mode, int3
   topk_kernel<<<kblocks, 256, 0, st>>>(mass, rows, p.nqb, p.nkb, k_uniform, hk, hk_out, kv_idx,
                                        kv_count, kv_stride);
   SP_CUDA(cudaGetLastError());
+  return SPARSED_OK;
+}
+
+// Steps 2-4 of pattern selection, after the dense pass wrote O and LSE.
+int select_after_dense(const Problem& p, float keep_ratio, int budget_mode, int32_t* kv_idx,
+                       int32_t* kv_count, int kv_stride, float* block_mass, int32_t* head_k,
+                       void* workspace, cudaStream_t st) {
+  const Workspace w = ws_layout(p.H, p.nqb, p.nkb);
+  float* mass = block_mass ? block_mass : reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + w.grid);
+  SP_TRY(launch_mass(p, mass, st));
+  return select_from_mass(p, mass, keep_ratio, budget_mode, kv_idx, kv_count, kv_stride, head_k, workspace, st);
+}
+
+// Fused selection of the step loop: the scratch after the selection workspace
+// holds the block-mass partials of the fused pass and a copy of the LSE of
+// the run's last full pass.
+struct FusedWorkspace {
+  size_t part, lse_prev, total;
+};
+
+FusedWorkspace fused_ws_layout(int H, int L, int nqb, int nkb) {
+  FusedWorkspace f;
+  f.part = ws_layout(H, nqb, nkb).total;
+  f.lse_prev = f.part + align256(static_cast<size_t>(H) * nqb * nkb * 8 * sizeof(float));
+  f.total = f.lse_prev + align256(static_cast<size_t>(H) * L * sizeof(float));
+  return f;
+}
+
+// A selecting step whose block mass comes from its own full pass: every row's
+// LSE is taken from lse_prev, the LSE of an earlier full pass of the same
+// inputs (so it equals the LSE this pass computes).
+int fused_select(const Problem& p, float keep_ratio, int budget_mode, int32_t* kv_idx, int32_t* kv_count,
+                 int kv_stride, void* workspace, cudaStream_t st) {
+  const FusedWorkspace f = fused_ws_layout(p.H, p.L, p.nqb, p.nkb);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  float* part = reinterpret_cast<float*>(ws + f.part);
+  const float* lse_prev = reinterpret_cast<const float*>(ws + f.lse_prev);
+  SP_TRY(launch_attn(p, false, nullptr, nullptr, 0, st, lse_prev, part));
+  float* mass = reinterpret_cast<float*>(ws + ws_layout(p.H, p.nqb, p.nkb).grid);
+  const long n = static_cast<long>(p.H) * p.nqb * p.nkb;
+  mass_from_parts_kernel<<<static_cast<unsigned>(cdiv(n, 256)), 256, 0, st>>>(reinterpret_cast<const float4*>(part),
+                                                                               n, mass);
+  SP_CUDA(cudaGetLastError());
+  return select_from_mass(p, mass, keep_ratio, budget_mode, kv_idx, kv_count, kv_stride, nullptr, workspace, st);
+}
+
+int save_lse(const Problem& p, void* workspace, cudaStream_t st) {
+  const FusedWorkspace f = fused_ws_layout(p.H, p.L, p.nqb, p.nkb);
+  SP_CUDA(cudaMemcpyAsync(static_cast<uint8_t*>(workspace) + f.lse_prev, p.LSE,
+                          static_cast<size_t>(p.H) * p.L * sizeof(float), cudaMemcpyDeviceToDevice, st));
   return SPARSED_OK;
 }
 
@@ -466,6 +519,13 @@ int sparsed_workspace_bytes(int H, int L, int bq, int bk, size_t* bytes) {
   return SPARSED_OK;
 }
 
+int sparsed_run_steps_workspace_bytes(int H, int L, int bq, int bk, size_t* bytes) {
+  if (!bytes || H < 0 || L < 0) return SPARSED_ERR_INVALID_ARG;
+  if ((bq != 64 && bq != 128) || (bk != 64 && bk != 128)) return SPARSED_ERR_UNSUPPORTED;
+  *bytes = fused_ws_layout(H, L, static_cast<int>(cdiv(L, bq)), static_cast<int>(cdiv(L, bk))).total;
+  return SPARSED_OK;
+}
+
 int sparsed_dense_attn(const uint16_t* Q, const uint16_t* K, const uint16_t* V, int H, int L, int d,
                        float scale, int bq, int bk, uint16_t* O, float* LSE, void* stream) {
   Problem p;
@@ -539,6 +599,11 @@ int sparsed_run_steps(const uint16_t* Q, const uint16_t* K, const uint16_t* V, i
   SP_TRY(require_sm100());
   SP_TRY(get_encoder());
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  // fused selection when the workspace has room for it (see the header)
+  const bool fused = any_select && workspace &&
+                     workspace_bytes >= fused_ws_layout(p.H, p.L, p.nqb, p.nkb).total &&
+                     static_cast<long long>(p.H) * p.nqb * p.nkb * 8 < (1ll << 31);
+  bool have_lse = false;  // a full pass of this call left its LSE in the workspace
   std::vector<cudaEvent_t> ev;
   if (step_ms && start_step < T) {
     ev.resize(static_cast<size_t>(T - start_step) + 1, nullptr);
@@ -550,12 +615,24 @@ int sparsed_run_steps(const uint16_t* Q, const uint16_t* K, const uint16_t* V, i
     switch (kinds[t]) {
       case SPARSED_STEP_DENSE:
         rc = launch_attn(p, false, nullptr, nullptr, 0, st);
+        if (rc == SPARSED_OK && fused && t + 1 < T && kinds[t + 1] == SPARSED_STEP_SELECT) {
+          rc = save_lse(p, workspace, st);
+          have_lse = true;
+        }
         break;
       case SPARSED_STEP_SELECT:
-        rc = launch_attn(p, false, nullptr, nullptr, 0, st);
-        if (rc == SPARSED_OK)
-          rc = select_after_dense(p, keep_ratio, budget_mode, kv_idx, kv_count, kv_stride, nullptr,
-                                  nullptr, workspace, st);
+        if (fused && have_lse) {
+          rc = fused_select(p, keep_ratio, budget_mode, kv_idx, kv_count, kv_stride, workspace, st);
+        } else {
+          rc = launch_attn(p, false, nullptr, nullptr, 0, st);
+          if (rc == SPARSED_OK)
+            rc = select_after_dense(p, keep_ratio, budget_mode, kv_idx, kv_count, kv_stride, nullptr,
+                                    nullptr, workspace, st);
+        }
+        if (rc == SPARSED_OK && fused) {
+          rc = save_lse(p, workspace, st);
+          have_lse = true;
+        }
         break;
       default:
         rc = launch_attn(p, true, kv_idx, kv_count, kv_stride, st);

@@ -147,6 +147,12 @@ int sparsed_select_pattern(const uint16_t* Q, const uint16_t* K, const uint16_t*
                            float* block_mass, int32_t* head_k,
                            void* workspace, size_t workspace_bytes, void* stream);
 
+/* Workspace bytes with which sparsed_run_steps fuses the block mass into
+ * the full pass of its SELECT steps: sparsed_workspace_bytes plus the
+ * per-warp mass partials [H, nqb, nkb, 8] fp32 and one [H, L] fp32 LSE copy,
+ * every part 256-byte aligned. */
+int sparsed_run_steps_workspace_bytes(int H, int L, int bq, int bk, size_t* bytes);
+
 /* Block-sparse attention over a cached pattern (Step-dLLM abstract: the mask
  * is reused within each interval; SparseD abstract: the precomputed pattern is
  * reused at all later steps). For each row r of query block i of head h, the
@@ -172,8 +178,16 @@ int sparsed_block_sparse_attn(const uint16_t* Q, const uint16_t* K, const uint16
  * step_kind (nullable, HOST [T] int8) receives the kinds of all T steps.
  * step_ms (nullable, HOST [T] fp32) receives each executed step's device time
  * in ms from CUDA events (0 for skipped steps); when given, the call
- * synchronises the stream before returning. workspace as in
- * sparsed_select_pattern. */
+ * synchronises the stream before returning. workspace: at least
+ * sparsed_workspace_bytes(H, L, bq, bk) bytes as in sparsed_select_pattern.
+ * With sparsed_run_steps_workspace_bytes(H, L, bq, bk) bytes, a SELECT step
+ * that follows an earlier full pass of this call (a DENSE step just before
+ * it, or an earlier SELECT) takes the block mass from its own full pass: the
+ * attention kernel sums each tile's probabilities with the LSE of that earlier
+ * pass, which equals this pass's LSE because the loop's inputs are fixed
+ * (Step-dLLM abstract: selection cost matters at every anchor). A SELECT step
+ * with no earlier full pass in the call, or a smaller workspace, runs the
+ * separate block-mass pass of sparsed_select_pattern. */
 int sparsed_run_steps(const uint16_t* Q, const uint16_t* K, const uint16_t* V,
                       int H, int L, int d, float scale, int bq, int bk,
                       float keep_ratio, int budget_mode,

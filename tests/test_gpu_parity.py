@@ -237,15 +237,45 @@ def test_run_steps_matches_calls_and_oracle():
     sp.device_check()
     assert r.kinds == O.schedule(6, 0.34, 2)
     assert all(ms > 0 for ms in r.step_ms)
-    p = sp.select_pattern(qc, kc, vc, keep=0.5)
-    o2, l2 = sp.block_sparse_attn(qc, kc, vc, p.kv_idx, p.kv_count)
-    assert torch.equal(r.kv_idx, p.kv_idx)
-    last = r.kinds[-1]
-    if last == O.SPARSE:
-        assert torch.equal(r.o.view(torch.int16), o2.view(torch.int16))
-    o_ref, l_ref, kinds, _ = O.run_steps(f64(q), f64(k), f64(v), scale, b, b, 0.5, "uniform", 6, 0.34, 2)
+    o_ref, l_ref, kinds, pat = O.run_steps(f64(q), f64(k), f64(v), scale, b, b, 0.5, "uniform", 6, 0.34, 2)
     assert kinds == r.kinds
     assert_o_lse(r.o, r.lse, o_ref, l_ref, "run_steps")
+    idx, cnt = r.kv_idx.cpu().numpy(), r.kv_count.cpu().numpy()
+    for h in range(H):
+        for i in range(idx.shape[1]):
+            check_selection(idx[h, i], cnt[h, i], pat["mass"][h, i], int(pat["head_k"][h]), f"h{h} i{i}")
+    # the last (sparse) step runs on the cached pattern, bit for bit
+    if r.kinds[-1] == O.SPARSE:
+        o2, _ = sp.block_sparse_attn(qc, kc, vc, r.kv_idx, r.kv_count)
+        assert torch.equal(r.o.view(torch.int16), o2.view(torch.int16))
+
+
+@pytest.mark.parametrize("budget", ["uniform", "entropy"])
+def test_run_steps_fused_selection_matches_separate_pass(budget):
+    """With the larger workspace, SELECT steps after a full pass take the block
+    mass from their own pass; with the selection workspace alone they run the
+    separate block-mass pass. Both must pick the oracle's pattern (margin
+    rule) and agree with each other wherever the oracle's margin is clear."""
+    H, L, d = 4, 1536, 128
+    q, k, v, scale = _inputs(H, L, d, seed=88, structure="band")
+    qc, kc, vc = _cuda(q, k, v)
+    small = torch.empty(sp.workspace_bytes(H, L), dtype=torch.uint8, device="cuda")
+    assert sp.run_steps_workspace_bytes(H, L) > small.numel()
+    kw = dict(T=8, warmup_frac=0.3, keep=0.25, budget=budget, refresh_every=3)
+    r_fused = sp.run_steps(qc, kc, vc, **kw)
+    r_sep = sp.run_steps(qc, kc, vc, workspace=small, **kw)
+    sp.device_check()
+    o_ref, l_ref, kinds, pat = O.run_steps(f64(q), f64(k), f64(v), scale, 128, 128, 0.25, budget, 8, 0.3, 3)
+    assert kinds == r_fused.kinds and kinds.count(O.SELECT) >= 2
+    assert_o_lse(r_fused.o, r_fused.lse, o_ref, l_ref, f"fused run_steps {budget}")
+    for r in (r_fused, r_sep):
+        idx, cnt = r.kv_idx.cpu().numpy(), r.kv_count.cpu().numpy()
+        for h in range(H):
+            for i in range(idx.shape[1]):
+                check_selection(idx[h, i], cnt[h, i], pat["mass"][h, i], int(pat["head_k"][h]), f"h{h} i{i}")
+    assert torch.equal(r_fused.kv_count, r_sep.kv_count)
+    same = (r_fused.kv_idx == r_sep.kv_idx).all(dim=-1).float().mean().item()
+    assert same > 0.95
 
 
 def test_run_steps_resume_with_pattern():
