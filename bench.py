@@ -590,6 +590,17 @@ def run_columns(args, wl, dev, rank, world, barrier, max_over_ranks):
     return 0
 
 
+def code_signature(src):
+    """The kernel source without comments and blank lines: traffic figures
+    stay valid across edits of the comments only."""
+    lines = []
+    for line in src.splitlines():
+        code = line.split("//", 1)[0].strip()
+        if code:
+            lines.append(code)
+    return "\n".join(lines)
+
+
 def load_traffic(workload):
     """DRAM bytes per launch from the committed ncu capture (profiles/traffic.json),
     used only while the attention kernel source is the one that was captured."""
@@ -599,8 +610,8 @@ def load_traffic(workload):
     try:
         with open(path) as f:
             t = json.load(f)
-        with open(src, "rb") as f:
-            sha = hashlib.sha256(f.read()).hexdigest()
+        with open(src) as f:
+            sha = hashlib.sha256(code_signature(f.read()).encode()).hexdigest()
     except (OSError, ValueError):
         return {}
     if t.get("attn_kernel_sha256") != sha:

@@ -45,6 +45,11 @@
 // they take the same decision, and each rescales its half of O.
 // The epilogue writes O straight from registers to global memory (each thread
 // one contiguous half row), so no shared memory is held across items.
+// MASS variant (dense only): the pass also yields the block mass of pattern
+// selection. Each tile's probabilities of a row sum to ps = sum_c 2^(s_c*sl2 - m)
+// in the exp pass; times 2^(m - lse2), with lse2 the row's LSE from an earlier
+// full pass of the same inputs, that is the row's mass in the tile, and the
+// warp writes its 16 rows' sum as one of 8 partials per tile.
 // Every wait is bounded (mbarriers only, no named barriers), so a timed-out
 // warp cannot strand the others.
 #pragma once
