@@ -250,22 +250,23 @@ def test_run_steps_matches_calls_and_oracle():
         assert torch.equal(r.o.view(torch.int16), o2.view(torch.int16))
 
 
-@pytest.mark.parametrize("budget", ["uniform", "entropy"])
-def test_run_steps_fused_selection_matches_separate_pass(budget):
+@pytest.mark.parametrize("budget,d,L,bq,bk", [("uniform", 128, 1536, 128, 128), ("entropy", 128, 1536, 128, 128),
+                                               ("uniform", 64, 1000, 64, 64), ("entropy", 128, 1000, 128, 64)])
+def test_run_steps_fused_selection_matches_separate_pass(budget, d, L, bq, bk):
     """With the larger workspace, SELECT steps after a full pass take the block
     mass from their own pass; with the selection workspace alone they run the
     separate block-mass pass. Both must pick the oracle's pattern (margin
     rule) and agree with each other wherever the oracle's margin is clear."""
-    H, L, d = 4, 1536, 128
-    q, k, v, scale = _inputs(H, L, d, seed=88, structure="band")
+    H = 4
+    q, k, v, scale = _inputs(H, L, d, seed=88 + d + bk, structure="band")
     qc, kc, vc = _cuda(q, k, v)
-    small = torch.empty(sp.workspace_bytes(H, L), dtype=torch.uint8, device="cuda")
-    assert sp.run_steps_workspace_bytes(H, L) > small.numel()
-    kw = dict(T=8, warmup_frac=0.3, keep=0.25, budget=budget, refresh_every=3)
+    small = torch.empty(sp.workspace_bytes(H, L, bq, bk), dtype=torch.uint8, device="cuda")
+    assert sp.run_steps_workspace_bytes(H, L, bq, bk) > small.numel()
+    kw = dict(T=8, warmup_frac=0.3, keep=0.25, budget=budget, refresh_every=3, bq=bq, bk=bk)
     r_fused = sp.run_steps(qc, kc, vc, **kw)
     r_sep = sp.run_steps(qc, kc, vc, workspace=small, **kw)
     sp.device_check()
-    o_ref, l_ref, kinds, pat = O.run_steps(f64(q), f64(k), f64(v), scale, 128, 128, 0.25, budget, 8, 0.3, 3)
+    o_ref, l_ref, kinds, pat = O.run_steps(f64(q), f64(k), f64(v), scale, bq, bk, 0.25, budget, 8, 0.3, 3)
     assert kinds == r_fused.kinds and kinds.count(O.SELECT) >= 2
     assert_o_lse(r_fused.o, r_fused.lse, o_ref, l_ref, f"fused run_steps {budget}")
     for r in (r_fused, r_sep):
