@@ -11,6 +11,11 @@ device memory and streams.
     block_sparse_attn(q, k, v, kv_idx, kv_count) -> (o, lse)
     run_steps(q, k, v, T, warmup_frac, ...)  -> RunResult (o, lse, kinds, step_ms, pattern)
 
+Head-sharded selection (the heads of one layer over several ranks; only the
+per-head entropies cross ranks):
+
+    select_pattern_sharded(q, k, v, keep, group) -> Pattern for this rank's heads
+
 Column-sparse path (per-head kept key columns shared by all queries):
 
     select_columns(q, k, v, keep)            -> ColumnPattern (o, lse, cols, col_mass)
@@ -37,7 +42,8 @@ __all__ = ["dense_attn", "select_pattern", "block_sparse_attn", "run_steps", "wo
            "run_steps_workspace_bytes",
            "uniform_keep", "schedule", "device_check", "version", "SparsedError", "Pattern",
            "RunResult", "default_scale", "column_keep", "column_workspace_bytes", "select_columns",
-           "column_sparse_attn", "run_steps_columns", "ColumnPattern"]
+           "column_sparse_attn", "run_steps_columns", "ColumnPattern", "select_head_entropy",
+           "entropy_budget", "select_with_head_k", "select_pattern_sharded", "gather_head_entropies"]
 
 
 def _ptr(t: torch.Tensor | None):
@@ -318,3 +324,77 @@ def run_steps_columns(q, k, v, T, warmup_frac=0.2, keep=0.1, refresh_every=0, sc
         None if ms is None else ctypes.cast(ms, ctypes.c_void_p), _ptr(ws), ws.numel(), _stream(stream))
     check(rc, "sparsed_run_steps_columns")
     return RunResult(out, lse, list(kinds[:T]), None if ms is None else list(ms[:T]), cols, None)
+
+
+# ---------------------------------------------------------------- head-sharded selection
+
+def select_head_entropy(q, k, v, scale=None, bq=128, bk=128, workspace=None, stream=None):
+    """Full pass, block mass and the mean row entropy of every head:
+    returns (o, lse, head_entropy [H] fp64 on the device, workspace). The
+    workspace keeps the block mass for select_with_head_k."""
+    H, L, d = _check_qkv(q, k, v)
+    scale = default_scale(d) if scale is None else scale
+    out, lse = _alloc_out(q, None, None)
+    ent = torch.empty(H, dtype=torch.float64, device=q.device)
+    ws = _workspace(q, bq, bk, workspace)
+    rc = _lib.load().sparsed_select_head_entropy(_ptr(q), _ptr(k), _ptr(v), H, L, d, scale, bq, bk, _ptr(out),
+                                                 _ptr(lse), _ptr(ent), _ptr(ws), ws.numel(), _stream(stream))
+    check(rc, "sparsed_select_head_entropy")
+    return out, lse, ent, ws
+
+
+def entropy_budget(head_entropy, nkb: int, keep: float) -> list[int]:
+    """The head-adaptive allocation on the host, from the entropies of all
+    heads of a layer (any float sequence) to k_h per head."""
+    vals = [float(x) for x in head_entropy]
+    H = len(vals)
+    src = (ctypes.c_double * max(H, 1))(*vals)
+    dst = (ctypes.c_int32 * max(H, 1))()
+    check(_lib.load().sparsed_entropy_budget(ctypes.cast(src, ctypes.c_void_p), H, nkb, keep,
+                                             ctypes.cast(dst, ctypes.c_void_p)), "sparsed_entropy_budget")
+    return list(dst[:H])
+
+
+def select_with_head_k(H, L, head_k, workspace, bq=128, bk=128, stream=None):
+    """Top-k per (head, query block) with given k_h over the block mass a
+    preceding select_head_entropy left in ``workspace``: (kv_idx, kv_count)."""
+    dev = workspace.device
+    nqb, nkb = -(-L // bq), -(-L // bk)
+    hk = torch.as_tensor(head_k, dtype=torch.int32).to(dev).contiguous()
+    kv_idx = torch.full((H, nqb, max(nkb, 1)), -1, dtype=torch.int32, device=dev)
+    kv_count = torch.zeros((H, nqb), dtype=torch.int32, device=dev)
+    rc = _lib.load().sparsed_select_with_head_k(H, L, bq, bk, _ptr(hk), _ptr(kv_idx), _ptr(kv_count),
+                                                kv_idx.shape[2], _ptr(workspace), workspace.numel(),
+                                                _stream(stream))
+    check(rc, "sparsed_select_with_head_k")
+    return kv_idx, kv_count, hk
+
+
+def gather_head_entropies(ent, group=None):
+    """All ranks' per-head entropies in rank order (a CPU fp64 tensor) and
+    this rank's index; the identity without a group. NCCL gathers device
+    tensors, other backends host tensors."""
+    if group is None:
+        return ent.cpu(), 0
+    import torch.distributed as dist
+    world = dist.get_world_size(group)
+    mine = ent if dist.get_backend(group) == "nccl" else ent.cpu()
+    parts = [torch.empty_like(mine) for _ in range(world)]
+    dist.all_gather(parts, mine, group=group)
+    return torch.cat([t.cpu() for t in parts]), dist.get_rank(group)
+
+
+def select_pattern_sharded(q, k, v, keep=0.1, group=None, scale=None, bq=128, bk=128, workspace=None,
+                           stream=None) -> Pattern:
+    """Entropy-budget pattern selection for this rank's heads of a layer whose
+    heads are split evenly over the ranks of ``group`` (in rank order). The
+    per-head entropies are all-gathered, every rank runs the same host
+    allocation over all heads, and keeps its own heads' k_h. Without a group
+    the local heads are the whole layer."""
+    H, L, d = _check_qkv(q, k, v)
+    out, lse, ent, ws = select_head_entropy(q, k, v, scale, bq, bk, workspace, stream)
+    ent_all, rank = gather_head_entropies(ent, group)
+    nkb = -(-L // bk)
+    head_k_all = entropy_budget(ent_all.tolist(), nkb, keep)
+    kv_idx, kv_count, hk = select_with_head_k(H, L, head_k_all[rank * H:(rank + 1) * H], ws, bq, bk, stream)
+    return Pattern(out, lse, kv_idx, kv_count, None, hk)

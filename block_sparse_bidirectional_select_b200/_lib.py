@@ -47,6 +47,9 @@ SIGNATURES = {
     "sparsed_run_steps": (_I, [_P, _P, _P, _I, _I, _I, _F, _I, _I, _F, _I, _I, _F, _I, _I, _I, _P, _P,
                                _I, _P, _P, _P, _P, _P, _SZ, _P]),
     "sparsed_run_steps_workspace_bytes": (_I, [_I, _I, _I, _I, ctypes.POINTER(_SZ)]),
+    "sparsed_select_head_entropy": (_I, [_P, _P, _P, _I, _I, _I, _F, _I, _I, _P, _P, _P, _P, _SZ, _P]),
+    "sparsed_entropy_budget": (_I, [_P, _I, _I, _F, _P]),
+    "sparsed_select_with_head_k": (_I, [_I, _I, _I, _I, _P, _P, _P, _I, _P, _SZ, _P]),
     "sparsed_column_keep": (_I, [_I, _F, ctypes.POINTER(_I)]),
     "sparsed_column_workspace_bytes": (_I, [_I, _I, _I, _I, ctypes.POINTER(_SZ)]),
     "sparsed_select_columns": (_I, [_P, _P, _P, _I, _I, _I, _F, _I, _I, _F, _P, _P, _P, _I, _P, _P, _SZ, _P]),

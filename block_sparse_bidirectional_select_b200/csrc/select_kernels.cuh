@@ -302,29 +302,29 @@ __global__ void __launch_bounds__(256)
   if (lane == 0) ent[row] = e;
 }
 
-// One block. E_h = (sum_i ent[h,i]) / nqb (sequential in i). Then one thread
-// allocates B = clamp(ceil(rho*H*nkb - 1e-6), H, H*nkb): one block per head,
-// the extra B-H split in proportion to E_h (evenly if the split heads' E sum to
-// 0), shares above nkb-1 capped and the rest re-split, then largest-remainder
-// rounding with ties to the lower head. Writes k_h = 1 + extra_h.
-// scratch: 4*H doubles (entropy, share, quota, mark).
-__global__ void budget_kernel(const double* __restrict__ ent, int H, int nqb, int nkb, float keep_ratio,
-                              int32_t* __restrict__ head_k, double* __restrict__ scratch) {
-  double* E = scratch;
-  double* extra = scratch + H;      // < 0: not yet decided
-  double* quota = scratch + 2 * H;
-  double* mark = scratch + 3 * H;
-  for (int h = threadIdx.x; h < H; h += blockDim.x) {
-    double s = 0.0;
-    for (int i = 0; i < nqb; ++i) s += ent[static_cast<long>(h) * nqb + i];
-    E[h] = s / nqb;
-    extra[h] = -1.0;
+// The head-adaptive allocation (one thread, fp64): B = clamp(ceil(rho*H*nkb -
+// 1e-6), H, H*nkb); one block per head, the extra B-H split in proportion to
+// E_h (evenly if the split heads' E sum to 0), shares above nkb-1 capped and
+// the rest re-split, then largest-remainder rounding with ties to the lower
+// head. Writes k_h = 1 + extra_h. Shared by the device budget kernel and the
+// host entry point for head-sharded selection; the budget product is formed
+// without fused multiply-add so both sides take identical steps.
+// scratch: extra, quota, mark (3*H doubles).
+__host__ __device__ inline void allocate_budget(const double* E, int H, int nkb, float keep_ratio,
+                                                double* extra, double* quota, double* mark, int32_t* head_k) {
+  for (int h = 0; h < H; ++h) {
+    extra[h] = -1.0;  // < 0: not yet decided
     mark[h] = 0.0;
   }
-  __syncthreads();
-  if (threadIdx.x != 0) return;
   const double rho = static_cast<double>(keep_ratio);
-  long B = static_cast<long>(ceil(rho * H * nkb - 1e-6));
+#ifdef __CUDA_ARCH__
+  const double prod = __dmul_rn(__dmul_rn(rho, static_cast<double>(H)), static_cast<double>(nkb));
+  long B = static_cast<long>(ceil(__dsub_rn(prod, 1e-6)));
+#else
+  volatile double prod = rho * static_cast<double>(H);
+  prod = prod * static_cast<double>(nkb);
+  long B = static_cast<long>(ceil(prod - 1e-6));
+#endif
   if (B < H) B = H;
   if (B > static_cast<long>(H) * nkb) B = static_cast<long>(H) * nkb;
   const double cap = nkb - 1;
@@ -395,6 +395,30 @@ __global__ void budget_kernel(const double* __restrict__ ent, int H, int nqb, in
     break;
   }
   for (int h = 0; h < H; ++h) head_k[h] = 1 + static_cast<int32_t>(extra[h]);
+}
+
+// Per-head mean of the row entropies: E_h = (sum_i ent[h,i]) / nqb, the sum
+// sequential in i.
+__device__ __forceinline__ double head_mean_entropy(const double* ent, int h, int nqb) {
+  double s = 0.0;
+  for (int i = 0; i < nqb; ++i) s += ent[static_cast<long>(h) * nqb + i];
+  return s / nqb;
+}
+
+__global__ void head_entropy_kernel(const double* __restrict__ ent, int H, int nqb, double* __restrict__ E) {
+  for (int h = threadIdx.x + blockIdx.x * blockDim.x; h < H; h += blockDim.x * gridDim.x)
+    E[h] = head_mean_entropy(ent, h, nqb);
+}
+
+// One block: the head means, then the allocation on one thread.
+// scratch: 4*H doubles (entropy, extra, quota, mark).
+__global__ void budget_kernel(const double* __restrict__ ent, int H, int nqb, int nkb, float keep_ratio,
+                              int32_t* __restrict__ head_k, double* __restrict__ scratch) {
+  double* E = scratch;
+  for (int h = threadIdx.x; h < H; h += blockDim.x) E[h] = head_mean_entropy(ent, h, nqb);
+  __syncthreads();
+  if (threadIdx.x != 0) return;
+  allocate_budget(E, H, nkb, keep_ratio, scratch + H, scratch + 2 * H, scratch + 3 * H, head_k);
 }
 
 }  // namespace sparsed

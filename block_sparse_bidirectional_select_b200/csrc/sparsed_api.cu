@@ -660,6 +660,65 @@ int sparsed_run_steps(const uint16_t* Q, const uint16_t* K, const uint16_t* V, i
   return rc;
 }
 
+// ---- head-sharded entropy budget (the heads of one layer split over ranks)
+
+int sparsed_entropy_budget(const double* head_entropy, int H, int nkb, float keep_ratio, int32_t* head_k) {
+  if (!head_entropy || !head_k || H < 1 || nkb < 1 || !(keep_ratio > 0.f && keep_ratio <= 1.f))
+    return SPARSED_ERR_INVALID_ARG;
+  std::vector<double> scratch(static_cast<size_t>(H) * 3);
+  allocate_budget(head_entropy, H, nkb, keep_ratio, scratch.data(), scratch.data() + H, scratch.data() + 2 * H,
+                  head_k);
+  return SPARSED_OK;
+}
+
+int sparsed_select_head_entropy(const uint16_t* Q, const uint16_t* K, const uint16_t* V, int H, int L, int d,
+                                float scale, int bq, int bk, uint16_t* O, float* LSE, double* head_entropy,
+                                void* workspace, size_t workspace_bytes, void* stream) {
+  Problem p;
+  bool empty = false;
+  SP_TRY(prepare(Q, K, V, H, L, d, scale, bq, bk, O, LSE, &p, &empty));
+  if (empty) return SPARSED_OK;
+  if (!head_entropy) return SPARSED_ERR_INVALID_ARG;
+  if (static_cast<long long>(p.H) * p.nqb * p.nkb >= (1ll << 31)) return SPARSED_ERR_UNSUPPORTED;
+  const Workspace w = ws_layout(p.H, p.nqb, p.nkb);
+  if (!workspace || workspace_bytes < w.total) return SPARSED_ERR_WORKSPACE;
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return SPARSED_ERR_WORKSPACE;
+  SP_TRY(require_sm100());
+  SP_TRY(get_encoder());
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  float* mass = reinterpret_cast<float*>(ws + w.grid);
+  double* ent = reinterpret_cast<double*>(ws + w.ent);
+  SP_TRY(launch_attn(p, false, nullptr, nullptr, 0, st));
+  SP_TRY(launch_mass(p, mass, st));
+  const int rows = p.H * p.nqb;
+  row_entropy_kernel<<<(rows + 7) / 8, 256, 0, st>>>(mass, rows, p.nkb, ent);
+  SP_CUDA(cudaGetLastError());
+  head_entropy_kernel<<<(p.H + 255) / 256, 256, 0, st>>>(ent, p.H, p.nqb, head_entropy);
+  SP_CUDA(cudaGetLastError());
+  return SPARSED_OK;
+}
+
+int sparsed_select_with_head_k(int H, int L, int bq, int bk, const int32_t* head_k, int32_t* kv_idx,
+                               int32_t* kv_count, int kv_stride, void* workspace, size_t workspace_bytes,
+                               void* stream) {
+  if (H < 0 || L < 0) return SPARSED_ERR_INVALID_ARG;
+  if ((bq != 64 && bq != 128) || (bk != 64 && bk != 128)) return SPARSED_ERR_UNSUPPORTED;
+  if (static_cast<long>(H) * L == 0) return SPARSED_OK;
+  const int nqb = static_cast<int>(cdiv(L, bq)), nkb = static_cast<int>(cdiv(L, bk));
+  if (!head_k || !kv_idx || !kv_count || kv_stride < nkb) return SPARSED_ERR_INVALID_ARG;
+  if (static_cast<long long>(H) * nqb * kv_stride >= (1ll << 31)) return SPARSED_ERR_UNSUPPORTED;
+  const Workspace w = ws_layout(H, nqb, nkb);
+  if (!workspace || workspace_bytes < w.total) return SPARSED_ERR_WORKSPACE;
+  SP_TRY(require_sm100());
+  const float* mass = reinterpret_cast<const float*>(static_cast<uint8_t*>(workspace) + w.grid);
+  const int rows = H * nqb;
+  topk_kernel<<<(rows + 7) / 8, 256, 0, static_cast<cudaStream_t>(stream)>>>(mass, rows, nqb, nkb, 0, head_k,
+                                                                              nullptr, kv_idx, kv_count, kv_stride);
+  SP_CUDA(cudaGetLastError());
+  return SPARSED_OK;
+}
+
 int sparsed_column_keep(int L, float keep_ratio, int* kc) {
   if (!kc || L < 1 || !(keep_ratio > 0.f && keep_ratio <= 1.f)) return SPARSED_ERR_INVALID_ARG;
   *kc = uniform_k(L, keep_ratio);

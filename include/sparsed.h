@@ -198,6 +198,36 @@ int sparsed_run_steps(const uint16_t* Q, const uint16_t* K, const uint16_t* V,
                       int8_t* step_kind, float* step_ms,
                       void* workspace, size_t workspace_bytes, void* stream);
 
+/* ---- Head-sharded selection with the entropy budget (the heads of one
+ * layer split over several GPUs: only the per-head entropies cross ranks, one
+ * all-gather of H doubles per selection; Step-dLLM abstract: head-adaptive
+ * global budget). The three calls below, with the entropies of all heads
+ * gathered in head order between the first and the second, give every head
+ * the same k_h, kv_idx and kv_count as sparsed_select_pattern with
+ * SPARSED_BUDGET_ENTROPY on the whole layer. */
+
+/* Steps 1-2 of sparsed_select_pattern for this rank's H heads, then the mean
+ * row entropy E_h of every head (as in the ENTROPY budget) into head_entropy
+ * (DEVICE [H] fp64). The block mass stays in the workspace (at least
+ * sparsed_workspace_bytes(H, L, bq, bk) bytes) for sparsed_select_with_head_k. */
+int sparsed_select_head_entropy(const uint16_t* Q, const uint16_t* K, const uint16_t* V,
+                                int H, int L, int d, float scale, int bq, int bk,
+                                uint16_t* O, float* LSE, double* head_entropy,
+                                void* workspace, size_t workspace_bytes, void* stream);
+
+/* The ENTROPY budget allocation of sparsed_select_pattern on the HOST: from
+ * the entropies of all H heads of the layer (HOST [H] fp64) to k_h (HOST [H]
+ * int32). Runs without a GPU; identical to the device allocation. */
+int sparsed_entropy_budget(const double* head_entropy, int H, int nkb, float keep_ratio, int32_t* head_k);
+
+/* Step 4 of sparsed_select_pattern for this rank's H heads with given k_h
+ * (DEVICE [H] int32), over the block mass a preceding
+ * sparsed_select_head_entropy left in the same workspace (stream-ordered).
+ * kv_stride >= nkb. */
+int sparsed_select_with_head_k(int H, int L, int bq, int bk, const int32_t* head_k,
+                               int32_t* kv_idx, int32_t* kv_count, int kv_stride,
+                               void* workspace, size_t workspace_bytes, void* stream);
+
 /* ---- Column-sparse path (PulseCol: Periodically Refreshed Column-Sparse
  * Attention for Accelerating Diffusion Language Models, abstract: the sparse
  * pattern is a set of key columns of the attention map instead of blocks,
