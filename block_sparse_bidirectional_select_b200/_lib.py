@@ -35,6 +35,7 @@ SIGNATURES = {
     "sparsed_strerror": (ctypes.c_char_p, [_I]),
     "sparsed_last_cuda_error": (_I, []),
     "sparsed_check": (_I, [_P]),
+    "sparsed_selftest_wait_timeout": (_I, [ctypes.c_ulonglong, _P]),
     "sparsed_uniform_keep": (_I, [_I, _I, _F, ctypes.POINTER(_I)]),
     "sparsed_schedule": (_I, [_I, _F, _I, _P]),
     "sparsed_workspace_bytes": (_I, [_I, _I, _I, _I, ctypes.POINTER(_SZ)]),

@@ -128,6 +128,24 @@ int make_map(CUtensorMap* m, const void* ptr, int H, int L, int d, int box_rows)
   return SPARSED_OK;
 }
 
+// One thread waits on an mbarrier that nothing arrives on: the bounded wait
+// gives up after timeout_ns, records SPARSED_ERR_DEVICE_TIMEOUT in the device
+// error word and returns. No copy or MMA is in flight.
+__global__ void wait_timeout_selftest_kernel(unsigned long long timeout_ns) {
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    ptx::mbar_init(ptx::smem_u32(&bar), 1);
+    abort_flag = 0;
+    ptx::fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    volatile int* ab = &abort_flag;
+    ptx::mbar_wait(ptx::smem_u32(&bar), 0, ab, timeout_ns, kErrTimeout);
+  }
+}
+
 struct Problem {
   const uint16_t *Q, *K, *V;
   uint16_t* O;
@@ -480,6 +498,14 @@ int sparsed_check(void* stream) {
     SP_CUDA(cudaMemcpyToSymbol(ptx::g_device_error, &zero, sizeof(int)));
   }
   return code;
+}
+
+int sparsed_selftest_wait_timeout(unsigned long long timeout_ns, void* stream) {
+  if (timeout_ns == 0 || timeout_ns > 1000000000ull) return SPARSED_ERR_INVALID_ARG;
+  SP_TRY(require_sm100());
+  wait_timeout_selftest_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(timeout_ns);
+  SP_CUDA(cudaGetLastError());
+  return SPARSED_OK;
 }
 
 int sparsed_uniform_keep(int L, int bk, float keep_ratio, int* k_out) {

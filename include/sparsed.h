@@ -88,6 +88,13 @@ int sparsed_last_cuda_error(void);
  * (SPARSED_ERR_BAD_PATTERN or SPARSED_ERR_DEVICE_TIMEOUT), else SPARSED_OK. */
 int sparsed_check(void* stream);
 
+/* Self-test of the bounded device waits (not part of the method): launches one
+ * thread that waits on an mbarrier nothing arrives on; after timeout_ns
+ * (1 .. 1e9) it gives up, records SPARSED_ERR_DEVICE_TIMEOUT and returns, so
+ * the next sparsed_check reports that status and clears it. No copy or MMA is
+ * in flight, and the context stays usable. */
+int sparsed_selftest_wait_timeout(unsigned long long timeout_ns, void* stream);
+
 /* Host-only. Kept key blocks per query block under the uniform budget:
  * k = clamp(ceil(keep_ratio * nkb - 1e-6), 1, nkb), nkb = ceil(L/bk)
  * (Step-dLLM abstract: a uniform budget across heads; "90% sparsity" keeps

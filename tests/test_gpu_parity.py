@@ -1,6 +1,7 @@
 """CUDA path against the fp64 oracle, element by element, at sizes the oracle
 finishes in seconds (several tiles, ragged tails, every kernel variant), plus
 bitwise properties of the kernels and device-side error reporting."""
+import ctypes
 import math
 
 import numpy as np
@@ -314,6 +315,24 @@ def test_bad_pattern_is_reported_not_faulted():
     cnt = torch.tensor([[2, 2, 0, 1]], dtype=torch.int32, device="cuda")
     sp.block_sparse_attn(qc, kc, vc, idx, cnt)
     sp.device_check()
+
+
+def test_expired_device_wait_is_reported_and_the_context_stays_usable():
+    """A bounded device wait that runs out (an mbarrier nothing arrives on)
+    records SPARSED_ERR_DEVICE_TIMEOUT; the next check reports and clears it,
+    and the library keeps working."""
+    lib = sp._lib.load()
+    stream = torch.cuda.current_stream()
+    assert lib.sparsed_selftest_wait_timeout(2_000_000, ctypes.c_void_p(stream.cuda_stream)) == 0
+    with pytest.raises(sp.SparsedError) as e:
+        sp.device_check()
+    assert e.value.status == sp._lib.ERR_DEVICE_TIMEOUT
+    sp.device_check()
+    q, k, v, scale = _inputs(1, 256, 64, seed=9)
+    o, lse = sp.dense_attn(*_cuda(q, k, v), bq=64, bk=64)
+    sp.device_check()
+    o_ref, l_ref = oracle_dense_heads(q, k, v, scale)
+    assert_o_lse(o, lse, o_ref, l_ref, "after an expired wait")
 
 
 def test_empty_problem_is_noop():
