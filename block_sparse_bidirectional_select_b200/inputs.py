@@ -22,6 +22,21 @@ The banded term: seeded N(0,1) anchor vectors every 512 positions, linearly
 interpolated to every position p as z(p); z(p) is added to both Q[p] and K[p],
 so scores are raised for |i-j| within a few hundred positions and fall off by
 about 1024.
+
+Block-wise workloads (the LoSA setting: a block of B tokens denoised over T
+steps on a prefix of P cached tokens), ``BLOCK_WORKLOADS``:
+
+* ``losa_tiny``  H=2,  P=1000,  B=48, d=64,  bq=bk=64, 3 blocks per token, T=4
+* ``losa_32k``   H=32, P=32768, B=64, d=128, bq=bk=64, 2 blocks per token
+                 (128 prefix positions, the page's tightest budget), T=16
+
+Prefix K, V ~ N(0,1) with 10% of the prefix positions of every head raised by
++2.0 on every key component (as c2_8k). The block's Q, K, V start from N(0,1)
+and evolve in fp32: at every step t >= 1 a seeded round(0.25*B) tokens change
+by N(0, 0.5^2) per element (active), every other token by N(0, 0.02^2)
+(stable); each step's tensors are the fp32 state rounded to bf16. The query
+MSE of an active token is then about 0.25 and of a stable one about 4e-4, on
+either side of the threshold tau = 0.01.
 """
 from __future__ import annotations
 
@@ -137,3 +152,67 @@ def zero_q(wl: Workload):
 def to_f64(t: torch.Tensor):
     """Exact widening of bf16 bits to a float64 numpy array (no arithmetic)."""
     return t.detach().to("cpu").to(torch.float64).numpy()
+
+
+@dataclass(frozen=True)
+class BlockWorkload:
+    name: str
+    H: int
+    P: int            # prefix tokens (cached keys and values)
+    B: int            # block tokens
+    d: int
+    bq: int
+    bk: int
+    n_sel: int        # prefix blocks selected per token
+    T: int            # denoising steps of the block
+    active_frac: float
+    tau: float
+    seed: int
+
+    @property
+    def scale(self) -> float:
+        return float(torch.tensor(1.0 / math.sqrt(self.d), dtype=torch.float32))
+
+    def scaled(self, **kw) -> "BlockWorkload":
+        return replace(self, **kw)
+
+
+BLOCK_WORKLOADS = {
+    "losa_tiny": BlockWorkload("losa_tiny", 2, 1000, 48, 64, 64, 64, 3, 4, 0.25, 0.01, 2001),
+    "losa_32k": BlockWorkload("losa_32k", 32, 32768, 64, 128, 64, 64, 2, 16, 0.25, 0.01, 2002),
+}
+
+ACTIVE_STD = 0.5
+STABLE_STD = 0.02
+
+
+def make_block_inputs(wl: BlockWorkload, device: str | torch.device = "cpu"):
+    """Return (k_pre, v_pre, qs, ks, vs): the prefix [H, P, d] and the block's
+    per-step tensors [T, H, B, d], all bf16 on ``device``.
+
+    Draw order: prefix K, prefix V, the hot positions of each head, block Q,
+    K, V at step 0, then per step the active set and the changes of Q, K, V.
+    """
+    H, P, B, d, T = wl.H, wl.P, wl.B, wl.d, wl.T
+    g = torch.Generator("cpu").manual_seed(wl.seed)
+    k_pre = torch.randn((H, P, d), generator=g)
+    v_pre = torch.randn((H, P, d), generator=g)
+    n_hot = int(round(0.1 * P))
+    for h in range(H):
+        pos = torch.randperm(P, generator=g)[:n_hot]
+        k_pre[h, pos, :] += 2.0
+    state = [torch.randn((H, B, d), generator=g) for _ in range(3)]
+    n_act = int(round(wl.active_frac * B))
+    steps = [[t.to(torch.bfloat16) for t in state]]
+    for _ in range(1, T):
+        act = torch.randperm(B, generator=g)[:n_act]
+        std = torch.full((B,), STABLE_STD)
+        std[act] = ACTIVE_STD
+        for i in range(3):
+            state[i] = state[i] + torch.randn((H, B, d), generator=g) * std[None, :, None]
+        steps.append([t.to(torch.bfloat16) for t in state])
+    qs, ks, vs = (torch.stack([s[i] for s in steps]) for i in range(3))
+    out = [k_pre.to(torch.bfloat16), v_pre.to(torch.bfloat16), qs, ks, vs]
+    if str(device) != "cpu":
+        out = [t.to(device) for t in out]
+    return tuple(out)

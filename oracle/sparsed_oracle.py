@@ -21,6 +21,13 @@ the pages define (citations name the page title and the part of the page):
 * PulseCol: Periodically Refreshed Column-Sparse Attention for Accelerating
   Diffusion Language Models, abstract -- the same periodic-refresh schedule,
   and column-level (per key position) instead of block-level sparsity.
+* LoSA: Locality Aware Sparse Attention for Block-Wise Diffusion Language
+  Models (a Dutch summary page) -- block-wise generation over a prefix KV
+  cache: per step, tokens whose query changed are "active" and get sparse
+  prefix attention over the union of their selections; "stable" tokens reuse
+  their cached prefix output; prefix and in-block parts are merged by their
+  log-sum-exp (section 1, the union cost; section 2, locality of the query
+  change; section 3, the method and its workflow).
 
 Where the pages leave a step open, the reading taken is stated in the function
 docstring (rule for what is scored, rounding of k, tie-break, list order, the
@@ -493,3 +500,190 @@ def run_steps_columns(q, k, v, scale, keep_ratio, T, warmup_frac, refresh_every=
 def effective_flops(bq, bk, d, kept_blocks):
     """Flops of QK^T plus PV over the kept blocks: 4 * bq * bk * d per block."""
     return 4.0 * bq * bk * d * float(kept_blocks)
+
+
+# --------------------------------------------------------------------------
+# O8  block-wise generation with active-token reuse (LoSA)
+# --------------------------------------------------------------------------
+#
+# Setting (LoSA page, section 1): a block of B tokens is denoised over several
+# steps on top of a prefix of P tokens whose keys and values are cached and
+# fixed while the block is generated. At every step each block token attends
+# bidirectionally to the whole block (the "suffix": the block's own current
+# keys and values) and to the prefix. Arrays: one head is [rows, d]; all heads
+# are [H, rows, d]; prefix key block j covers positions [j*bk, min((j+1)*bk, P)).
+
+
+def merge_partials(o1, lse1, o2, lse2):
+    """Attention over the union of two disjoint key sets from the attention
+    over each set: with m = max(lse1, lse2) and w_i = exp(lse_i - m),
+        o = (w1*o1 + w2*o2) / (w1 + w2),   lse = m + ln(w1 + w2).
+
+    LoSA page, section 3 (methodology), workflow: the prefix and suffix
+    contributions are combined by online softmax; this is that identity
+    applied once. A part over no keys (lse = -inf) contributes nothing; two
+    empty parts give o = 0, lse = -inf."""
+    o1, o2 = np.asarray(o1, dtype=np.float64), np.asarray(o2, dtype=np.float64)
+    lse1, lse2 = np.asarray(lse1, dtype=np.float64), np.asarray(lse2, dtype=np.float64)
+    m = np.maximum(lse1, lse2)
+    both_empty = np.isneginf(m)
+    msafe = np.where(both_empty, 0.0, m)
+    w1 = np.where(np.isneginf(lse1), 0.0, np.exp(lse1 - msafe))
+    w2 = np.where(np.isneginf(lse2), 0.0, np.exp(lse2 - msafe))
+    z = w1 + w2
+    zsafe = np.where(both_empty, 1.0, z)
+    o = (w1[..., None] * o1 + w2[..., None] * o2) / zsafe[..., None]
+    o = np.where(both_empty[..., None], 0.0, o)
+    lse = np.where(both_empty, -np.inf, msafe + np.log(zsafe))
+    return o, lse
+
+
+def query_mse(q_t, q_prev):
+    """Locality score of every block token: the mean squared change of its
+    query between two consecutive denoising steps,
+        mse_b = 1/(H*d) * sum_h sum_c (q_t[h,b,c] - q_prev[h,b,c])^2.
+
+    LoSA page, section 2 (only a few tokens change much between steps t-1 and
+    t, shown by MSE measurements) and section 3 (locality pruning measures the
+    query change of every token by MSE at the start of a step). Reading taken:
+    one score per token over its whole query vector (every head), so all heads
+    share one active set. q_t, q_prev are [H, B, d]; returns [B]."""
+    diff = np.asarray(q_t, dtype=np.float64) - np.asarray(q_prev, dtype=np.float64)
+    return (diff * diff).mean(axis=(0, 2))
+
+
+def active_tokens(mse, tau):
+    """Active tokens: mse_b > tau, strictly (LoSA page, section 3: tokens with
+    a high change are active, the rest stable). Reading taken: "high" is a
+    caller-given threshold tau, an fp32 value widened to double."""
+    return np.asarray(mse, dtype=np.float64) > float(np.float32(tau))
+
+
+def token_block_mass(q, k_pre, scale, lse, bk):
+    """Per-token prefix block mass of one head,
+        M[b, j] = sum over prefix keys c in block j of exp(scale*<q_b,k_c> - lse_b),
+    i.e. the block mass of O2 with query blocks of a single row.
+
+    The selector of the active tokens (LoSA page, section 3: the method works
+    with any sparse selector; the page names QUEST only by name). Reading
+    taken: the selector of the SparseD abstract -- the pattern is computed once
+    from full attention and reused -- at token granularity: each block token's
+    prefix blocks are scored by its post-softmax mass in the block's first,
+    dense step, with ``lse`` that step's prefix LSE of the token."""
+    return block_mass(q, k_pre, scale, lse, 1, bk)
+
+
+def token_select(M, n_sel):
+    """Per token, its ``n_sel`` prefix blocks of largest mass (``topk_blocks``:
+    ties to the lower block, ascending). n_sel is clamped to [1, nkb].
+    Returns [B, n_sel'] int32."""
+    M = np.asarray(M, dtype=np.float64)
+    k = min(max(int(n_sel), 1), M.shape[1])
+    return np.stack([topk_blocks(M[b], k) for b in range(M.shape[0])]).astype(np.int32)
+
+
+def kv_union(sel, active):
+    """The prefix blocks one head loads in a step: the union, over the active
+    tokens, of their selected blocks, ascending (LoSA page, section 1: the cost
+    of a block's sparse attention is set by the union of the positions its
+    queries select; section 3: the selector's output for the active tokens only
+    forms the union that is loaded). Returns int32 [u]."""
+    rows = np.nonzero(np.asarray(active))[0]
+    if rows.size == 0:
+        return np.zeros(0, dtype=np.int32)
+    return np.unique(np.asarray(sel)[rows].ravel()).astype(np.int32)
+
+
+def prefix_attention(q_rows, k_pre, v_pre, scale, blocks, bk):
+    """Attention of the given query rows over every prefix key of the listed
+    blocks, in ascending key order (LoSA page, section 3: only the union's
+    positions are loaded and the active tokens' prefix attention is computed
+    over them). Reading taken: each active token attends to the whole loaded
+    union, not only to its own selection."""
+    keys = kept_keys(blocks, bk, np.asarray(k_pre).shape[0])
+    return softmax_attention(q_rows, np.asarray(k_pre)[keys], np.asarray(v_pre)[keys], scale)
+
+
+def losa_init(q, k, v, k_pre, v_pre, scale, bk, n_sel):
+    """First denoising step of a block (LoSA page, section 3, workflow,
+    initialisation: dense attention fills the cache).
+
+    For every head and block token: the prefix attention over all P prefix
+    keys is the cached prefix output and LSE; its per-token block mass gives
+    the token's ``n_sel`` blocks (``token_block_mass``); the suffix attention
+    is dense over the block; the step's output merges the two.
+    q, k, v: [H, B, d]; k_pre, v_pre: [H, P, d]. Returns dict with o [H,B,d],
+    lse [H,B], mass [H,B,nkb] and state = {o_pre, lse_pre, sel [H,B,n_sel']}."""
+    H, B, d = np.asarray(q).shape
+    o = np.empty((H, B, d))
+    lse = np.empty((H, B))
+    o_pre = np.empty((H, B, d))
+    lse_pre = np.empty((H, B))
+    nkb = n_blocks(np.asarray(k_pre).shape[1], bk)
+    mass = np.empty((H, B, nkb))
+    sels = []
+    for h in range(H):
+        o_pre[h], lse_pre[h] = dense_attention(q[h], k_pre[h], v_pre[h], scale)
+        mass[h] = token_block_mass(q[h], k_pre[h], scale, lse_pre[h], bk)
+        sels.append(token_select(mass[h], n_sel))
+        o_suf, lse_suf = dense_attention(q[h], k[h], v[h], scale)
+        o[h], lse[h] = merge_partials(o_pre[h], lse_pre[h], o_suf, lse_suf)
+    state = dict(o_pre=o_pre, lse_pre=lse_pre, sel=np.stack(sels))
+    return dict(o=o, lse=lse, mass=mass, state=state)
+
+
+def losa_step(q, k, v, q_prev, k_pre, v_pre, scale, bk, tau, state):
+    """A later denoising step of the block (LoSA page, section 3, workflow,
+    iteration), in the page's order:
+      1. locality scores (``query_mse``) against the previous step's queries,
+         active tokens (``active_tokens``);
+      2. per head, the union of the active tokens' selected blocks
+         (``kv_union``);
+      3. only those blocks are read;
+      4. the active tokens' prefix attention over the union replaces their
+         cached prefix output and LSE; stable tokens keep theirs (section 3,
+         reuse for stable tokens);
+      5. every token's suffix attention (dense over the block) is merged with
+         its prefix part (``merge_partials``).
+    ``state`` (from ``losa_init`` or an earlier step) is updated in place.
+    Returns dict with o, lse, mse [B], active [B] bool, union (list of H
+    int32 arrays)."""
+    H, B, d = np.asarray(q).shape
+    mse = query_mse(q, q_prev)
+    act = active_tokens(mse, tau)
+    rows = np.nonzero(act)[0]
+    o = np.empty((H, B, d))
+    lse = np.empty((H, B))
+    unions = []
+    for h in range(H):
+        u = kv_union(state["sel"][h], act)
+        unions.append(u)
+        if rows.size:
+            o_a, l_a = prefix_attention(np.asarray(q[h])[rows], k_pre[h], v_pre[h], scale, u, bk)
+            state["o_pre"][h][rows] = o_a
+            state["lse_pre"][h][rows] = l_a
+        o_suf, lse_suf = dense_attention(q[h], k[h], v[h], scale)
+        o[h], lse[h] = merge_partials(state["o_pre"][h], state["lse_pre"][h], o_suf, lse_suf)
+    return dict(o=o, lse=lse, mse=mse, active=act, union=unions)
+
+
+def losa_block(qs, ks, vs, k_pre, v_pre, scale, bk, n_sel, tau):
+    """All T denoising steps of one block: ``losa_init`` at step 0, then
+    ``losa_step`` with the previous step's queries. qs, ks, vs: [T, H, B, d].
+    Returns dict with o [T,H,B,d], lse [T,H,B], active [T,B] (step 0: all),
+    union_count [T,H] (step 0: every prefix block), state."""
+    T, H, B, d = np.asarray(qs).shape
+    nkb = n_blocks(np.asarray(k_pre).shape[1], bk)
+    o = np.empty((T, H, B, d))
+    lse = np.empty((T, H, B))
+    active = np.ones((T, B), dtype=bool)
+    ucount = np.full((T, H), nkb, dtype=np.int64)
+    first = losa_init(qs[0], ks[0], vs[0], k_pre, v_pre, scale, bk, n_sel)
+    o[0], lse[0] = first["o"], first["lse"]
+    state = first["state"]
+    for t in range(1, T):
+        r = losa_step(qs[t], ks[t], vs[t], qs[t - 1], k_pre, v_pre, scale, bk, tau, state)
+        o[t], lse[t] = r["o"], r["lse"]
+        active[t] = r["active"]
+        ucount[t] = [len(u) for u in r["union"]]
+    return dict(o=o, lse=lse, active=active, union_count=ucount, state=state)
