@@ -37,7 +37,8 @@ import torch
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-from block_sparse_bidirectional_select_b200.inputs import WORKLOADS, make_inputs, to_f64  # noqa: E402
+from block_sparse_bidirectional_select_b200.inputs import (BLOCK_WORKLOADS, WORKLOADS, make_block_inputs,  # noqa: E402
+                                                           make_inputs, to_f64)
 
 METRIC = "block-sparse attn effective TFLOP/s & ms/step at 64k, % of B200 bf16 peak"
 UNIT = "TFLOP/s"
@@ -288,9 +289,11 @@ def main():
                     help="run: the full denoising run (the benchmark); dense/sparse/select and the column "
                          "path's col_sparse/col_select: time one library call alone, K launches after W "
                          "warm-up launches (for profiling)")
-    ap.add_argument("--path", choices=["blocks", "columns"], default="blocks",
+    ap.add_argument("--path", choices=["blocks", "columns", "losa"], default="blocks",
                     help="blocks: the block-sparse path (the benchmark); columns: the same denoising run "
-                         "with the column-sparse pattern")
+                         "with the column-sparse pattern; losa: block-wise generation over a prefix cache "
+                         "with active-token reuse (--block-workload)")
+    ap.add_argument("--block-workload", default="losa_32k", choices=sorted(BLOCK_WORKLOADS))
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     rank = int(os.environ.get("RANK", "0"))
@@ -319,6 +322,8 @@ def main():
         return time_one_op(args, wl, dev, rank)
     if args.path == "columns":
         return run_columns(args, wl, dev, rank, world, barrier, max_over_ranks)
+    if args.path == "losa":
+        return run_losa(args, dev, rank, world, barrier, max_over_ranks)
     log(f"[rank {rank}] inputs for {wl.name}")
     q_cpu, k_cpu, v_cpu = make_inputs(rank_workload(wl, rank))
     q, k, v = (t.to(dev) for t in (q_cpu, k_cpu, v_cpu))
@@ -585,6 +590,111 @@ def run_columns(args, wl, dev, rank, world, barrier, max_over_ranks):
                                    "frac_of_peak_burst": sparse / (ms_alone * 1e-3) / 1e12 / peak_burst,
                                    "peak_source": peak_src},
             "gpu_launches": (n_dense + 3 * n_select + 2 * n_sparse) * args.steps, "clocks": clk}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+def losa_bytes(wl, union_counts):
+    """Algorithmic HBM bytes of one block run: the first step reads the whole
+    prefix K and V; a later step reads the K and V rows of its heads' unions;
+    every step reads the block's Q, K, V (and the previous Q) and writes O and
+    LSE. union_counts: [T, H] blocks per head (step 0: all)."""
+    row = wl.d * 2
+    full = 2 * wl.H * wl.P * row
+    blk = wl.H * wl.B * (4 * row + 4)
+    per_step = [full + blk]
+    for t in range(1, union_counts.shape[0]):
+        keys = float(union_counts[t].sum()) * wl.bk  # a ragged last prefix block counts whole
+        per_step.append(2 * keys * row + blk + wl.H * wl.B * row)
+    return per_step
+
+
+def run_losa(args, dev, rank, world, barrier, max_over_ranks):
+    """Block-wise generation (LoSA page, section 3): one bench step is one
+    block's T denoising steps through sparsed_losa_block -- a dense first step
+    over the whole prefix (and the per-token selection), then steps in which
+    only the active tokens attend to the union of their blocks. The path is
+    bound by HBM reads of the prefix cache: value = algorithmic bytes of the
+    run / device time (GB/s). The L2 is flushed before every timed run."""
+    import block_sparse_bidirectional_select_b200 as sp
+    wl = BLOCK_WORKLOADS[args.block_workload]
+    k_pre, v_pre, qs, ks, vs = (t.to(dev) for t in make_block_inputs(wl.scaled(seed=wl.seed + 7919 * rank)))
+    stream = torch.cuda.current_stream()
+    splits = sp.losa_splits(wl.H, wl.B, wl.P, wl.bq, wl.bk)
+    ws = torch.empty(sp.losa_workspace_bytes(wl.H, wl.B, wl.P, wl.d, wl.bq, wl.bk, splits), dtype=torch.uint8,
+                     device=dev)
+    out = torch.empty_like(qs)
+    lse = torch.empty((wl.T, wl.H, wl.B), dtype=torch.float32, device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+
+    def one_run():
+        return sp.losa_block(qs, ks, vs, k_pre, v_pre, n_sel=wl.n_sel, tau=wl.tau, bq=wl.bq, bk=wl.bk,
+                             splits=splits, out=out, lse=lse, workspace=ws)
+
+    for _ in range(args.warmup):
+        res = one_run()
+    sp.device_check()
+    ucount = res.union_count.cpu().numpy()
+    n_active = res.active.cpu().numpy().sum(axis=1)
+    per_step_bytes = losa_bytes(wl, ucount)
+    run_bytes = float(sum(per_step_bytes))
+    torch.cuda.synchronize()
+    barrier()
+    clocks = ClockSampler(dev.index or 0)
+    clocks.start()
+    total = 0.0
+    for _ in range(args.steps):
+        flush.zero_()
+        s_ev = torch.cuda.Event(enable_timing=True)
+        e_ev = torch.cuda.Event(enable_timing=True)
+        s_ev.record(stream)
+        one_run()
+        e_ev.record(stream)
+        e_ev.synchronize()
+        total += s_ev.elapsed_time(e_ev)
+    barrier()
+    clk = clocks.stop()
+    total_ms = max_over_ranks(total)
+    sp.device_check()
+    # the steps one by one, each timed with events (the first step after an L2 flush)
+    flush.zero_()
+    times = []
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(wl.T + 1)]
+    ev[0].record(stream)
+    _, _, st = sp.losa_init(qs[0], ks[0], vs[0], k_pre, v_pre, n_sel=wl.n_sel, bq=wl.bq, bk=wl.bk,
+                            splits=splits, workspace=ws)
+    ev[1].record(stream)
+    for t in range(1, wl.T):
+        sp.losa_step(qs[t], ks[t], vs[t], qs[t - 1], k_pre, v_pre, st, wl.tau)
+        ev[t + 1].record(stream)
+    ev[-1].synchronize()
+    times = [ev[t].elapsed_time(ev[t + 1]) for t in range(wl.T)]
+    sp.device_check()
+    peaks, peak_src = load_peaks()
+    hbm = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
+    gbs = run_bytes * args.steps * world / (total_ms * 1e-3) / 1e9
+    step_ms = statistics.mean(times[1:]) if wl.T > 1 else None
+    step_bytes = statistics.mean(per_step_bytes[1:]) if wl.T > 1 else None
+    nkb = -(-wl.P // wl.bk)
+    line = {"metric": "block-wise generation with active-token reuse: HBM GB/s of a block's steps",
+            "value": gbs, "unit": "GB/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": total_ms / args.steps, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": wl.name, "H": wl.H, "prefix": wl.P, "block": wl.B, "d": wl.d, "bq": wl.bq,
+                       "bk": wl.bk, "blocks_per_token": wl.n_sel, "T": wl.T, "tau": wl.tau, "splits": splits,
+                       "l2": "flushed before every timed run"},
+            "ms_per_denoise_step": total_ms / args.steps / wl.T,
+            "first_step_ms": times[0], "later_step_ms": step_ms,
+            "active_tokens_per_step": float(n_active[1:].mean()) if wl.T > 1 else None,
+            "union_blocks_per_head": float(ucount[1:].mean()) if wl.T > 1 else None,
+            "prefix_density": float(ucount[1:].mean()) / nkb if wl.T > 1 else None,
+            "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm, "unit": "GB/s", "frac": gbs / hbm,
+                         "traffic": None, "peak_source": peak_src},
+            "later_step_roofline": None if step_ms is None else
+            {"bound": "hbm", "achieved": step_bytes / (step_ms * 1e-3) / 1e9, "peak": hbm, "unit": "GB/s",
+             "frac": step_bytes / (step_ms * 1e-3) / 1e9 / hbm, "bytes": step_bytes},
+            "gpu_launches": (6 + 5 * (wl.T - 1) + 2) * args.steps, "clocks": clk}
     if rank == 0:
         print(json.dumps(line), flush=True)
     return 0

@@ -22,6 +22,13 @@ Column-sparse path (per-head kept key columns shared by all queries):
     column_sparse_attn(q, k, v, cols)        -> (o, lse)
     run_steps_columns(q, k, v, T, warmup_frac, ...) -> RunResult (kv_idx holds cols [H, kc])
 
+Block-wise generation over a prefix cache with active-token reuse (a block
+of B tokens denoised over T steps; q, k, v of the block are [H, B, d]):
+
+    losa_init(q, k, v, k_pre, v_pre, n_sel)  -> (o, lse, BlockState)
+    losa_step(q, k, v, q_prev, k_pre, v_pre, state, tau) -> LosaStep
+    losa_block(qs, ks, vs, k_pre, v_pre, n_sel, tau) -> LosaBlock (all T steps)
+
 q, k, v are [H, L, d] bf16 CUDA tensors (d in {64, 128}); o is [H, L, d] bf16,
 lse [H, L] fp32 natural log; kv_idx [H, nqb, kv_stride] int32 and kv_count
 [H, nqb] int32 hold the per-(head, query block) kept key blocks, ascending.
@@ -43,7 +50,9 @@ __all__ = ["dense_attn", "select_pattern", "block_sparse_attn", "run_steps", "wo
            "uniform_keep", "schedule", "device_check", "version", "SparsedError", "Pattern",
            "RunResult", "default_scale", "column_keep", "column_workspace_bytes", "select_columns",
            "column_sparse_attn", "run_steps_columns", "ColumnPattern", "select_head_entropy",
-           "entropy_budget", "select_with_head_k", "select_pattern_sharded", "gather_head_entropies"]
+           "entropy_budget", "select_with_head_k", "select_pattern_sharded", "gather_head_entropies",
+           "losa_splits", "losa_workspace_bytes", "losa_init", "losa_step", "losa_block", "BlockState",
+           "LosaStep", "LosaBlock"]
 
 
 def _ptr(t: torch.Tensor | None):
@@ -398,3 +407,145 @@ def select_pattern_sharded(q, k, v, keep=0.1, group=None, scale=None, bq=128, bk
     head_k_all = entropy_budget(ent_all.tolist(), nkb, keep)
     kv_idx, kv_count, hk = select_with_head_k(H, L, head_k_all[rank * H:(rank + 1) * H], ws, bq, bk, stream)
     return Pattern(out, lse, kv_idx, kv_count, None, hk)
+
+
+# ---------------------------------------------------------------- block-wise generation with active-token reuse
+
+def losa_splits(H: int, B: int, P: int, bq: int = 64, bk: int = 64, sm_count: int | None = None) -> int:
+    """Splits of a head's block list for a step of these sizes (sm_count: the
+    current device's SM count by default)."""
+    if sm_count is None:
+        sm_count = torch.cuda.get_device_properties(torch.cuda.current_device()).multi_processor_count
+    s = ctypes.c_int()
+    check(_lib.load().sparsed_losa_splits(H, B, bq, P, bk, sm_count, ctypes.byref(s)), "sparsed_losa_splits")
+    return s.value
+
+
+def losa_workspace_bytes(H: int, B: int, P: int, d: int, bq: int = 64, bk: int = 64, splits: int = 1) -> int:
+    n = ctypes.c_size_t()
+    check(_lib.load().sparsed_losa_workspace_bytes(H, B, P, d, bq, bk, splits, ctypes.byref(n)),
+          "sparsed_losa_workspace_bytes")
+    return n.value
+
+
+@dataclass
+class BlockState:
+    """What a block carries across its denoising steps (caller memory)."""
+    o_cache: torch.Tensor    # [H, B, d] bf16: every token's prefix attention output
+    lse_cache: torch.Tensor  # [H, B] fp32: its LSE over the prefix keys it attended
+    sel: torch.Tensor        # [H, B, n_sel] int32: each token's prefix blocks, ascending
+    scale: float
+    bq: int
+    bk: int
+    splits: int
+    workspace: torch.Tensor
+
+
+@dataclass
+class LosaStep:
+    o: torch.Tensor
+    lse: torch.Tensor
+    active: torch.Tensor            # [B] int32 0/1
+    union_count: torch.Tensor       # [H] int32
+    union_idx: torch.Tensor | None  # [H, nkb] int32, first union_count[h] entries
+
+
+@dataclass
+class LosaBlock:
+    o: torch.Tensor            # [T, H, B, d]
+    lse: torch.Tensor          # [T, H, B]
+    active: torch.Tensor       # [T, B] int32 (step 0: all 1)
+    union_count: torch.Tensor  # [T, H] int32 (step 0: nkb)
+    state: BlockState
+
+
+def _check_prefix(k_pre, v_pre, H, d, device):
+    for name, t in (("k_pre", k_pre), ("v_pre", v_pre)):
+        if not isinstance(t, torch.Tensor) or t.dtype != torch.bfloat16 or t.device != device \
+                or t.dim() != 3 or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous [H, P, d] bf16 tensor on {device}")
+    if k_pre.shape != v_pre.shape or k_pre.shape[0] != H or k_pre.shape[2] != d:
+        raise ValueError(f"prefix shapes {tuple(k_pre.shape)} / {tuple(v_pre.shape)} do not match H={H}, d={d}")
+    return k_pre.shape[1]
+
+
+def _block_state(q, P, n_sel, scale, bq, bk, splits, workspace):
+    H, B, d = q.shape
+    splits = losa_splits(H, B, P, bq, bk) if splits is None else splits
+    need = losa_workspace_bytes(H, B, P, d, bq, bk, splits)
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    return BlockState(torch.empty_like(q), torch.empty((H, B), dtype=torch.float32, device=q.device),
+                      torch.empty((H, B, n_sel), dtype=torch.int32, device=q.device), scale, bq, bk, splits,
+                      workspace)
+
+
+def losa_init(q, k, v, k_pre, v_pre, n_sel=2, scale=None, bq=64, bk=64, splits=None, return_mass=False,
+              workspace=None, stream=None):
+    """First denoising step of a block: dense prefix attention of every token
+    (the cache), each token's n_sel prefix blocks, the block's own attention
+    and the merged output. Returns (o, lse, state) or (o, lse, state, mass)."""
+    H, B, d = _check_qkv(q, k, v)
+    P = _check_prefix(k_pre, v_pre, H, d, q.device)
+    scale = default_scale(d) if scale is None else scale
+    st = _block_state(q, P, n_sel, scale, bq, bk, splits, workspace)
+    out, lse = _alloc_out(q, None, None)
+    nkb = (P + bk - 1) // bk
+    mass = torch.empty((H, B, nkb), dtype=torch.float32, device=q.device) if return_mass else None
+    rc = _lib.load().sparsed_losa_init(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(k_pre), _ptr(v_pre), H, B, P, d, scale, bq, bk, n_sel, st.splits,
+        _ptr(st.o_cache), _ptr(st.lse_cache), _ptr(st.sel), _ptr(out), _ptr(lse), _ptr(mass),
+        _ptr(st.workspace), st.workspace.numel(), _stream(stream))
+    check(rc, "sparsed_losa_init")
+    return (out, lse, st, mass) if return_mass else (out, lse, st)
+
+
+def losa_step(q, k, v, q_prev, k_pre, v_pre, state: BlockState, tau: float, return_union=False,
+              stream=None) -> LosaStep:
+    """A later step of the block: active tokens by query MSE against q_prev,
+    the union of their blocks, their prefix attention over it (cache update),
+    the block's own attention, and the merge. Updates ``state`` in place."""
+    H, B, d = _check_qkv(q, k, v)
+    _check_qkv(q, q_prev, q_prev)
+    P = _check_prefix(k_pre, v_pre, H, d, q.device)
+    n_sel = state.sel.shape[2]
+    out, lse = _alloc_out(q, None, None)
+    active = torch.empty(B, dtype=torch.int32, device=q.device)
+    ucount = torch.empty(H, dtype=torch.int32, device=q.device)
+    nkb = (P + state.bk - 1) // state.bk
+    uidx = torch.empty((H, nkb), dtype=torch.int32, device=q.device) if return_union else None
+    rc = _lib.load().sparsed_losa_step(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(q_prev), _ptr(k_pre), _ptr(v_pre), H, B, P, d, state.scale, state.bq,
+        state.bk, n_sel, tau, state.splits, _ptr(state.o_cache), _ptr(state.lse_cache), _ptr(state.sel),
+        _ptr(out), _ptr(lse), _ptr(active), _ptr(uidx), _ptr(ucount), _ptr(state.workspace),
+        state.workspace.numel(), _stream(stream))
+    check(rc, "sparsed_losa_step")
+    return LosaStep(out, lse, active, ucount, uidx)
+
+
+def losa_block(qs, ks, vs, k_pre, v_pre, n_sel=2, tau=0.01, scale=None, bq=64, bk=64, splits=None, out=None,
+               lse=None, workspace=None, stream=None) -> LosaBlock:
+    """All T steps of one block (qs, ks, vs: [T, H, B, d] bf16): the first
+    step dense, every later one with active-token reuse."""
+    for name, t in (("qs", qs), ("ks", ks), ("vs", vs)):
+        if not isinstance(t, torch.Tensor) or t.dtype != torch.bfloat16 or t.device.type != "cuda" \
+                or t.dim() != 4 or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous [T, H, B, d] bf16 CUDA tensor")
+    if not (qs.shape == ks.shape == vs.shape):
+        raise ValueError("qs, ks, vs shapes differ")
+    T, H, B, d = qs.shape
+    P = _check_prefix(k_pre, v_pre, H, d, qs.device)
+    scale = default_scale(d) if scale is None else scale
+    st = _block_state(qs[0], P, n_sel, scale, bq, bk, splits, workspace)
+    if out is None:
+        out = torch.empty_like(qs)
+    if lse is None:
+        lse = torch.empty((T, H, B), dtype=torch.float32, device=qs.device)
+    active = torch.empty((T, B), dtype=torch.int32, device=qs.device)
+    ucount = torch.empty((T, H), dtype=torch.int32, device=qs.device)
+    rc = _lib.load().sparsed_losa_block(
+        _ptr(qs), _ptr(ks), _ptr(vs), _ptr(k_pre), _ptr(v_pre), T, H, B, P, d, scale, bq, bk, n_sel, tau,
+        st.splits, _ptr(st.o_cache), _ptr(st.lse_cache), _ptr(st.sel), _ptr(out), _ptr(lse), _ptr(active),
+        _ptr(ucount), _ptr(st.workspace), st.workspace.numel(), _stream(stream))
+    check(rc, "sparsed_losa_block")
+    return LosaBlock(out, lse, active, ucount, st)

@@ -57,6 +57,14 @@ SIGNATURES = {
     "sparsed_column_sparse_attn": (_I, [_P, _P, _P, _I, _I, _I, _F, _I, _I, _P, _I, _I, _P, _P, _P, _SZ, _P]),
     "sparsed_run_steps_columns": (_I, [_P, _P, _P, _I, _I, _I, _F, _I, _I, _F, _I, _F, _I, _I, _I, _P, _I,
                                        _P, _P, _P, _P, _P, _SZ, _P]),
+    "sparsed_losa_splits": (_I, [_I, _I, _I, _I, _I, _I, ctypes.POINTER(_I)]),
+    "sparsed_losa_workspace_bytes": (_I, [_I, _I, _I, _I, _I, _I, _I, ctypes.POINTER(_SZ)]),
+    "sparsed_losa_init": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _F, _I, _I, _I, _I, _P, _P, _P, _P, _P,
+                               _P, _P, _SZ, _P]),
+    "sparsed_losa_step": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _F, _I, _I, _I, _F, _I, _P, _P, _P,
+                               _P, _P, _P, _P, _P, _P, _SZ, _P]),
+    "sparsed_losa_block": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _I, _I, _I, _F, _I, _P, _P, _P,
+                                _P, _P, _P, _P, _P, _SZ, _P]),
 }
 
 _lib = None

@@ -1,7 +1,8 @@
 // Host side of the C ABI declared in include/sparsed.h: argument validation,
 // workspace layout, TMA descriptor encoding, kernel launches and the
-// denoising-step driver. Every step of the computation runs in the kernels of
-// attn_kernel.cuh and select_kernels.cuh; nothing here computes attention.
+// denoising-step drivers. Every step of the computation runs in the kernels of
+// attn_kernel.cuh, select_kernels.cuh, column_kernels.cuh and
+// losa_kernels.cuh; nothing here computes attention.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <cuda_runtime.h>
@@ -17,6 +18,7 @@
 #include "attn_kernel.cuh"
 #include "select_kernels.cuh"
 #include "column_kernels.cuh"
+#include "losa_kernels.cuh"
 
 using namespace sparsed;
 
@@ -926,3 +928,363 @@ extern "C" int sparsed_select_pattern_noalloc(const uint16_t* Q, const uint16_t*
   return select_after_dense(p, keep_ratio, budget_mode, kv_idx, kv_count, kv_stride, block_mass, head_k,
                             scratch, st);
 }
+
+// ---- block-wise generation with active-token reuse (LoSA: Locality Aware
+// Sparse Attention for Block-Wise Diffusion Language Models, section 3)
+
+namespace {
+
+struct LosaDims {
+  int H, B, P, d, bq, bk;
+  int nkb;     // prefix key blocks
+  int n_sel;   // blocks selected per token, clamped to nkb
+  int S;       // splits of a head's block list
+  int tiles;   // query tiles of the block: ceil(B / bq)
+  int R;       // rows per split: tiles * bq
+  int stride;  // kv list row stride: the longest split
+};
+
+int losa_dims(int H, int B, int P, int d, int bq, int bk, int n_sel, int splits, LosaDims* g) {
+  if (H < 1 || B < 1 || P < 1 || n_sel < 1 || splits < 1) return SPARSED_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return SPARSED_ERR_UNSUPPORTED;
+  if ((bq != 64 && bq != 128) || (bk != 64 && bk != 128)) return SPARSED_ERR_UNSUPPORTED;
+  if (H > 65535 || B > kLosaMaxB) return SPARSED_ERR_UNSUPPORTED;
+  const long nkb = cdiv(P, bk);
+  if (nkb > static_cast<long>(kLosaMaxWords) * 32) return SPARSED_ERR_UNSUPPORTED;
+  if (static_cast<long long>(H) * P * d >= (1ll << 31)) return SPARSED_ERR_UNSUPPORTED;
+  g->H = H;
+  g->B = B;
+  g->P = P;
+  g->d = d;
+  g->bq = bq;
+  g->bk = bk;
+  g->nkb = static_cast<int>(nkb);
+  g->n_sel = n_sel < g->nkb ? n_sel : g->nkb;
+  // a split past ceil(nkb / kLosaMinChunk) could never hold a block
+  const int s_max = static_cast<int>(cdiv(nkb, kLosaMinChunk));
+  g->S = splits < s_max ? splits : s_max;
+  g->tiles = static_cast<int>(cdiv(B, bq));
+  g->R = g->tiles * bq;
+  long stride = cdiv(nkb, g->S);
+  if (stride < kLosaMinChunk) stride = kLosaMinChunk;
+  if (stride > nkb) stride = nkb;
+  g->stride = static_cast<int>(stride);
+  if (static_cast<long long>(H) * g->S * g->R * d >= (1ll << 31)) return SPARSED_ERR_UNSUPPORTED;
+  if (static_cast<long long>(H) * g->S * g->tiles * g->stride >= (1ll << 31)) return SPARSED_ERR_UNSUPPORTED;
+  if (static_cast<long long>(H) * B * nkb >= (1ll << 31)) return SPARSED_ERR_UNSUPPORTED;
+  return SPARSED_OK;
+}
+
+struct LosaWorkspace {
+  size_t active, pos, ucount, uidx, kvc, kvi, qrep, orep, lserep, mass, selcnt, total;
+};
+
+LosaWorkspace losa_ws_layout(const LosaDims& g) {
+  LosaWorkspace w;
+  const size_t items = static_cast<size_t>(g.H) * g.S * g.tiles;
+  const size_t rep_rows = static_cast<size_t>(g.H) * g.S * g.R;
+  w.active = 0;
+  w.pos = w.active + align256(static_cast<size_t>(g.B) * 4);
+  w.ucount = w.pos + align256(static_cast<size_t>(g.B) * 4);
+  w.uidx = w.ucount + align256(static_cast<size_t>(g.H) * 4);
+  w.kvc = w.uidx + align256(static_cast<size_t>(g.H) * g.nkb * 4);
+  w.kvi = w.kvc + align256(items * 4);
+  w.qrep = w.kvi + align256(items * g.stride * 4);
+  w.orep = w.qrep + align256(rep_rows * g.d * 2);
+  w.lserep = w.orep + align256(rep_rows * g.d * 2);
+  w.mass = w.lserep + align256(rep_rows * 4);
+  w.selcnt = w.mass + align256(static_cast<size_t>(g.H) * g.B * g.nkb * 4);
+  w.total = w.selcnt + align256(static_cast<size_t>(g.H) * g.B * 4);
+  return w;
+}
+
+int losa_check_ws(const LosaDims& g, const void* workspace, size_t ws_bytes) {
+  if (!workspace || ws_bytes < losa_ws_layout(g).total) return SPARSED_ERR_WORKSPACE;
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return SPARSED_ERR_WORKSPACE;
+  return SPARSED_OK;
+}
+
+// The block's own tensors, the prefix cache and the carried state.
+int losa_check_ptrs(const void* Q, const void* K, const void* V, const void* Kp, const void* Vp,
+                    const void* o_cache, const float* lse_cache, const int32_t* sel, const void* O,
+                    const float* LSE) {
+  if (!Q || !K || !V || !Kp || !Vp || !o_cache || !lse_cache || !sel || !O || !LSE) return SPARSED_ERR_INVALID_ARG;
+  if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(Kp) || !aligned16(Vp) || !aligned16(o_cache) ||
+      !aligned16(O))
+    return SPARSED_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(lse_cache) & 3u) || (reinterpret_cast<uintptr_t>(LSE) & 3u) ||
+      (reinterpret_cast<uintptr_t>(sel) & 3u))
+    return SPARSED_ERR_INVALID_ARG;
+  return SPARSED_OK;
+}
+
+// Suffix part: dense attention of the block over its own keys, into O / LSE.
+int losa_suffix(const LosaDims& g, const uint16_t* Q, const uint16_t* K, const uint16_t* V, float scale, uint16_t* O,
+                float* LSE, cudaStream_t st) {
+  Problem p;
+  p.Q = Q;
+  p.K = K;
+  p.V = V;
+  p.O = O;
+  p.LSE = LSE;
+  p.H = g.H;
+  p.L = g.B;
+  p.d = g.d;
+  p.bq = g.bq;
+  p.bk = g.bk;
+  p.nqb = g.tiles;
+  p.nkb = static_cast<int>(cdiv(g.B, g.bk));
+  p.Lk = g.B;
+  p.scale = scale;
+  return launch_attn(p, false, nullptr, nullptr, 0, st);
+}
+
+// The union, the split lists and the replicated queries; active == nullptr
+// for the first step of a block (every token, every prefix block).
+int losa_lists(const LosaDims& g, const int32_t* active, const int32_t* sel, int sel_stride, const uint16_t* Q,
+               int32_t* union_idx, int32_t* union_count, uint8_t* ws, cudaStream_t st) {
+  const LosaWorkspace w = losa_ws_layout(g);
+  LosaListArgs a;
+  a.H = g.H;
+  a.B = g.B;
+  a.d = g.d;
+  a.nkb = g.nkb;
+  a.n_sel = g.n_sel;
+  a.sel_stride = sel_stride;
+  a.bq = g.bq;
+  a.tiles = g.tiles;
+  a.R = g.R;
+  a.S = g.S;
+  a.kv_stride = g.stride;
+  a.active = active;
+  a.sel = sel;
+  a.q = Q;
+  a.pos = reinterpret_cast<int32_t*>(ws + w.pos);
+  a.union_idx = union_idx ? union_idx : reinterpret_cast<int32_t*>(ws + w.uidx);
+  a.union_count = union_count ? union_count : reinterpret_cast<int32_t*>(ws + w.ucount);
+  a.kv_idx = reinterpret_cast<int32_t*>(ws + w.kvi);
+  a.kv_count = reinterpret_cast<int32_t*>(ws + w.kvc);
+  a.q_rep = reinterpret_cast<uint16_t*>(ws + w.qrep);
+  losa_lists_kernel<<<g.H, 256, 0, st>>>(a);
+  SP_CUDA(cudaGetLastError());
+  return SPARSED_OK;
+}
+
+// Prefix pass over the split lists (block-sparse kernel, the replicated
+// queries against the prefix cache), then the merge into cache and output.
+int losa_prefix_and_merge(const LosaDims& g, const uint16_t* Kp, const uint16_t* Vp, float scale, bool all_active,
+                          uint16_t* o_cache, float* lse_cache, uint16_t* O, float* LSE, uint8_t* ws,
+                          cudaStream_t st) {
+  const LosaWorkspace w = losa_ws_layout(g);
+  Problem p;
+  p.Q = reinterpret_cast<const uint16_t*>(ws + w.qrep);
+  p.K = Kp;
+  p.V = Vp;
+  p.O = reinterpret_cast<uint16_t*>(ws + w.orep);
+  p.LSE = reinterpret_cast<float*>(ws + w.lserep);
+  p.H = g.H;
+  p.L = g.S * g.R;
+  p.d = g.d;
+  p.bq = g.bq;
+  p.bk = g.bk;
+  p.nqb = g.S * g.tiles;
+  p.nkb = g.nkb;
+  p.Lk = g.P;
+  p.scale = scale;
+  const int32_t* kvc = reinterpret_cast<const int32_t*>(ws + w.kvc);
+  SP_TRY(launch_attn(p, true, reinterpret_cast<const int32_t*>(ws + w.kvi), kvc, g.stride, st));
+  LosaMergeArgs m;
+  m.H = g.H;
+  m.B = g.B;
+  m.d = g.d;
+  m.S = g.S;
+  m.R = g.R;
+  m.tiles = g.tiles;
+  m.bq = g.bq;
+  m.pos = all_active ? nullptr : reinterpret_cast<const int32_t*>(ws + w.pos);
+  m.kv_count = kvc;
+  m.o_rep = p.O;
+  m.lse_rep = p.LSE;
+  m.o_cache = o_cache;
+  m.lse_cache = lse_cache;
+  m.o = O;
+  m.lse = LSE;
+  const unsigned grid = static_cast<unsigned>(cdiv(static_cast<long>(g.H) * g.B, 8));
+  if (g.d == 64)
+    losa_merge_kernel<64><<<grid, 256, 0, st>>>(m);
+  else
+    losa_merge_kernel<128><<<grid, 256, 0, st>>>(m);
+  SP_CUDA(cudaGetLastError());
+  return SPARSED_OK;
+}
+
+template <int D, int BK>
+int launch_tok_mass_t(const LosaDims& g, const uint16_t* Q, const uint16_t* Kp, float scale, const float* lse,
+                      float* mass, cudaStream_t st) {
+  using C = TokMassCfg<D>;
+  CUtensorMap tq, tk;
+  SP_TRY(make_map(&tq, Q, g.H, g.B, D, C::M));
+  SP_TRY(make_map(&tk, Kp, g.H, g.P, D, C::N));
+  TokMassArgs a;
+  a.H = g.H;
+  a.B = g.B;
+  a.P = g.P;
+  a.nkb = g.nkb;
+  a.tiles_per_cta = 8;
+  a.scale_log2 = scale * 1.44269504088896340736f;
+  a.lse = lse;
+  a.mass = mass;
+  a.timeout_ns = kWaitTimeoutNs;
+  auto kern = token_block_mass_kernel<D, BK>;
+  SP_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES));
+  const long ntiles = cdiv(g.P, C::N);
+  const dim3 grid(static_cast<unsigned>(cdiv(ntiles, a.tiles_per_cta)), static_cast<unsigned>(g.H),
+                  static_cast<unsigned>(cdiv(g.B, C::M)));
+  kern<<<grid, 256, C::SMEM_BYTES, st>>>(tq, tk, a);
+  SP_CUDA(cudaGetLastError());
+  return SPARSED_OK;
+}
+
+int launch_tok_mass(const LosaDims& g, const uint16_t* Q, const uint16_t* Kp, float scale, const float* lse,
+                    float* mass, cudaStream_t st) {
+  if (g.d == 64 && g.bk == 64) return launch_tok_mass_t<64, 64>(g, Q, Kp, scale, lse, mass, st);
+  if (g.d == 64 && g.bk == 128) return launch_tok_mass_t<64, 128>(g, Q, Kp, scale, lse, mass, st);
+  if (g.d == 128 && g.bk == 64) return launch_tok_mass_t<128, 64>(g, Q, Kp, scale, lse, mass, st);
+  if (g.d == 128 && g.bk == 128) return launch_tok_mass_t<128, 128>(g, Q, Kp, scale, lse, mass, st);
+  return SPARSED_ERR_UNSUPPORTED;
+}
+
+int losa_init_impl(const LosaDims& g, const uint16_t* Q, const uint16_t* K, const uint16_t* V, const uint16_t* Kp,
+                   const uint16_t* Vp, float scale, int sel_stride, uint16_t* o_cache, float* lse_cache,
+                   int32_t* sel, uint16_t* O, float* LSE, float* token_mass, uint8_t* ws, cudaStream_t st) {
+  const LosaWorkspace w = losa_ws_layout(g);
+  SP_TRY(losa_suffix(g, Q, K, V, scale, O, LSE, st));
+  SP_TRY(losa_lists(g, nullptr, nullptr, sel_stride, Q, nullptr, nullptr, ws, st));
+  SP_TRY(losa_prefix_and_merge(g, Kp, Vp, scale, true, o_cache, lse_cache, O, LSE, ws, st));
+  float* mass = token_mass ? token_mass : reinterpret_cast<float*>(ws + w.mass);
+  SP_TRY(launch_tok_mass(g, Q, Kp, scale, lse_cache, mass, st));
+  const int rows = g.H * g.B;
+  topk_kernel<<<(rows + 7) / 8, 256, 0, st>>>(mass, rows, g.B, g.nkb, g.n_sel, nullptr, nullptr, sel,
+                                             reinterpret_cast<int32_t*>(ws + w.selcnt), sel_stride);
+  SP_CUDA(cudaGetLastError());
+  return SPARSED_OK;
+}
+
+int losa_step_impl(const LosaDims& g, const uint16_t* Q, const uint16_t* K, const uint16_t* V,
+                   const uint16_t* Q_prev, const uint16_t* Kp, const uint16_t* Vp, float scale, float tau,
+                   int sel_stride, uint16_t* o_cache, float* lse_cache, const int32_t* sel, uint16_t* O,
+                   float* LSE, int32_t* active, int32_t* union_idx, int32_t* union_count, uint8_t* ws,
+                   cudaStream_t st) {
+  const LosaWorkspace w = losa_ws_layout(g);
+  int32_t* act = active ? active : reinterpret_cast<int32_t*>(ws + w.active);
+  query_mse_kernel<<<g.B, 256, 0, st>>>(Q, Q_prev, g.H, g.B, g.d, static_cast<double>(tau), act);
+  SP_CUDA(cudaGetLastError());
+  SP_TRY(losa_lists(g, act, sel, sel_stride, Q, union_idx, union_count, ws, st));
+  SP_TRY(losa_suffix(g, Q, K, V, scale, O, LSE, st));
+  return losa_prefix_and_merge(g, Kp, Vp, scale, false, o_cache, lse_cache, O, LSE, ws, st);
+}
+
+int losa_prepare(int H, int B, int P, int d, int bq, int bk, int n_sel, int splits, float scale, LosaDims* g) {
+  SP_TRY(losa_dims(H, B, P, d, bq, bk, n_sel, splits, g));
+  if (!std::isfinite(scale)) return SPARSED_ERR_INVALID_ARG;
+  return SPARSED_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int sparsed_losa_splits(int H, int B, int bq, int P, int bk, int sm_count, int* splits) {
+  if (!splits || H < 1 || B < 1 || P < 1 || sm_count < 1) return SPARSED_ERR_INVALID_ARG;
+  if ((bq != 64 && bq != 128) || (bk != 64 && bk != 128)) return SPARSED_ERR_UNSUPPORTED;
+  const long per_split = static_cast<long>(H) * cdiv(B, bq);  // work items of one split
+  long s = sm_count / per_split;
+  if (s < 1) s = 1;
+  const long s_max = cdiv(cdiv(P, bk), kLosaMinChunk);
+  if (s > s_max) s = s_max;
+  *splits = static_cast<int>(s);
+  return SPARSED_OK;
+}
+
+int sparsed_losa_workspace_bytes(int H, int B, int P, int d, int bq, int bk, int splits, size_t* bytes) {
+  if (!bytes) return SPARSED_ERR_INVALID_ARG;
+  LosaDims g;
+  SP_TRY(losa_dims(H, B, P, d, bq, bk, 1, splits, &g));
+  *bytes = losa_ws_layout(g).total;
+  return SPARSED_OK;
+}
+
+int sparsed_losa_init(const uint16_t* Q, const uint16_t* K, const uint16_t* V, const uint16_t* K_prefix,
+                      const uint16_t* V_prefix, int H, int B, int P, int d, float scale, int bq, int bk,
+                      int n_sel, int splits, uint16_t* o_cache, float* lse_cache, int32_t* sel, uint16_t* O,
+                      float* LSE, float* token_mass, void* workspace, size_t workspace_bytes, void* stream) {
+  LosaDims g;
+  SP_TRY(losa_prepare(H, B, P, d, bq, bk, n_sel, splits, scale, &g));
+  SP_TRY(losa_check_ptrs(Q, K, V, K_prefix, V_prefix, o_cache, lse_cache, sel, O, LSE));
+  if (token_mass && (reinterpret_cast<uintptr_t>(token_mass) & 3u)) return SPARSED_ERR_INVALID_ARG;
+  SP_TRY(losa_check_ws(g, workspace, workspace_bytes));
+  SP_TRY(require_sm100());
+  SP_TRY(get_encoder());
+  return losa_init_impl(g, Q, K, V, K_prefix, V_prefix, scale, n_sel, o_cache, lse_cache, sel, O, LSE, token_mass,
+                        static_cast<uint8_t*>(workspace), static_cast<cudaStream_t>(stream));
+}
+
+int sparsed_losa_step(const uint16_t* Q, const uint16_t* K, const uint16_t* V, const uint16_t* Q_prev,
+                      const uint16_t* K_prefix, const uint16_t* V_prefix, int H, int B, int P, int d, float scale,
+                      int bq, int bk, int n_sel, float tau, int splits, uint16_t* o_cache, float* lse_cache,
+                      const int32_t* sel, uint16_t* O, float* LSE, int32_t* active, int32_t* union_idx,
+                      int32_t* union_count, void* workspace, size_t workspace_bytes, void* stream) {
+  LosaDims g;
+  SP_TRY(losa_prepare(H, B, P, d, bq, bk, n_sel, splits, scale, &g));
+  SP_TRY(losa_check_ptrs(Q, K, V, K_prefix, V_prefix, o_cache, lse_cache, sel, O, LSE));
+  if (!Q_prev || !aligned16(Q_prev)) return SPARSED_ERR_INVALID_ARG;
+  if (!std::isfinite(tau) || tau < 0.f) return SPARSED_ERR_INVALID_ARG;
+  SP_TRY(losa_check_ws(g, workspace, workspace_bytes));
+  SP_TRY(require_sm100());
+  SP_TRY(get_encoder());
+  return losa_step_impl(g, Q, K, V, Q_prev, K_prefix, V_prefix, scale, tau, n_sel, o_cache, lse_cache, sel, O, LSE,
+                        active, union_idx, union_count, static_cast<uint8_t*>(workspace),
+                        static_cast<cudaStream_t>(stream));
+}
+
+int sparsed_losa_block(const uint16_t* Qs, const uint16_t* Ks, const uint16_t* Vs, const uint16_t* K_prefix,
+                       const uint16_t* V_prefix, int T, int H, int B, int P, int d, float scale, int bq, int bk,
+                       int n_sel, float tau, int splits, uint16_t* o_cache, float* lse_cache, int32_t* sel,
+                       uint16_t* Os, float* LSEs, int32_t* actives, int32_t* union_counts, void* workspace,
+                       size_t workspace_bytes, void* stream) {
+  if (T < 1) return SPARSED_ERR_INVALID_ARG;
+  LosaDims g;
+  SP_TRY(losa_prepare(H, B, P, d, bq, bk, n_sel, splits, scale, &g));
+  SP_TRY(losa_check_ptrs(Qs, Ks, Vs, K_prefix, V_prefix, o_cache, lse_cache, sel, Os, LSEs));
+  if (!std::isfinite(tau) || tau < 0.f) return SPARSED_ERR_INVALID_ARG;
+  if ((actives && (reinterpret_cast<uintptr_t>(actives) & 3u)) ||
+      (union_counts && (reinterpret_cast<uintptr_t>(union_counts) & 3u)))
+    return SPARSED_ERR_INVALID_ARG;
+  SP_TRY(losa_check_ws(g, workspace, workspace_bytes));
+  SP_TRY(require_sm100());
+  SP_TRY(get_encoder());
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  const size_t blk = static_cast<size_t>(H) * B * d;  // elements of one step's Q, K, V or O
+  const size_t rows = static_cast<size_t>(H) * B;
+  SP_TRY(losa_init_impl(g, Qs, Ks, Vs, K_prefix, V_prefix, scale, n_sel, o_cache, lse_cache, sel, Os, LSEs, nullptr,
+                        ws, st));
+  // step 0: every token active, every prefix block read
+  if (actives) {
+    fill_i32_kernel<<<static_cast<unsigned>(cdiv(B, 256)), 256, 0, st>>>(actives, B, 1);
+    SP_CUDA(cudaGetLastError());
+  }
+  if (union_counts) {
+    fill_i32_kernel<<<static_cast<unsigned>(cdiv(H, 256)), 256, 0, st>>>(union_counts, H, g.nkb);
+    SP_CUDA(cudaGetLastError());
+  }
+  for (int t = 1; t < T; ++t) {
+    SP_TRY(losa_step_impl(g, Qs + t * blk, Ks + t * blk, Vs + t * blk, Qs + (t - 1) * blk, K_prefix, V_prefix, scale,
+                          tau, n_sel, o_cache, lse_cache, sel, Os + t * blk, LSEs + t * rows,
+                          actives ? actives + static_cast<size_t>(t) * B : nullptr, nullptr,
+                          union_counts ? union_counts + static_cast<size_t>(t) * H : nullptr, ws, st));
+  }
+  return SPARSED_OK;
+}
+
+}  // extern "C"

@@ -323,6 +323,107 @@ int sparsed_select_pattern_noalloc(const uint16_t* Q, const uint16_t* K, const u
                                    int32_t* kv_idx, int32_t* kv_count, int kv_stride,
                                    float* block_mass, int32_t* head_k, void* stream);
 
+/* ---- Block-wise generation with active-token reuse
+ *
+ * LoSA: Locality Aware Sparse Attention for Block-Wise Diffusion Language
+ * Models (section 1: a block's queries load the union of the prefix positions
+ * they select; section 2: between consecutive steps only a few tokens' queries
+ * change much; section 3: active tokens -- large query change, measured by
+ * MSE -- get sparse prefix attention over the union of their selections,
+ * stable tokens reuse their cached prefix output, and prefix and in-block
+ * ("suffix") parts are merged by online softmax; the first step of a block is
+ * dense and fills the cache).
+ *
+ * Setting. A block of B tokens is denoised over T steps on top of a prefix of
+ * P cached tokens.
+ *   Q, K, V          [H, B, d] bf16: the block's queries, keys, values at this step
+ *   K_prefix, V_prefix  [H, P, d] bf16: the prefix cache (fixed during the block)
+ *   Prefix key block j covers prefix positions [j*bk, min((j+1)*bk, P));
+ *   nkb = ceil(P / bk).
+ * State carried across the block's steps (caller memory, written by
+ * sparsed_losa_init, read and updated by sparsed_losa_step):
+ *   o_cache   [H, B, d] bf16: every token's prefix attention output
+ *   lse_cache [H, B] fp32: its natural-log LSE over the prefix keys it attended
+ *   sel       [H, B, n_sel] int32: each token's n_sel prefix blocks (ascending)
+ * Every step's output O [H, B, d] bf16 and LSE [H, B] fp32 is attention over
+ * the token's prefix part (from the cache) together with all B block keys.
+ *
+ * Selector. The pages name the selector only (QUEST, a separate method); the
+ * method works with any. This library uses the SparseD selector at token
+ * granularity: in the block's first (dense) step each token's prefix blocks
+ * are scored by their post-softmax probability mass
+ *   M[h,b,j] = sum over c in block j of exp(scale*<q_b,k_c> - lse_cache[h,b])
+ * and the n_sel largest (ties to the lower block) are kept for the block.
+ * An active token attends to every key of its head's union.
+ *
+ * Work is split: a head's union is cut into `splits` chunks processed as
+ * separate work items of the block-sparse kernel and merged by LSE, so that a
+ * step keeps the SMs busy although a block holds few query rows.
+ *
+ * Sizes: 1 <= B <= 1024; P >= 1; nkb <= 32768; d in {64, 128}; bq, bk in
+ * {64, 128}; n_sel >= 1 (values above nkb act as nkb); splits >= 1 (values
+ * above ceil(nkb/4) act as ceil(nkb/4)); H*P*d < 2^31.
+ * Pointers: device memory, Q/K/V/prefix/o_cache/O 16-byte aligned, the rest
+ * 4-byte aligned; the workspace 256-byte aligned. Returns as every entry
+ * point; the union-building kernel reports a selection entry outside [0, nkb)
+ * as SPARSED_ERR_BAD_PATTERN (skipping it). */
+
+/* Splits for a step of these sizes on a GPU with sm_count SMs: as many as
+ * keep one split's H*ceil(B/bq) work items per SM at most
+ * (floor(sm_count / (H*ceil(B/bq))), at least 1, at most ceil(nkb/4)). */
+int sparsed_losa_splits(int H, int B, int bq, int P, int bk, int sm_count, int* splits);
+
+/* Workspace bytes of sparsed_losa_init / _step / _block for these sizes:
+ * the active flags and union (B + H*nkb + H int32), the split lists, the
+ * replicated queries and partial outputs ([H, splits*ceil(B/bq)*bq, d] bf16
+ * each, plus their LSE), the per-token block mass [H, B, nkb] fp32 and its
+ * counts, every part 256-byte aligned. */
+int sparsed_losa_workspace_bytes(int H, int B, int P, int d, int bq, int bk, int splits,
+                                 size_t* bytes);
+
+/* First step of a block: dense prefix attention of every token (the cache),
+ * each token's n_sel blocks (sel, row stride n_sel), the suffix attention and
+ * the merged output O, LSE. token_mass (nullable, [H, B, nkb] fp32) receives
+ * the per-token block mass. */
+int sparsed_losa_init(const uint16_t* Q, const uint16_t* K, const uint16_t* V,
+                      const uint16_t* K_prefix, const uint16_t* V_prefix,
+                      int H, int B, int P, int d, float scale, int bq, int bk, int n_sel, int splits,
+                      uint16_t* o_cache, float* lse_cache, int32_t* sel,
+                      uint16_t* O, float* LSE, float* token_mass,
+                      void* workspace, size_t workspace_bytes, void* stream);
+
+/* A later step of the block, in the page's order:
+ *   1. mse_b = mean over heads and dimensions of (Q - Q_prev)^2 (fp64), and
+ *      active[b] = (mse_b > tau) as int32 0/1 (active: nullable [B]);
+ *   2. per head, the ascending union of the active tokens' sel blocks
+ *      (union_idx: nullable [H, nkb], first union_count[h] entries;
+ *      union_count: nullable [H]);
+ *   3. prefix attention of the active tokens over every key of the union:
+ *      their o_cache / lse_cache entries are replaced; stable tokens keep
+ *      theirs;
+ *   4. suffix attention over the block, merged with the prefix part into O, LSE.
+ * Q_prev is the block's queries at the previous step ([H, B, d] bf16); tau is
+ * finite and >= 0. */
+int sparsed_losa_step(const uint16_t* Q, const uint16_t* K, const uint16_t* V, const uint16_t* Q_prev,
+                      const uint16_t* K_prefix, const uint16_t* V_prefix,
+                      int H, int B, int P, int d, float scale, int bq, int bk, int n_sel, float tau,
+                      int splits, uint16_t* o_cache, float* lse_cache, const int32_t* sel,
+                      uint16_t* O, float* LSE, int32_t* active, int32_t* union_idx,
+                      int32_t* union_count, void* workspace, size_t workspace_bytes, void* stream);
+
+/* All T >= 1 steps of a block: sparsed_losa_init on step 0, then
+ * sparsed_losa_step with the previous step's queries. Qs, Ks, Vs, Os are
+ * [T, H, B, d], LSEs [T, H, B]. actives (nullable, [T, B]) and union_counts
+ * (nullable, [T, H]) record each step's active flags and union sizes; step 0
+ * records every token active and nkb blocks per head. o_cache, lse_cache and
+ * sel hold the state after the last step. */
+int sparsed_losa_block(const uint16_t* Qs, const uint16_t* Ks, const uint16_t* Vs,
+                       const uint16_t* K_prefix, const uint16_t* V_prefix, int T,
+                       int H, int B, int P, int d, float scale, int bq, int bk, int n_sel, float tau,
+                       int splits, uint16_t* o_cache, float* lse_cache, int32_t* sel,
+                       uint16_t* Os, float* LSEs, int32_t* actives, int32_t* union_counts,
+                       void* workspace, size_t workspace_bytes, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -604,7 +604,7 @@ def prefix_attention(q_rows, k_pre, v_pre, scale, blocks, bk):
     return softmax_attention(q_rows, np.asarray(k_pre)[keys], np.asarray(v_pre)[keys], scale)
 
 
-def losa_init(q, k, v, k_pre, v_pre, scale, bk, n_sel):
+def losa_init(q, k, v, k_pre, v_pre, scale, bk, n_sel, sel=None):
     """First denoising step of a block (LoSA page, section 3, workflow,
     initialisation: dense attention fills the cache).
 
@@ -612,8 +612,10 @@ def losa_init(q, k, v, k_pre, v_pre, scale, bk, n_sel):
     keys is the cached prefix output and LSE; its per-token block mass gives
     the token's ``n_sel`` blocks (``token_block_mass``); the suffix attention
     is dense over the block; the step's output merges the two.
-    q, k, v: [H, B, d]; k_pre, v_pre: [H, P, d]. Returns dict with o [H,B,d],
-    lse [H,B], mass [H,B,nkb] and state = {o_pre, lse_pre, sel [H,B,n_sel']}."""
+    q, k, v: [H, B, d]; k_pre, v_pre: [H, P, d]. ``sel`` (optional, [H, B,
+    n_sel']) replaces the selection, so that the later steps can be followed
+    from a selection made elsewhere. Returns dict with o [H,B,d], lse [H,B],
+    mass [H,B,nkb] and state = {o_pre, lse_pre, sel [H,B,n_sel']}."""
     H, B, d = np.asarray(q).shape
     o = np.empty((H, B, d))
     lse = np.empty((H, B))
@@ -625,7 +627,7 @@ def losa_init(q, k, v, k_pre, v_pre, scale, bk, n_sel):
     for h in range(H):
         o_pre[h], lse_pre[h] = dense_attention(q[h], k_pre[h], v_pre[h], scale)
         mass[h] = token_block_mass(q[h], k_pre[h], scale, lse_pre[h], bk)
-        sels.append(token_select(mass[h], n_sel))
+        sels.append(token_select(mass[h], n_sel) if sel is None else np.asarray(sel[h], dtype=np.int32))
         o_suf, lse_suf = dense_attention(q[h], k[h], v[h], scale)
         o[h], lse[h] = merge_partials(o_pre[h], lse_pre[h], o_suf, lse_suf)
     state = dict(o_pre=o_pre, lse_pre=lse_pre, sel=np.stack(sels))
@@ -667,18 +669,19 @@ def losa_step(q, k, v, q_prev, k_pre, v_pre, scale, bk, tau, state):
     return dict(o=o, lse=lse, mse=mse, active=act, union=unions)
 
 
-def losa_block(qs, ks, vs, k_pre, v_pre, scale, bk, n_sel, tau):
+def losa_block(qs, ks, vs, k_pre, v_pre, scale, bk, n_sel, tau, sel=None):
     """All T denoising steps of one block: ``losa_init`` at step 0, then
     ``losa_step`` with the previous step's queries. qs, ks, vs: [T, H, B, d].
     Returns dict with o [T,H,B,d], lse [T,H,B], active [T,B] (step 0: all),
-    union_count [T,H] (step 0: every prefix block), state."""
+    union_count [T,H] (step 0: every prefix block), state. ``sel`` as in
+    ``losa_init``."""
     T, H, B, d = np.asarray(qs).shape
     nkb = n_blocks(np.asarray(k_pre).shape[1], bk)
     o = np.empty((T, H, B, d))
     lse = np.empty((T, H, B))
     active = np.ones((T, B), dtype=bool)
     ucount = np.full((T, H), nkb, dtype=np.int64)
-    first = losa_init(qs[0], ks[0], vs[0], k_pre, v_pre, scale, bk, n_sel)
+    first = losa_init(qs[0], ks[0], vs[0], k_pre, v_pre, scale, bk, n_sel, sel)
     o[0], lse[0] = first["o"], first["lse"]
     state = first["state"]
     for t in range(1, T):

@@ -161,3 +161,73 @@ def test_python_binding_type_checks():
     q = torch.zeros((1, 64, 64), dtype=torch.bfloat16)
     with pytest.raises(ValueError):
         sp.dense_attn(q, q, q)
+
+
+def _losa_splits(H=32, B=64, bq=64, P_=32768, bk=64, sms=148):
+    s = ctypes.c_int(-1)
+    rc = lib.sparsed_losa_splits(H, B, bq, P_, bk, sms, ctypes.byref(s))
+    return rc, s.value
+
+
+def test_losa_splits():
+    assert _losa_splits() == (_lib.OK, 4)                      # 148 SMs / 32 work items per split
+    assert _losa_splits(B=128) == (_lib.OK, 2)                 # two query tiles per split
+    assert _losa_splits(H=200) == (_lib.OK, 1)                 # at least one split
+    assert _losa_splits(H=1, P_=100) == (_lib.OK, 1)           # at most ceil(nkb / 4): nkb = 2
+    assert _losa_splits(H=1, P_=64 * 40) == (_lib.OK, 10)      # nkb = 40 -> at most 10
+    assert _losa_splits(sms=0)[0] == _lib.ERR_INVALID_ARG
+    assert _losa_splits(bq=32)[0] == _lib.ERR_UNSUPPORTED
+
+
+def _losa_ws(H=32, B=64, P_=32768, d=128, bq=64, bk=64, splits=4):
+    n = ctypes.c_size_t(0)
+    rc = lib.sparsed_losa_workspace_bytes(H, B, P_, d, bq, bk, splits, ctypes.byref(n))
+    return rc, n.value
+
+
+def test_losa_workspace_bytes():
+    rc, n4 = _losa_ws()
+    assert rc == _lib.OK
+    # the per-token block mass [H, B, nkb] fp32 and the replicated queries and
+    # partial outputs [H, splits*64, d] bf16 are the large parts
+    assert n4 >= 32 * 64 * 512 * 4 + 2 * 32 * 4 * 64 * 128 * 2
+    assert _losa_ws(splits=8)[1] > n4
+    assert _losa_ws(splits=1000)[1] == _losa_ws(splits=128)[1]  # clamped to ceil(nkb / 4)
+    assert _losa_ws(B=1025)[0] == _lib.ERR_UNSUPPORTED
+    assert _losa_ws(d=96)[0] == _lib.ERR_UNSUPPORTED
+    assert _losa_ws(P_=0)[0] == _lib.ERR_INVALID_ARG
+    assert _losa_ws(splits=0)[0] == _lib.ERR_INVALID_ARG
+    assert _losa_ws(P_=64 * 32768 + 1, H=1, d=64)[0] == _lib.ERR_UNSUPPORTED  # nkb > 32768
+
+
+def _losa_step(tau=0.01, ws=P, ws_bytes=1 << 30, qprev=P, sel=P, n_sel=2, B=64):
+    return lib.sparsed_losa_step(P, P, P, qprev, P, P, 2, B, 4096, 128, 0.088, 64, 64, n_sel, tau, 2,
+                                 P, P, sel, P, P, None, None, None, ws, ws_bytes, None)
+
+
+def test_losa_step_validation():
+    assert _losa_step(tau=float("nan")) == _lib.ERR_INVALID_ARG
+    assert _losa_step(tau=-1.0) == _lib.ERR_INVALID_ARG
+    assert _losa_step(qprev=None) == _lib.ERR_INVALID_ARG
+    assert _losa_step(qprev=MIS) == _lib.ERR_INVALID_ARG
+    assert _losa_step(sel=None) == _lib.ERR_INVALID_ARG
+    assert _losa_step(n_sel=0) == _lib.ERR_INVALID_ARG
+    assert _losa_step(ws=None) == _lib.ERR_WORKSPACE
+    assert _losa_step(ws_bytes=4096) == _lib.ERR_WORKSPACE
+    assert _losa_step(B=2000) == _lib.ERR_UNSUPPORTED
+    if not GPU:
+        assert _losa_step() == _lib.ERR_NO_DEVICE
+
+
+def test_losa_block_validation():
+    f = lib.sparsed_losa_block
+    args = [P, P, P, P, P, 3, 2, 64, 4096, 128, 0.088, 64, 64, 2, 0.01, 2, P, P, P, P, P, None, None,
+            P, 1 << 30, None]
+    a = list(args)
+    a[5] = 0  # T
+    assert f(*a) == _lib.ERR_INVALID_ARG
+    a = list(args)
+    a[21] = ctypes.c_void_p(0x10002)  # actives not 4-byte aligned
+    assert f(*a) == _lib.ERR_INVALID_ARG
+    if not GPU:
+        assert f(*args) == _lib.ERR_NO_DEVICE
