@@ -488,9 +488,10 @@ def losa_init(q, k, v, k_pre, v_pre, n_sel=2, scale=None, bq=64, bk=64, splits=N
     H, B, d = _check_qkv(q, k, v)
     P = _check_prefix(k_pre, v_pre, H, d, q.device)
     scale = default_scale(d) if scale is None else scale
+    nkb = (P + bk - 1) // bk
+    n_sel = max(1, min(n_sel, nkb))  # a token cannot keep more blocks than the prefix has
     st = _block_state(q, P, n_sel, scale, bq, bk, splits, workspace)
     out, lse = _alloc_out(q, None, None)
-    nkb = (P + bk - 1) // bk
     mass = torch.empty((H, B, nkb), dtype=torch.float32, device=q.device) if return_mass else None
     rc = _lib.load().sparsed_losa_init(
         _ptr(q), _ptr(k), _ptr(v), _ptr(k_pre), _ptr(v_pre), H, B, P, d, scale, bq, bk, n_sel, st.splits,
@@ -536,6 +537,7 @@ def losa_block(qs, ks, vs, k_pre, v_pre, n_sel=2, tau=0.01, scale=None, bq=64, b
     T, H, B, d = qs.shape
     P = _check_prefix(k_pre, v_pre, H, d, qs.device)
     scale = default_scale(d) if scale is None else scale
+    n_sel = max(1, min(n_sel, (P + bk - 1) // bk))
     st = _block_state(qs[0], P, n_sel, scale, bq, bk, splits, workspace)
     if out is None:
         out = torch.empty_like(qs)

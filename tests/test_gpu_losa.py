@@ -206,7 +206,9 @@ def test_split_count_changes_rounding_only():
         sp.device_check()
     a, b = outs
     assert torch.equal(a.active, b.active) and torch.equal(a.union_count, b.union_count)
-    assert torch.equal(a.union_idx, b.union_idx)
+    for h in range(2):
+        n = int(a.union_count[h])
+        assert torch.equal(a.union_idx[h, :n], b.union_idx[h, :n])
     ref = O.losa_step(f64(qs[1]), f64(ks[1]), f64(vs[1]), f64(qs[0]), f64(k_pre), f64(v_pre), wl.scale, wl.bk,
                       wl.tau, ref_state)
     for splits, r in zip((1, 8), outs):
