@@ -39,6 +39,7 @@ namespace sparsed {
 constexpr int kLosaMaxB = 1024;        // block tokens (the active list lives in shared memory)
 constexpr int kLosaMaxWords = 1024;    // union bitmask words: at most 32768 prefix blocks
 constexpr int kLosaMinChunk = 4;       // fewest blocks a non-empty split holds
+constexpr int kLosaMaxSplits = 32;     // splits of a head's list (one per lane in the merge)
 
 __device__ __forceinline__ float bf16_to_f32(uint16_t u) { return __uint_as_float(static_cast<uint32_t>(u) << 16); }
 
@@ -51,21 +52,32 @@ __global__ void __launch_bounds__(256) fill_i32_kernel(int32_t* __restrict__ p, 
 // ---------------------------------------------------------------- locality score
 
 // One CTA of 256 threads per block token b: the squared query change summed
-// over every head and dimension in fp64 (a per-thread strided sum, then a
-// fixed shuffle tree and the 8 warps in order), divided by H*d.
+// over every head and dimension in fp64 (each thread takes 16-byte pieces of
+// the token's rows, 8 elements each, then a fixed shuffle tree and the 8
+// warps in order), divided by H*d. d is a multiple of 8.
 __global__ void __launch_bounds__(256)
     query_mse_kernel(const uint16_t* __restrict__ q, const uint16_t* __restrict__ q_prev, int H, int B, int d,
                      double tau, int32_t* __restrict__ active) {
   __shared__ double s_part[8];
   const int b = blockIdx.x;
-  const int n = H * d;
+  const int row_u4 = d / 8;
+  const int n_u4 = H * row_u4;
+  const uint4* q4 = reinterpret_cast<const uint4*>(q);
+  const uint4* p4 = reinterpret_cast<const uint4*>(q_prev);
   double acc = 0.0;
-  for (int e = threadIdx.x; e < n; e += blockDim.x) {
-    const int h = e / d;
-    const int c = e - h * d;
-    const long idx = (static_cast<long>(h) * B + b) * d + c;
-    const double x = static_cast<double>(bf16_to_f32(q[idx])) - static_cast<double>(bf16_to_f32(q_prev[idx]));
-    acc += x * x;
+#pragma unroll 4
+  for (int e = threadIdx.x; e < n_u4; e += blockDim.x) {
+    const int h = e / row_u4;
+    const long idx = (static_cast<long>(h) * B + b) * row_u4 + (e - h * row_u4);
+    const uint4 x = q4[idx], y = p4[idx];
+    const uint32_t xs[4] = {x.x, x.y, x.z, x.w}, ys[4] = {y.x, y.y, y.z, y.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const double d0 = static_cast<double>(__uint_as_float(xs[i] << 16)) - __uint_as_float(ys[i] << 16);
+      const double d1 = static_cast<double>(__uint_as_float(xs[i] & 0xffff0000u)) -
+                        __uint_as_float(ys[i] & 0xffff0000u);
+      acc += d0 * d0 + d1 * d1;
+    }
   }
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
@@ -74,7 +86,7 @@ __global__ void __launch_bounds__(256)
   if (threadIdx.x == 0) {
     double t = 0.0;
     for (int w = 0; w < 8; ++w) t += s_part[w];
-    active[b] = (t / static_cast<double>(n)) > tau ? 1 : 0;
+    active[b] = (t / static_cast<double>(H * d)) > tau ? 1 : 0;
   }
 }
 
@@ -110,11 +122,11 @@ struct LosaListArgs {
 //      max(kLosaMinChunk, ceil(u / S)); work item (s, t) of query tile t gets
 //      that chunk when the tile holds an active token, else nothing
 //   5. row s*R + a of q_rep is the a-th active token's query (zero past the
-//      active count) for every tile that has work
+//      active count) for every split and tile that have work
 __global__ void __launch_bounds__(256) losa_lists_kernel(const LosaListArgs a) {
   __shared__ int s_act[kLosaMaxB];
   __shared__ uint32_t s_bits[kLosaMaxWords];
-  __shared__ int s_scan[256];
+  __shared__ int s_scan[8];
   __shared__ int s_warp[8];
   __shared__ int s_u;
   const int h = blockIdx.x;
@@ -173,20 +185,28 @@ __global__ void __launch_bounds__(256) losa_lists_kernel(const LosaListArgs a) {
   const int w1 = w0 + wpt < words ? w0 + wpt : words;
   int cnt = 0;
   for (int w = w0; w < w1; ++w) cnt += __popc(s_bits[w]);
-  s_scan[tid] = cnt;
+  // exclusive scan of the 256 counts: within each warp by shuffles, then
+  // over the 8 warp totals
+  int incl = cnt;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, incl, off);
+    if (lane >= off) incl += y;
+  }
+  if (lane == 31) s_scan[wid] = incl;
   __syncthreads();
   if (tid == 0) {
     int run = 0;
-    for (int t = 0; t < 256; ++t) {
-      const int c = s_scan[t];
-      s_scan[t] = run;
+    for (int w = 0; w < 8; ++w) {
+      const int c = s_scan[w];
+      s_scan[w] = run;
       run += c;
     }
     s_u = run;
   }
   __syncthreads();
   int32_t* ulist = a.union_idx + static_cast<long>(h) * a.nkb;
-  int outp = s_scan[tid];
+  int outp = s_scan[wid] + incl - cnt;
   for (int w = w0; w < w1; ++w) {
     uint32_t m = s_bits[w];
     while (m) {
@@ -221,18 +241,18 @@ __global__ void __launch_bounds__(256) losa_lists_kernel(const LosaListArgs a) {
     if (t * a.bq < na && jj < split_len(s)) a.kv_idx[(item0 + it) * a.kv_stride + jj] = ulist[s * chunk + jj];
   }
 
-  // 5. replicated queries of the tiles that have work
+  // 5. replicated queries of the tiles that have work: each 16-byte piece of
+  // an active token's query is read once and stored into every split
   const int row_u4 = a.d / 8;
   const uint4* qsrc = reinterpret_cast<const uint4*>(a.q) + static_cast<long>(h) * a.B * row_u4;
   uint4* qdst = reinterpret_cast<uint4*>(a.q_rep) + static_cast<long>(h) * a.S * a.R * row_u4;
-  const long n_u4 = static_cast<long>(a.S) * a.R * row_u4;
-  for (long e = tid; e < n_u4; e += 256) {
-    const int row = static_cast<int>(e / row_u4);  // s * R + r
-    const int c = static_cast<int>(e - static_cast<long>(row) * row_u4);
-    const int s = row / a.R;
-    const int r = row - s * a.R;
-    if ((r / a.bq) * a.bq >= na || split_len(s) == 0) continue;
-    qdst[e] = r < na ? qsrc[static_cast<long>(s_act[r]) * row_u4 + c] : make_uint4(0u, 0u, 0u, 0u);
+  const int rows = ((na + a.bq - 1) / a.bq) * a.bq;  // rows of the tiles with work (<= R)
+  for (int e = tid; e < rows * row_u4; e += 256) {
+    const int r = e / row_u4;
+    const int c = e - r * row_u4;
+    const uint4 val = r < na ? qsrc[static_cast<long>(s_act[r]) * row_u4 + c] : make_uint4(0u, 0u, 0u, 0u);
+    for (int s = 0; s < a.S; ++s)
+      if (split_len(s) > 0) qdst[(static_cast<long>(s) * a.R + r) * row_u4 + c] = val;
   }
 }
 
@@ -251,9 +271,10 @@ struct LosaMergeArgs {
 };
 
 // One warp per (h, b). An active token's prefix part is the LSE-weighted sum
-// of its splits' partial outputs (empty splits skipped), written back to the
-// cache in bf16; a stable token's is the cache entry. The output merges that
-// prefix part with the suffix part the same way (fp32 arithmetic).
+// of its splits' partial outputs (lane s holds split s's LSE and weight; an
+// empty split weighs 0), written back to the cache in bf16; a stable token's
+// is the cache entry. The output merges that prefix part with the suffix part
+// the same way (fp32 arithmetic, fixed reduction order). At most 32 splits.
 template <int D>
 __global__ void __launch_bounds__(256) losa_merge_kernel(const LosaMergeArgs a) {
   constexpr int PER = D / 32;  // contiguous elements per lane
@@ -264,30 +285,38 @@ __global__ void __launch_bounds__(256) losa_merge_kernel(const LosaMergeArgs a) 
   const int b = static_cast<int>(row - static_cast<long>(h) * a.B);
   const int c0 = lane * PER;
   const float kNegInf = -__int_as_float(0x7f800000);
-  float op[PER];
-#pragma unroll
-  for (int e = 0; e < PER; ++e) op[e] = 0.f;
-  float lp;
-  const int ap = a.pos ? a.pos[b] : b;
   const long crow = (static_cast<long>(h) * a.B + b) * a.d;
+  const long lrow = static_cast<long>(h) * a.B + b;
+  const int ap = a.pos ? a.pos[b] : b;
+  // the suffix part, read before any branch
+  float osuf[PER];
+#pragma unroll
+  for (int e = 0; e < PER; ++e) osuf[e] = bf16_to_f32(a.o[crow + c0 + e]);
+  const float ls = a.lse[lrow];
+  float op[PER];
+  float lp;
   if (ap >= 0) {
     const int t = ap / a.bq;
-    const int* cnt = a.kv_count + static_cast<long>(h) * a.S * a.tiles + t;
     const long rep0 = static_cast<long>(h) * a.S * a.R + ap;
-    float m = kNegInf;
-    for (int s = 0; s < a.S; ++s)
-      if (cnt[s * a.tiles] > 0) m = fmaxf(m, a.lse_rep[rep0 + static_cast<long>(s) * a.R]);
-    float z = 0.f;
-    if (m != kNegInf) {
-      for (int s = 0; s < a.S; ++s) {
-        if (cnt[s * a.tiles] <= 0) continue;
-        const long r = rep0 + static_cast<long>(s) * a.R;
-        const float w = expf(a.lse_rep[r] - m);
-        z += w;
-        const uint16_t* src = a.o_rep + r * a.d + c0;
+    float l_s = kNegInf;
+    if (lane < a.S && a.kv_count[static_cast<long>(h) * a.S * a.tiles + lane * a.tiles + t] > 0)
+      l_s = a.lse_rep[rep0 + static_cast<long>(lane) * a.R];
+    float m = l_s;
 #pragma unroll
-        for (int e = 0; e < PER; ++e) op[e] += w * bf16_to_f32(src[e]);
-      }
+    for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+    const float w = (m == kNegInf || l_s == kNegInf) ? 0.f : expf(l_s - m);
+    float z = w;
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) z += __shfl_xor_sync(0xffffffffu, z, off);
+#pragma unroll
+    for (int e = 0; e < PER; ++e) op[e] = 0.f;
+    // every split's rows are written by the prefix pass (zeros for an empty one)
+#pragma unroll 4
+    for (int s = 0; s < a.S; ++s) {
+      const float ws = __shfl_sync(0xffffffffu, w, s);
+      const uint16_t* src = a.o_rep + (rep0 + static_cast<long>(s) * a.R) * a.d + c0;
+#pragma unroll
+      for (int e = 0; e < PER; ++e) op[e] += ws * bf16_to_f32(src[e]);
     }
     if (z > 0.f) {
       const float inv = 1.f / z;
@@ -300,26 +329,74 @@ __global__ void __launch_bounds__(256) losa_merge_kernel(const LosaMergeArgs a) 
 #pragma unroll
     for (int e = 0; e < PER; e += 2)
       *reinterpret_cast<uint32_t*>(a.o_cache + crow + c0 + e) = ptx::pack_bf16x2(op[e], op[e + 1]);
-    if (lane == 0) a.lse_cache[static_cast<long>(h) * a.B + b] = lp;
+    if (lane == 0) a.lse_cache[lrow] = lp;
   } else {
 #pragma unroll
     for (int e = 0; e < PER; ++e) op[e] = bf16_to_f32(a.o_cache[crow + c0 + e]);
-    lp = a.lse_cache[static_cast<long>(h) * a.B + b];
+    lp = a.lse_cache[lrow];
   }
-  const float ls = a.lse[static_cast<long>(h) * a.B + b];
-  __syncwarp();  // every lane has read its suffix inputs before any lane overwrites them
   const float m2 = fmaxf(lp, ls);
   const float wp = lp == kNegInf ? 0.f : expf(lp - m2);
-  const float ws = ls == kNegInf ? 0.f : expf(ls - m2);
-  const float z2 = wp + ws;
+  const float ws2 = ls == kNegInf ? 0.f : expf(ls - m2);
+  const float z2 = wp + ws2;
   const float inv2 = z2 > 0.f ? 1.f / z2 : 0.f;
   float out[PER];
 #pragma unroll
-  for (int e = 0; e < PER; ++e) out[e] = (wp * op[e] + ws * bf16_to_f32(a.o[crow + c0 + e])) * inv2;
+  for (int e = 0; e < PER; ++e) out[e] = (wp * op[e] + ws2 * osuf[e]) * inv2;
+  __syncwarp();  // every lane has read its suffix inputs before any lane overwrites them
 #pragma unroll
   for (int e = 0; e < PER; e += 2)
     *reinterpret_cast<uint32_t*>(a.o + crow + c0 + e) = ptx::pack_bf16x2(out[e], out[e + 1]);
-  if (lane == 0) a.lse[static_cast<long>(h) * a.B + b] = z2 > 0.f ? m2 + logf(z2) : kNegInf;
+  if (lane == 0) a.lse[lrow] = z2 > 0.f ? m2 + logf(z2) : kNegInf;
+}
+
+// ---------------------------------------------------------------- per-token top-k
+
+// One warp per row of mass[rows, n]: the k <= 32 largest entries (ties to the
+// lower index), written in ascending index order to idx[row * stride ..]. In
+// the order "mass descending, index ascending", round r takes the best entry
+// after the pick of round r-1: each lane scans its strided share of the row,
+// a shuffle reduction gives the warp's best, and lane r keeps it. Each lane's
+// rank among the k picks by index is its output slot. The kept set is the one
+// of topk_kernel (rank(j) < k in the same order).
+__global__ void __launch_bounds__(256)
+    topk_small_kernel(const float* __restrict__ mass, int rows, int n, int k, int32_t* __restrict__ idx,
+                      int stride) {
+  const int lane = threadIdx.x & 31;
+  const long row = static_cast<long>(blockIdx.x) * 8 + (threadIdx.x >> 5);
+  if (row >= rows) return;
+  const float* m = mass + row * n;
+  const float kInf = __int_as_float(0x7f800000);
+  float pv = kInf;  // the previous pick; every finite entry comes after (+inf, -1)
+  int pj = -1;
+  int mine = 0;     // lane r: the pick of round r
+  for (int r = 0; r < k; ++r) {
+    float bv = -kInf;
+    int bj = 0x7fffffff;
+    for (int j = lane; j < n; j += 32) {
+      const float v = m[j];
+      const bool after = v < pv || (v == pv && j > pj);
+      if (after && (v > bv || (v == bv && j < bj))) {
+        bv = v;
+        bj = j;
+      }
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+      const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
+      const int oj = __shfl_xor_sync(0xffffffffu, bj, off);
+      if (ov > bv || (ov == bv && oj < bj)) {
+        bv = ov;
+        bj = oj;
+      }
+    }
+    pv = bv;
+    pj = bj;
+    if (lane == r) mine = bj;
+  }
+  int rank = 0;
+  for (int s = 0; s < k; ++s) rank += __shfl_sync(0xffffffffu, mine, s) < mine;
+  if (lane < k) idx[row * stride + rank] = mine;
 }
 
 // ---------------------------------------------------------------- per-token block mass

@@ -960,8 +960,10 @@ int losa_dims(int H, int B, int P, int d, int bq, int bk, int n_sel, int splits,
   g->bk = bk;
   g->nkb = static_cast<int>(nkb);
   g->n_sel = n_sel < g->nkb ? n_sel : g->nkb;
-  // a split past ceil(nkb / kLosaMinChunk) could never hold a block
-  const int s_max = static_cast<int>(cdiv(nkb, kLosaMinChunk));
+  // a split past ceil(nkb / kLosaMinChunk) could never hold a block; the merge
+  // holds one split per lane
+  int s_max = static_cast<int>(cdiv(nkb, kLosaMinChunk));
+  if (s_max > kLosaMaxSplits) s_max = kLosaMaxSplits;
   g->S = splits < s_max ? splits : s_max;
   g->tiles = static_cast<int>(cdiv(B, bq));
   g->R = g->tiles * bq;
@@ -1164,8 +1166,11 @@ int losa_init_impl(const LosaDims& g, const uint16_t* Q, const uint16_t* K, cons
   float* mass = token_mass ? token_mass : reinterpret_cast<float*>(ws + w.mass);
   SP_TRY(launch_tok_mass(g, Q, Kp, scale, lse_cache, mass, st));
   const int rows = g.H * g.B;
-  topk_kernel<<<(rows + 7) / 8, 256, 0, st>>>(mass, rows, g.B, g.nkb, g.n_sel, nullptr, nullptr, sel,
-                                             reinterpret_cast<int32_t*>(ws + w.selcnt), sel_stride);
+  if (g.n_sel <= 32)
+    topk_small_kernel<<<(rows + 7) / 8, 256, 0, st>>>(mass, rows, g.nkb, g.n_sel, sel, sel_stride);
+  else
+    topk_kernel<<<(rows + 7) / 8, 256, 0, st>>>(mass, rows, g.B, g.nkb, g.n_sel, nullptr, nullptr, sel,
+                                               reinterpret_cast<int32_t*>(ws + w.selcnt), sel_stride);
   SP_CUDA(cudaGetLastError());
   return SPARSED_OK;
 }
@@ -1200,7 +1205,8 @@ int sparsed_losa_splits(int H, int B, int bq, int P, int bk, int sm_count, int* 
   const long per_split = static_cast<long>(H) * cdiv(B, bq);  // work items of one split
   long s = sm_count / per_split;
   if (s < 1) s = 1;
-  const long s_max = cdiv(cdiv(P, bk), kLosaMinChunk);
+  long s_max = cdiv(cdiv(P, bk), kLosaMinChunk);
+  if (s_max > kLosaMaxSplits) s_max = kLosaMaxSplits;
   if (s > s_max) s = s_max;
   *splits = static_cast<int>(s);
   return SPARSED_OK;

@@ -362,7 +362,7 @@ int sparsed_select_pattern_noalloc(const uint16_t* Q, const uint16_t* K, const u
  *
  * Sizes: 1 <= B <= 1024; P >= 1; nkb <= 32768; d in {64, 128}; bq, bk in
  * {64, 128}; n_sel >= 1 (values above nkb act as nkb); splits >= 1 (values
- * above ceil(nkb/4) act as ceil(nkb/4)); H*P*d < 2^31.
+ * above min(32, ceil(nkb/4)) act as that bound); H*P*d < 2^31.
  * Pointers: device memory, Q/K/V/prefix/o_cache/O 16-byte aligned, the rest
  * 4-byte aligned; the workspace 256-byte aligned. Returns as every entry
  * point; the union-building kernel reports a selection entry outside [0, nkb)
@@ -370,7 +370,7 @@ int sparsed_select_pattern_noalloc(const uint16_t* Q, const uint16_t* K, const u
 
 /* Splits for a step of these sizes on a GPU with sm_count SMs: as many as
  * keep one split's H*ceil(B/bq) work items per SM at most
- * (floor(sm_count / (H*ceil(B/bq))), at least 1, at most ceil(nkb/4)). */
+ * (floor(sm_count / (H*ceil(B/bq))), at least 1, at most min(32, ceil(nkb/4))). */
 int sparsed_losa_splits(int H, int B, int bq, int P, int bk, int sm_count, int* splits);
 
 /* Workspace bytes of sparsed_losa_init / _step / _block for these sizes:

@@ -175,6 +175,7 @@ def test_losa_splits():
     assert _losa_splits(H=200) == (_lib.OK, 1)                 # at least one split
     assert _losa_splits(H=1, P_=100) == (_lib.OK, 1)           # at most ceil(nkb / 4): nkb = 2
     assert _losa_splits(H=1, P_=64 * 40) == (_lib.OK, 10)      # nkb = 40 -> at most 10
+    assert _losa_splits(H=1, P_=64 * 1000) == (_lib.OK, 32)    # never more than 32
     assert _losa_splits(sms=0)[0] == _lib.ERR_INVALID_ARG
     assert _losa_splits(bq=32)[0] == _lib.ERR_UNSUPPORTED
 
