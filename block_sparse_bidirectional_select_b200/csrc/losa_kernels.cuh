@@ -41,7 +41,22 @@ constexpr int kLosaMaxWords = 1024;    // union bitmask words: at most 32768 pre
 constexpr int kLosaMinChunk = 4;       // fewest blocks a non-empty split holds
 constexpr int kLosaMaxSplits = 32;     // splits of a head's list (one per lane in the merge)
 
-__device__ __forceinline__ float bf16_to_f32(uint16_t u) { return __uint_as_float(static_cast<uint32_t>(u) << 16); }
+// PER (2 or 4) consecutive bf16 from an address aligned to 2*PER bytes, widened to fp32.
+template <int PER>
+__device__ __forceinline__ void load_bf16(const uint16_t* p, float (&f)[PER]) {
+  static_assert(PER == 2 || PER == 4, "2 or 4 elements");
+  if constexpr (PER == 4) {
+    const uint2 u = *reinterpret_cast<const uint2*>(p);
+    f[0] = __uint_as_float(u.x << 16);
+    f[1] = __uint_as_float(u.x & 0xffff0000u);
+    f[2] = __uint_as_float(u.y << 16);
+    f[3] = __uint_as_float(u.y & 0xffff0000u);
+  } else {
+    const uint32_t u = *reinterpret_cast<const uint32_t*>(p);
+    f[0] = __uint_as_float(u << 16);
+    f[1] = __uint_as_float(u & 0xffff0000u);
+  }
+}
 
 // p[0..n) = value (the step-0 rows of the per-step records).
 __global__ void __launch_bounds__(256) fill_i32_kernel(int32_t* __restrict__ p, int n, int32_t value) {
@@ -290,8 +305,7 @@ __global__ void __launch_bounds__(256) losa_merge_kernel(const LosaMergeArgs a) 
   const int ap = a.pos ? a.pos[b] : b;
   // the suffix part, read before any branch
   float osuf[PER];
-#pragma unroll
-  for (int e = 0; e < PER; ++e) osuf[e] = bf16_to_f32(a.o[crow + c0 + e]);
+  load_bf16<PER>(a.o + crow + c0, osuf);
   const float ls = a.lse[lrow];
   float op[PER];
   float lp;
@@ -314,9 +328,10 @@ __global__ void __launch_bounds__(256) losa_merge_kernel(const LosaMergeArgs a) 
 #pragma unroll 4
     for (int s = 0; s < a.S; ++s) {
       const float ws = __shfl_sync(0xffffffffu, w, s);
-      const uint16_t* src = a.o_rep + (rep0 + static_cast<long>(s) * a.R) * a.d + c0;
+      float part[PER];
+      load_bf16<PER>(a.o_rep + (rep0 + static_cast<long>(s) * a.R) * a.d + c0, part);
 #pragma unroll
-      for (int e = 0; e < PER; ++e) op[e] += ws * bf16_to_f32(src[e]);
+      for (int e = 0; e < PER; ++e) op[e] += ws * part[e];
     }
     if (z > 0.f) {
       const float inv = 1.f / z;
@@ -331,8 +346,7 @@ __global__ void __launch_bounds__(256) losa_merge_kernel(const LosaMergeArgs a) 
       *reinterpret_cast<uint32_t*>(a.o_cache + crow + c0 + e) = ptx::pack_bf16x2(op[e], op[e + 1]);
     if (lane == 0) a.lse_cache[lrow] = lp;
   } else {
-#pragma unroll
-    for (int e = 0; e < PER; ++e) op[e] = bf16_to_f32(a.o_cache[crow + c0 + e]);
+    load_bf16<PER>(a.o_cache + crow + c0, op);
     lp = a.lse_cache[lrow];
   }
   const float m2 = fmaxf(lp, ls);

@@ -1000,6 +1000,36 @@ LosaWorkspace losa_ws_layout(const LosaDims& g) {
   return w;
 }
 
+// A second stream per device on which a step's suffix attention (the block
+// over its own keys) runs beside the union building and the prefix pass of
+// the caller's stream: forked from and joined back to the caller's stream by
+// events, so the caller sees one ordered stream (and a graph capture of it
+// takes both branches). Created at the first use on a device; the lock keeps
+// the fork / join of concurrent callers apart.
+struct SideStream {
+  cudaStream_t s = nullptr;
+  cudaEvent_t fork = nullptr, join = nullptr;
+  std::mutex mu;
+};
+constexpr int kSideMaxDevices = 64;
+SideStream g_side[kSideMaxDevices];
+std::mutex g_side_init_mu;
+
+int side_stream(SideStream** out) {
+  int dev = 0;
+  SP_CUDA(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= kSideMaxDevices) return SPARSED_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_side_init_mu);
+  SideStream& ss = g_side[dev];
+  if (ss.s == nullptr) {
+    SP_CUDA(cudaStreamCreateWithFlags(&ss.s, cudaStreamNonBlocking));
+    SP_CUDA(cudaEventCreateWithFlags(&ss.fork, cudaEventDisableTiming));
+    SP_CUDA(cudaEventCreateWithFlags(&ss.join, cudaEventDisableTiming));
+  }
+  *out = &ss;
+  return SPARSED_OK;
+}
+
 int losa_check_ws(const LosaDims& g, const void* workspace, size_t ws_bytes) {
   if (!workspace || ws_bytes < losa_ws_layout(g).total) return SPARSED_ERR_WORKSPACE;
   if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return SPARSED_ERR_WORKSPACE;
@@ -1076,7 +1106,7 @@ int losa_lists(const LosaDims& g, const int32_t* active, const int32_t* sel, int
 // queries against the prefix cache), then the merge into cache and output.
 int losa_prefix_and_merge(const LosaDims& g, const uint16_t* Kp, const uint16_t* Vp, float scale, bool all_active,
                           uint16_t* o_cache, float* lse_cache, uint16_t* O, float* LSE, uint8_t* ws,
-                          cudaStream_t st) {
+                          cudaStream_t st, cudaEvent_t suffix_done = nullptr) {
   const LosaWorkspace w = losa_ws_layout(g);
   Problem p;
   p.Q = reinterpret_cast<const uint16_t*>(ws + w.qrep);
@@ -1095,6 +1125,7 @@ int losa_prefix_and_merge(const LosaDims& g, const uint16_t* Kp, const uint16_t*
   p.scale = scale;
   const int32_t* kvc = reinterpret_cast<const int32_t*>(ws + w.kvc);
   SP_TRY(launch_attn(p, true, reinterpret_cast<const int32_t*>(ws + w.kvi), kvc, g.stride, st));
+  if (suffix_done) SP_CUDA(cudaStreamWaitEvent(st, suffix_done, 0));  // the merge reads the suffix part
   LosaMergeArgs m;
   m.H = g.H;
   m.B = g.B;
@@ -1160,9 +1191,17 @@ int losa_init_impl(const LosaDims& g, const uint16_t* Q, const uint16_t* K, cons
                    const uint16_t* Vp, float scale, int sel_stride, uint16_t* o_cache, float* lse_cache,
                    int32_t* sel, uint16_t* O, float* LSE, float* token_mass, uint8_t* ws, cudaStream_t st) {
   const LosaWorkspace w = losa_ws_layout(g);
-  SP_TRY(losa_suffix(g, Q, K, V, scale, O, LSE, st));
-  SP_TRY(losa_lists(g, nullptr, nullptr, sel_stride, Q, nullptr, nullptr, ws, st));
-  SP_TRY(losa_prefix_and_merge(g, Kp, Vp, scale, true, o_cache, lse_cache, O, LSE, ws, st));
+  SideStream* side = nullptr;
+  SP_TRY(side_stream(&side));
+  {
+    std::lock_guard<std::mutex> lock(side->mu);
+    SP_CUDA(cudaEventRecord(side->fork, st));
+    SP_CUDA(cudaStreamWaitEvent(side->s, side->fork, 0));
+    SP_TRY(losa_suffix(g, Q, K, V, scale, O, LSE, side->s));
+    SP_CUDA(cudaEventRecord(side->join, side->s));
+    SP_TRY(losa_lists(g, nullptr, nullptr, sel_stride, Q, nullptr, nullptr, ws, st));
+    SP_TRY(losa_prefix_and_merge(g, Kp, Vp, scale, true, o_cache, lse_cache, O, LSE, ws, st, side->join));
+  }
   float* mass = token_mass ? token_mass : reinterpret_cast<float*>(ws + w.mass);
   SP_TRY(launch_tok_mass(g, Q, Kp, scale, lse_cache, mass, st));
   const int rows = g.H * g.B;
@@ -1182,11 +1221,17 @@ int losa_step_impl(const LosaDims& g, const uint16_t* Q, const uint16_t* K, cons
                    cudaStream_t st) {
   const LosaWorkspace w = losa_ws_layout(g);
   int32_t* act = active ? active : reinterpret_cast<int32_t*>(ws + w.active);
+  SideStream* side = nullptr;
+  SP_TRY(side_stream(&side));
+  std::lock_guard<std::mutex> lock(side->mu);
+  SP_CUDA(cudaEventRecord(side->fork, st));
+  SP_CUDA(cudaStreamWaitEvent(side->s, side->fork, 0));
+  SP_TRY(losa_suffix(g, Q, K, V, scale, O, LSE, side->s));
+  SP_CUDA(cudaEventRecord(side->join, side->s));
   query_mse_kernel<<<g.B, 256, 0, st>>>(Q, Q_prev, g.H, g.B, g.d, static_cast<double>(tau), act);
   SP_CUDA(cudaGetLastError());
   SP_TRY(losa_lists(g, act, sel, sel_stride, Q, union_idx, union_count, ws, st));
-  SP_TRY(losa_suffix(g, Q, K, V, scale, O, LSE, st));
-  return losa_prefix_and_merge(g, Kp, Vp, scale, false, o_cache, lse_cache, O, LSE, ws, st);
+  return losa_prefix_and_merge(g, Kp, Vp, scale, false, o_cache, lse_cache, O, LSE, ws, st, side->join);
 }
 
 int losa_prepare(int H, int B, int P, int d, int bq, int bk, int n_sel, int splits, float scale, LosaDims* g) {
