@@ -507,7 +507,9 @@ def losa_step(q, k, v, q_prev, k_pre, v_pre, state: BlockState, tau: float, retu
     the union of their blocks, their prefix attention over it (cache update),
     the block's own attention, and the merge. Updates ``state`` in place."""
     H, B, d = _check_qkv(q, k, v)
-    _check_qkv(q, q_prev, q_prev)
+    if not isinstance(q_prev, torch.Tensor) or q_prev.dtype != torch.bfloat16 or q_prev.shape != q.shape \
+            or q_prev.device != q.device or not q_prev.is_contiguous():
+        raise ValueError(f"q_prev must be a contiguous bf16 tensor shaped like q {tuple(q.shape)} on {q.device}")
     P = _check_prefix(k_pre, v_pre, H, d, q.device)
     n_sel = state.sel.shape[2]
     out, lse = _alloc_out(q, None, None)
@@ -543,6 +545,10 @@ def losa_block(qs, ks, vs, k_pre, v_pre, n_sel=2, tau=0.01, scale=None, bq=64, b
         out = torch.empty_like(qs)
     if lse is None:
         lse = torch.empty((T, H, B), dtype=torch.float32, device=qs.device)
+    if out.shape != qs.shape or out.dtype != torch.bfloat16 or out.device != qs.device or not out.is_contiguous():
+        raise ValueError(f"out must be a contiguous bf16 tensor shaped {tuple(qs.shape)} on {qs.device}")
+    if lse.shape != (T, H, B) or lse.dtype != torch.float32 or lse.device != qs.device or not lse.is_contiguous():
+        raise ValueError(f"lse must be a contiguous fp32 tensor shaped {(T, H, B)} on {qs.device}")
     active = torch.empty((T, B), dtype=torch.int32, device=qs.device)
     ucount = torch.empty((T, H), dtype=torch.int32, device=qs.device)
     rc = _lib.load().sparsed_losa_block(

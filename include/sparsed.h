@@ -366,7 +366,14 @@ int sparsed_select_pattern_noalloc(const uint16_t* Q, const uint16_t* K, const u
  * Pointers: device memory, Q/K/V/prefix/o_cache/O 16-byte aligned, the rest
  * 4-byte aligned; the workspace 256-byte aligned. Returns as every entry
  * point; the union-building kernel reports a selection entry outside [0, nkb)
- * as SPARSED_ERR_BAD_PATTERN (skipping it). */
+ * as SPARSED_ERR_BAD_PATTERN (skipping it).
+ *
+ * Streams: the block's own attention of a step runs on a second stream that
+ * the library creates once per device (non-blocking), forked from `stream`
+ * with an event before it and joined back into `stream` with an event before
+ * the merge; to the caller the step is ordered on `stream` alone, and a graph
+ * capture of `stream` records both branches. Make the first call on a device
+ * outside a graph capture (it creates that stream and its two events). */
 
 /* Splits for a step of these sizes on a GPU with sm_count SMs: as many as
  * keep one split's H*ceil(B/bq) work items per SM at most
