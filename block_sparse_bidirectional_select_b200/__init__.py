@@ -51,6 +51,7 @@ __all__ = ["dense_attn", "select_pattern", "block_sparse_attn", "run_steps", "wo
            "RunResult", "default_scale", "column_keep", "column_workspace_bytes", "select_columns",
            "column_sparse_attn", "run_steps_columns", "ColumnPattern", "select_head_entropy",
            "entropy_budget", "select_with_head_k", "select_pattern_sharded", "gather_head_entropies",
+           "run_steps_sharded", "step_segments",
            "losa_splits", "losa_workspace_bytes", "losa_init", "losa_step", "losa_block", "BlockState",
            "LosaStep", "LosaBlock"]
 
@@ -215,9 +216,10 @@ class RunResult:
 
 def run_steps(q, k, v, T, warmup_frac=0.2, keep=0.1, budget="uniform", refresh_every=0, scale=None,
               bq=128, bk=128, start_step=0, pattern=None, time_steps=False, out=None, lse=None,
-              workspace=None, stream=None) -> RunResult:
+              workspace=None, stream=None, end_step=None) -> RunResult:
     """The denoising loop over one layer: dense warm-up, pattern selection at
-    the switch (and at anchors), block-sparse attention afterwards."""
+    the switch (and at anchors), block-sparse attention afterwards. With
+    ``end_step`` only steps start_step .. end_step-1 of the T-step schedule run."""
     H, L, d = _check_qkv(q, k, v)
     scale = default_scale(d) if scale is None else scale
     mode = {"uniform": BUDGET_UNIFORM, "entropy": BUDGET_ENTROPY}[budget]
@@ -236,12 +238,18 @@ def run_steps(q, k, v, T, warmup_frac=0.2, keep=0.1, budget="uniform", refresh_e
     ws = workspace
     kinds = (ctypes.c_int8 * max(T, 1))()
     ms = (ctypes.c_float * max(T, 1))() if time_steps else None
-    rc = _lib.load().sparsed_run_steps(
-        _ptr(q), _ptr(k), _ptr(v), H, L, d, scale, bq, bk, keep, mode, T, warmup_frac, refresh_every,
-        start_step, have, _ptr(kv_idx), _ptr(kv_count), kv_idx.shape[2], _ptr(out), _ptr(lse),
-        ctypes.cast(kinds, ctypes.c_void_p), None if ms is None else ctypes.cast(ms, ctypes.c_void_p),
-        _ptr(ws), ws.numel(), _stream(stream))
-    check(rc, "sparsed_run_steps")
+    tail = (_ptr(kv_idx), _ptr(kv_count), kv_idx.shape[2], _ptr(out), _ptr(lse),
+            ctypes.cast(kinds, ctypes.c_void_p), None if ms is None else ctypes.cast(ms, ctypes.c_void_p),
+            _ptr(ws), ws.numel(), _stream(stream))
+    if end_step is None:
+        rc = _lib.load().sparsed_run_steps(_ptr(q), _ptr(k), _ptr(v), H, L, d, scale, bq, bk, keep, mode, T,
+                                           warmup_frac, refresh_every, start_step, have, *tail)
+        check(rc, "sparsed_run_steps")
+    else:
+        rc = _lib.load().sparsed_run_steps_span(_ptr(q), _ptr(k), _ptr(v), H, L, d, scale, bq, bk, keep, mode,
+                                                T, warmup_frac, refresh_every, start_step, end_step, have,
+                                                *tail)
+        check(rc, "sparsed_run_steps_span")
     return RunResult(out, lse, list(kinds[:T]), None if ms is None else list(ms[:T]), kv_idx, kv_count)
 
 
@@ -337,13 +345,13 @@ def run_steps_columns(q, k, v, T, warmup_frac=0.2, keep=0.1, refresh_every=0, sc
 
 # ---------------------------------------------------------------- head-sharded selection
 
-def select_head_entropy(q, k, v, scale=None, bq=128, bk=128, workspace=None, stream=None):
+def select_head_entropy(q, k, v, scale=None, bq=128, bk=128, workspace=None, stream=None, out=None, lse=None):
     """Full pass, block mass and the mean row entropy of every head:
     returns (o, lse, head_entropy [H] fp64 on the device, workspace). The
     workspace keeps the block mass for select_with_head_k."""
     H, L, d = _check_qkv(q, k, v)
     scale = default_scale(d) if scale is None else scale
-    out, lse = _alloc_out(q, None, None)
+    out, lse = _alloc_out(q, out, lse)
     ent = torch.empty(H, dtype=torch.float64, device=q.device)
     ws = _workspace(q, bq, bk, workspace)
     rc = _lib.load().sparsed_select_head_entropy(_ptr(q), _ptr(k), _ptr(v), H, L, d, scale, bq, bk, _ptr(out),
@@ -394,15 +402,17 @@ def gather_head_entropies(ent, group=None):
 
 
 def select_pattern_sharded(q, k, v, keep=0.1, group=None, scale=None, bq=128, bk=128, workspace=None,
-                           stream=None) -> Pattern:
+                           stream=None, out=None, lse=None, gather=None) -> Pattern:
     """Entropy-budget pattern selection for this rank's heads of a layer whose
     heads are split evenly over the ranks of ``group`` (in rank order). The
     per-head entropies are all-gathered, every rank runs the same host
     allocation over all heads, and keeps its own heads' k_h. Without a group
-    the local heads are the whole layer."""
+    the local heads are the whole layer. ``gather`` (optional) replaces the
+    all-gather: a function from this rank's entropies to (all entropies in
+    head order as a CPU tensor, this rank's index)."""
     H, L, d = _check_qkv(q, k, v)
-    out, lse, ent, ws = select_head_entropy(q, k, v, scale, bq, bk, workspace, stream)
-    ent_all, rank = gather_head_entropies(ent, group)
+    out, lse, ent, ws = select_head_entropy(q, k, v, scale, bq, bk, workspace, stream, out, lse)
+    ent_all, rank = gather(ent) if gather is not None else gather_head_entropies(ent, group)
     nkb = -(-L // bk)
     head_k_all = entropy_budget(ent_all.tolist(), nkb, keep)
     kv_idx, kv_count, hk = select_with_head_k(H, L, head_k_all[rank * H:(rank + 1) * H], ws, bq, bk, stream)
@@ -557,3 +567,56 @@ def losa_block(qs, ks, vs, k_pre, v_pre, n_sel=2, tau=0.01, scale=None, bq=64, b
         _ptr(ucount), _ptr(st.workspace), st.workspace.numel(), _stream(stream))
     check(rc, "sparsed_losa_block")
     return LosaBlock(out, lse, active, ucount, st)
+
+
+# ---------------------------------------------------------------- head-sharded denoising loop
+
+def step_segments(kinds):
+    """The schedule cut at its SELECT steps: a list of ("select", t) and
+    ("span", t0, t1) entries in step order, spans holding no SELECT step."""
+    segs, t0 = [], 0
+    for t, kind in enumerate(kinds):
+        if kind == STEP_SELECT:
+            if t > t0:
+                segs.append(("span", t0, t))
+            segs.append(("select", t))
+            t0 = t + 1
+    if t0 < len(kinds):
+        segs.append(("span", t0, len(kinds)))
+    return segs
+
+
+def run_steps_sharded(q, k, v, T, warmup_frac=0.2, keep=0.1, budget="entropy", refresh_every=0, group=None,
+                      scale=None, bq=128, bk=128, out=None, lse=None, workspace=None, stream=None,
+                      gather=None) -> RunResult:
+    """The denoising loop for this rank's heads of a layer whose heads are
+    split evenly over the ranks of ``group`` (rank order = head order).
+
+    A uniform budget is per head, so the loop is run_steps on the local heads
+    and nothing crosses ranks. The entropy budget spans every head of the
+    layer: each SELECT step is select_pattern_sharded (full pass, per-head
+    entropies, one all-gather of H values, the allocation on every rank, local
+    top-k), and the steps between run through sparsed_run_steps_span with the
+    pattern so far. ``gather`` as in select_pattern_sharded."""
+    H, L, d = _check_qkv(q, k, v)
+    scale = default_scale(d) if scale is None else scale
+    if budget == "uniform":
+        return run_steps(q, k, v, T, warmup_frac, keep, "uniform", refresh_every, scale, bq, bk, out=out,
+                         lse=lse, workspace=workspace, stream=stream)
+    if budget != "entropy":
+        raise ValueError(f"unknown budget {budget!r}")
+    out, lse = _alloc_out(q, out, lse)
+    if workspace is None:
+        workspace = torch.empty(run_steps_workspace_bytes(H, L, bq, bk), dtype=torch.uint8, device=q.device)
+    kinds = schedule(T, warmup_frac, refresh_every)
+    kv_idx = kv_count = None
+    for seg in step_segments(kinds):
+        if seg[0] == "select":
+            pat = select_pattern_sharded(q, k, v, keep, group, scale, bq, bk, workspace, stream, out, lse, gather)
+            kv_idx, kv_count = pat.kv_idx, pat.kv_count
+        else:
+            _, t0, t1 = seg
+            run_steps(q, k, v, T, warmup_frac, keep, "entropy", refresh_every, scale, bq, bk, start_step=t0,
+                      pattern=None if kv_idx is None else (kv_idx, kv_count), out=out, lse=lse,
+                      workspace=workspace, stream=stream, end_step=t1)
+    return RunResult(out, lse, kinds, None, kv_idx, kv_count)

@@ -48,6 +48,8 @@ SIGNATURES = {
     "sparsed_run_steps": (_I, [_P, _P, _P, _I, _I, _I, _F, _I, _I, _F, _I, _I, _F, _I, _I, _I, _P, _P,
                                _I, _P, _P, _P, _P, _P, _SZ, _P]),
     "sparsed_run_steps_workspace_bytes": (_I, [_I, _I, _I, _I, ctypes.POINTER(_SZ)]),
+    "sparsed_run_steps_span": (_I, [_P, _P, _P, _I, _I, _I, _F, _I, _I, _F, _I, _I, _F, _I, _I, _I, _I, _P,
+                                    _P, _I, _P, _P, _P, _P, _P, _SZ, _P]),
     "sparsed_select_head_entropy": (_I, [_P, _P, _P, _I, _I, _I, _F, _I, _I, _P, _P, _P, _P, _SZ, _P]),
     "sparsed_entropy_budget": (_I, [_P, _I, _I, _F, _P]),
     "sparsed_select_with_head_k": (_I, [_I, _I, _I, _I, _P, _P, _P, _I, _P, _SZ, _P]),

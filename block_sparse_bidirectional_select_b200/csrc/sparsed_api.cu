@@ -604,7 +604,18 @@ int sparsed_run_steps(const uint16_t* Q, const uint16_t* K, const uint16_t* V, i
                       int32_t* kv_idx, int32_t* kv_count, int kv_stride, uint16_t* O, float* LSE,
                       int8_t* step_kind, float* step_ms, void* workspace, size_t workspace_bytes,
                       void* stream) {
-  if (T < 0 || start_step < 0 || start_step > T) return SPARSED_ERR_INVALID_ARG;
+  return sparsed_run_steps_span(Q, K, V, H, L, d, scale, bq, bk, keep_ratio, budget_mode, T, warmup_frac,
+                                refresh_every, start_step, T, have_pattern, kv_idx, kv_count, kv_stride, O, LSE,
+                                step_kind, step_ms, workspace, workspace_bytes, stream);
+}
+
+int sparsed_run_steps_span(const uint16_t* Q, const uint16_t* K, const uint16_t* V, int H, int L, int d,
+                           float scale, int bq, int bk, float keep_ratio, int budget_mode, int T,
+                           float warmup_frac, int refresh_every, int start_step, int end_step,
+                           int have_pattern, int32_t* kv_idx, int32_t* kv_count, int kv_stride, uint16_t* O,
+                           float* LSE, int8_t* step_kind, float* step_ms, void* workspace,
+                           size_t workspace_bytes, void* stream) {
+  if (T < 0 || start_step < 0 || start_step > end_step || end_step > T) return SPARSED_ERR_INVALID_ARG;
   std::vector<int8_t> kinds(static_cast<size_t>(T) + 1);
   SP_TRY(sparsed_schedule(T, warmup_frac, refresh_every, kinds.data()));
   if (step_kind && T > 0) std::memcpy(step_kind, kinds.data(), static_cast<size_t>(T));
@@ -615,14 +626,14 @@ int sparsed_run_steps(const uint16_t* Q, const uint16_t* K, const uint16_t* V, i
   SP_TRY(prepare(Q, K, V, H, L, d, scale, bq, bk, O, LSE, &p, &empty));
   if (empty) return SPARSED_OK;
   bool any_select = false, pattern_ready = have_pattern != 0;
-  for (int t = start_step; t < T; ++t) {
+  for (int t = start_step; t < end_step; ++t) {
     if (kinds[t] == SPARSED_STEP_SELECT) pattern_ready = any_select = true;
     if (kinds[t] == SPARSED_STEP_SPARSE && !pattern_ready) return SPARSED_ERR_INVALID_ARG;
   }
   if (any_select)
     SP_TRY(check_select_args(p, keep_ratio, budget_mode, kv_idx, kv_count, kv_stride, workspace,
                              workspace_bytes));
-  else if (start_step < T && pattern_ready && (!kv_idx || !kv_count || kv_stride < 1))
+  else if (start_step < end_step && pattern_ready && (!kv_idx || !kv_count || kv_stride < 1))
     return SPARSED_ERR_INVALID_ARG;
   SP_TRY(require_sm100());
   SP_TRY(get_encoder());
@@ -633,17 +644,17 @@ int sparsed_run_steps(const uint16_t* Q, const uint16_t* K, const uint16_t* V, i
                      static_cast<long long>(p.H) * p.nqb * p.nkb * 8 < (1ll << 31);
   bool have_lse = false;  // a full pass of this call left its LSE in the workspace
   std::vector<cudaEvent_t> ev;
-  if (step_ms && start_step < T) {
-    ev.resize(static_cast<size_t>(T - start_step) + 1, nullptr);
+  if (step_ms && start_step < end_step) {
+    ev.resize(static_cast<size_t>(end_step - start_step) + 1, nullptr);
     for (auto& e : ev) SP_CUDA(cudaEventCreate(&e));
     SP_CUDA(cudaEventRecord(ev[0], st));
   }
   int rc = SPARSED_OK;
-  for (int t = start_step; t < T && rc == SPARSED_OK; ++t) {
+  for (int t = start_step; t < end_step && rc == SPARSED_OK; ++t) {
     switch (kinds[t]) {
       case SPARSED_STEP_DENSE:
         rc = launch_attn(p, false, nullptr, nullptr, 0, st);
-        if (rc == SPARSED_OK && fused && t + 1 < T && kinds[t + 1] == SPARSED_STEP_SELECT) {
+        if (rc == SPARSED_OK && fused && t + 1 < end_step && kinds[t + 1] == SPARSED_STEP_SELECT) {
           rc = save_lse(p, workspace, st);
           have_lse = true;
         }
@@ -675,7 +686,7 @@ int sparsed_run_steps(const uint16_t* Q, const uint16_t* K, const uint16_t* V, i
     if (rc == SPARSED_OK) {
       cudaError_t e = cudaEventSynchronize(ev.back());
       if (e != cudaSuccess) rc = fail_cuda(e);
-      for (int t = start_step; t < T && rc == SPARSED_OK; ++t) {
+      for (int t = start_step; t < end_step && rc == SPARSED_OK; ++t) {
         float ms = 0.f;
         e = cudaEventElapsedTime(&ms, ev[t - start_step], ev[t - start_step + 1]);
         if (e != cudaSuccess) rc = fail_cuda(e);

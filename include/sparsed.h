@@ -205,6 +205,23 @@ int sparsed_run_steps(const uint16_t* Q, const uint16_t* K, const uint16_t* V,
                       int8_t* step_kind, float* step_ms,
                       void* workspace, size_t workspace_bytes, void* stream);
 
+/* Steps start_step .. end_step-1 of the same loop (0 <= start_step <=
+ * end_step <= T): the schedule is still that of T steps, so a run can be cut
+ * into spans and continued -- e.g. around SELECT steps that the caller runs
+ * itself (the head-sharded entropy selection below). Arguments and outputs
+ * as sparsed_run_steps; step_ms receives the span's steps (0 elsewhere); a
+ * SELECT step inside the span uses the fused block mass only when a full pass
+ * of the same span comes before it. */
+int sparsed_run_steps_span(const uint16_t* Q, const uint16_t* K, const uint16_t* V,
+                           int H, int L, int d, float scale, int bq, int bk,
+                           float keep_ratio, int budget_mode,
+                           int T, float warmup_frac, int refresh_every,
+                           int start_step, int end_step, int have_pattern,
+                           int32_t* kv_idx, int32_t* kv_count, int kv_stride,
+                           uint16_t* O, float* LSE,
+                           int8_t* step_kind, float* step_ms,
+                           void* workspace, size_t workspace_bytes, void* stream);
+
 /* ---- Head-sharded selection with the entropy budget (the heads of one
  * layer split over several GPUs: only the per-head entropies cross ranks, one
  * all-gather of H doubles per selection; Step-dLLM abstract: head-adaptive

@@ -103,3 +103,87 @@ def test_two_shards_on_one_gpu_equal_the_unsharded_selection():
                 assert torch.equal(kv_idx[h, i, :c], full.kv_idx[s][h, i, :c])
         assert torch.equal(o.view(torch.int16), full.o[s].view(torch.int16))
         assert torch.equal(lse, full.lse[s])
+
+
+def test_step_segments_cut_the_schedule_at_select_steps():
+    kinds = sp.schedule(10, 0.3, 3)
+    assert kinds == [0, 0, 1, 2, 2, 1, 2, 2, 1, 2]
+    assert sp.step_segments(kinds) == [("span", 0, 2), ("select", 2), ("span", 3, 5), ("select", 5),
+                                       ("span", 6, 8), ("select", 8), ("span", 9, 10)]
+    assert sp.step_segments(sp.schedule(4, 1.0, 0)) == [("span", 0, 4)]          # all dense, no select
+    assert sp.step_segments(sp.schedule(5, 0.2, 0)) == [("select", 0), ("span", 1, 5)]
+    assert sp.step_segments([]) == []
+    # every step is covered once, in order
+    for T, w, r in [(1, 0.0, 0), (7, 0.5, 1), (256, 0.2, 0), (512, 0.2, 64)]:
+        steps = []
+        for seg in sp.step_segments(sp.schedule(T, w, r)):
+            steps += [seg[1]] if seg[0] == "select" else list(range(seg[1], seg[2]))
+        assert steps == list(range(T))
+
+
+@pytest.mark.gpu
+def test_sharded_denoising_loop_two_shards_in_two_threads():
+    """Two ranks emulated by two host threads on one GPU (each its own stream;
+    the all-gather replaced by an in-process exchange behind a barrier; no
+    kernel waits on another): the loop with the entropy budget, anchors
+    included, gives each shard exactly the heads of the unsharded loop."""
+    import threading
+
+    from block_sparse_bidirectional_select_b200.inputs import WORKLOADS, make_inputs
+    wl = WORKLOADS["tiny"].scaled(H=4, L=1024, d=128, bq=128, bk=128, seed=404, structure="band")
+    q, k, v = (t.cuda() for t in make_inputs(wl))
+    T, w, r, keep = 7, 0.3, 2, 0.2
+    full = sp.run_steps_sharded(q, k, v, T, w, keep, "entropy", r)
+    sp.device_check()
+    shards = [slice(0, 2), slice(2, 4)]
+    barrier = threading.Barrier(2)
+    slots = [None, None]
+    results = [None, None]
+    errors = []
+
+    def make_gather(rank):
+        def gather(ent):
+            slots[rank] = ent.cpu()
+            barrier.wait(timeout=120)
+            ent_all = torch.cat(slots)
+            barrier.wait(timeout=120)
+            return ent_all, rank
+        return gather
+
+    def worker(rank):
+        try:
+            s = torch.cuda.Stream()
+            with torch.cuda.stream(s):
+                sl = shards[rank]
+                res = sp.run_steps_sharded(q[sl].contiguous(), k[sl].contiguous(), v[sl].contiguous(), T, w,
+                                           keep, "entropy", r, stream=s, gather=make_gather(rank))
+                s.synchronize()
+                results[rank] = res
+        except Exception as e:  # reported below; the barrier times out for the other thread
+            errors.append(e)
+            barrier.abort()
+
+    threads = [threading.Thread(target=worker, args=(i,)) for i in range(2)]
+    for t in threads:
+        t.start()
+    for t in threads:
+        t.join(300)
+    assert not errors, errors
+    sp.device_check()
+    assert full.kinds.count(sp.STEP_SELECT) == 3
+    for res, sl in zip(results, shards):
+        assert torch.equal(res.kv_count, full.kv_count[sl])
+        for h in range(2):
+            for i in range(res.kv_count.shape[1]):
+                c = int(res.kv_count[h, i])
+                assert torch.equal(res.kv_idx[h, i, :c], full.kv_idx[sl][h, i, :c])
+        assert torch.equal(res.o.view(torch.int16), full.o[sl].view(torch.int16))
+        assert torch.equal(res.lse, full.lse[sl])
+    # the last step's output is the block-sparse attention over the final pattern
+    qh, kh, vh = (t.float().cpu().numpy().astype(np.float64) for t in (q, k, v))
+    idx, cnt = full.kv_idx.cpu().numpy(), full.kv_count.cpu().numpy()
+    for h in range(4):
+        lists = [idx[h, i, :cnt[h, i]] for i in range(idx.shape[1])]
+        o_ref, l_ref = O.masked_attention(qh[h], kh[h], vh[h], wl.scale, lists, cnt[h], 128, 128)
+        assert np.abs(full.o[h].float().cpu().numpy() - o_ref).max() <= 2e-2
+        assert np.abs(full.lse[h].cpu().numpy() - l_ref).max() <= 1e-3
