@@ -132,7 +132,7 @@ def test_sharded_denoising_loop_two_shards_in_two_threads():
     from block_sparse_bidirectional_select_b200.inputs import WORKLOADS, make_inputs
     wl = WORKLOADS["tiny"].scaled(H=4, L=1024, d=128, bq=128, bk=128, seed=404, structure="band")
     q, k, v = (t.cuda() for t in make_inputs(wl))
-    T, w, r, keep = 7, 0.3, 2, 0.2
+    T, w, r, keep = 8, 0.3, 2, 0.2  # selects at steps 2, 4, 6; the last step is block-sparse
     full = sp.run_steps_sharded(q, k, v, T, w, keep, "entropy", r)
     sp.device_check()
     shards = [slice(0, 2), slice(2, 4)]
@@ -170,7 +170,7 @@ def test_sharded_denoising_loop_two_shards_in_two_threads():
         t.join(300)
     assert not errors, errors
     sp.device_check()
-    assert full.kinds.count(sp.STEP_SELECT) == 3
+    assert full.kinds.count(sp.STEP_SELECT) == 3 and full.kinds[-1] == sp.STEP_SPARSE
     for res, sl in zip(results, shards):
         assert torch.equal(res.kv_count, full.kv_count[sl])
         for h in range(2):
