@@ -4,7 +4,6 @@ pass, the block-mass row, the selection (margin rule and kernel-precision
 exactness), and the block-sparse output with the GPU's own pattern."""
 import numpy as np
 import pytest
-import torch
 
 import oracle as O
 import block_sparse_bidirectional_select_b200 as sp
