@@ -232,3 +232,37 @@ def test_losa_block_validation():
     assert f(*a) == _lib.ERR_INVALID_ARG
     if not GPU:
         assert f(*args) == _lib.ERR_NO_DEVICE
+
+
+def test_run_steps_span_validation():
+    f = lib.sparsed_run_steps_span
+    # T=10, warm-up 0.2: steps 0 dense, 1 select, 2..9 sparse
+    args = [P, P, P, 2, 512, 128, 0.088, 128, 128, 0.5, 0, 10, 0.2, 0, 0, 10, 0, P, P, 2, P, P, None, None,
+            P, 1 << 20, None]
+    a = list(args)
+    a[14], a[15] = 4, 3             # start after end
+    assert f(*a) == _lib.ERR_INVALID_ARG
+    a = list(args)
+    a[15] = 11                      # end past T
+    assert f(*a) == _lib.ERR_INVALID_ARG
+    a = list(args)
+    a[14], a[15] = 2, 5             # sparse steps without a pattern
+    assert f(*a) == _lib.ERR_INVALID_ARG
+    a = list(args)
+    a[14], a[15], a[16] = 2, 5, 1   # ... with one: no workspace needed (no select in the span)
+    a[24] = None
+    if not GPU:
+        assert f(*a) == _lib.ERR_NO_DEVICE
+    a = list(args)
+    a[14], a[15] = 0, 2             # the span holds the select: it needs the workspace
+    a[24] = None
+    assert f(*a) == _lib.ERR_WORKSPACE
+    a = list(args)
+    a[14], a[15] = 3, 3             # an empty span validates and launches nothing
+    a[16] = 1
+    kinds = (ctypes.c_int8 * 10)()
+    a[22] = ctypes.cast(kinds, ctypes.c_void_p)
+    rc = f(*a)
+    assert list(kinds) == O.schedule(10, 0.2, 0)
+    if not GPU:
+        assert rc == _lib.ERR_NO_DEVICE
