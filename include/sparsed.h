@@ -17,6 +17,10 @@
  *   - block-sparse attention that visits only the kept key blocks
  *     (Step-dLLM abstract: block-sparse attention kernel; PulseCol abstract:
  *      block-sparse computation in the later iterations).
+ * Beside these: a column-sparse pattern (PulseCol abstract), a head-sharded
+ * entropy selection and step driver, and block-wise generation over a prefix
+ * cache with active-token reuse (LoSA: Locality Aware Sparse Attention for
+ * Block-Wise Diffusion Language Models); each section below says which.
  *
  * Conventions shared by every entry point
  *   Layout    Q, K, V, O are [H, L, d] bf16 (raw 16-bit patterns), row-major,
