@@ -77,7 +77,7 @@ enum {
 enum { SPARSED_BUDGET_UNIFORM = 0, SPARSED_BUDGET_ENTROPY = 1 };
 enum { SPARSED_STEP_DENSE = 0, SPARSED_STEP_SELECT = 1, SPARSED_STEP_SPARSE = 2 };
 
-/* Library version (SPARSED_VERSION of the build). Never fails. */
+/* Library version (the SPARSED_VERSION it was compiled with). Never fails. */
 int sparsed_version(void);
 
 /* Static message for a status code; never NULL. */
