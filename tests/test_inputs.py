@@ -56,3 +56,26 @@ def test_low_rank_scores_concentrated():
 def test_zero_q():
     q, k, v = zero_q(WORKLOADS["tiny"].scaled(H=1, L=64))
     assert (q == 0).all() and k.abs().sum() > 0
+
+
+def test_block_workload_recipe():
+    """The block-wise inputs: deterministic per seed, bf16, and at every step
+    after the first exactly round(0.25*B) tokens change by far more than tau
+    while every other token's query MSE stays far below it."""
+    import numpy as np
+
+    import oracle as O
+    from block_sparse_bidirectional_select_b200.inputs import BLOCK_WORKLOADS, make_block_inputs, to_f64
+    wl = BLOCK_WORKLOADS["losa_tiny"]
+    a = make_block_inputs(wl)
+    b = make_block_inputs(wl)
+    for x, y in zip(a, b):
+        assert x.dtype == torch.bfloat16 and torch.equal(x.view(torch.int16), y.view(torch.int16))
+    k_pre, v_pre, qs, ks, vs = a
+    assert k_pre.shape == (wl.H, wl.P, wl.d) and qs.shape == (wl.T, wl.H, wl.B, wl.d)
+    n_act = round(wl.active_frac * wl.B)
+    for t in range(1, wl.T):
+        mse = O.query_mse(to_f64(qs[t]), to_f64(qs[t - 1]))
+        act = mse > wl.tau
+        assert act.sum() == n_act
+        assert mse[act].min() > 10 * wl.tau and mse[~act].max() < wl.tau / 10
