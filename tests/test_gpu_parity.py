@@ -342,3 +342,19 @@ def test_empty_problem_is_noop():
     q = torch.zeros((2, 0, 64), dtype=torch.bfloat16, device="cuda")
     o, lse = sp.dense_attn(q, q, q)
     sp.device_check()
+
+
+@pytest.mark.parametrize("d,L", [(64, 1000), (128, 2048)])
+def test_dense_attn_agrees_with_torch_sdpa(d, L):
+    """A library cross-check beside the oracle: torch's scaled_dot_product_attention
+    (flash / cuDNN kernels) on the same bf16 inputs, and the LSE of fp32 scores."""
+    import torch.nn.functional as F
+    q, k, v, scale = _inputs(2, L, d, seed=500 + d)
+    qc, kc, vc = _cuda(q, k, v)
+    o, lse = sp.dense_attn(qc, kc, vc)
+    sp.device_check()
+    ref = F.scaled_dot_product_attention(qc.unsqueeze(0), kc.unsqueeze(0), vc.unsqueeze(0), scale=scale)[0]
+    err = (o.float() - ref.float()).abs()
+    assert err.max().item() <= 2e-2 and err.mean().item() <= 2e-3
+    s = torch.matmul(qc.float(), kc.float().transpose(1, 2)) * scale
+    assert (lse - torch.logsumexp(s, dim=-1)).abs().max().item() <= 1e-3
