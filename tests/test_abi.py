@@ -266,3 +266,32 @@ def test_run_steps_span_validation():
     assert list(kinds) == O.schedule(10, 0.2, 0)
     if not GPU:
         assert rc == _lib.ERR_NO_DEVICE
+
+
+def _losa_init(**kw):
+    a = dict(Q=P, K=P, V=P, Kp=P, Vp=P, H=2, B=64, P_=4096, d=128, scale=0.088, bq=64, bk=64, n_sel=2, splits=2,
+             oc=P, lc=P, sel=P, O_=P, LSE=P, mass=None, ws=P, ws_bytes=1 << 30)
+    a.update(kw)
+    return lib.sparsed_losa_init(a["Q"], a["K"], a["V"], a["Kp"], a["Vp"], a["H"], a["B"], a["P_"], a["d"],
+                                 a["scale"], a["bq"], a["bk"], a["n_sel"], a["splits"], a["oc"], a["lc"],
+                                 a["sel"], a["O_"], a["LSE"], a["mass"], a["ws"], a["ws_bytes"], None)
+
+
+def test_losa_init_validation():
+    assert _losa_init(Kp=None) == _lib.ERR_INVALID_ARG
+    assert _losa_init(sel=None) == _lib.ERR_INVALID_ARG
+    assert _losa_init(oc=MIS) == _lib.ERR_INVALID_ARG            # the cache must be 16-byte aligned
+    assert _losa_init(lc=ctypes.c_void_p(0x10002)) == _lib.ERR_INVALID_ARG
+    assert _losa_init(mass=ctypes.c_void_p(0x10001)) == _lib.ERR_INVALID_ARG
+    assert _losa_init(scale=float("inf")) == _lib.ERR_INVALID_ARG
+    assert _losa_init(d=96) == _lib.ERR_UNSUPPORTED
+    assert _losa_init(bk=32) == _lib.ERR_UNSUPPORTED
+    assert _losa_init(B=0) == _lib.ERR_INVALID_ARG
+    assert _losa_init(P_=0) == _lib.ERR_INVALID_ARG
+    assert _losa_init(n_sel=0) == _lib.ERR_INVALID_ARG
+    assert _losa_init(splits=0) == _lib.ERR_INVALID_ARG
+    assert _losa_init(ws=None) == _lib.ERR_WORKSPACE
+    assert _losa_init(ws=ctypes.c_void_p(0x10010)) == _lib.ERR_WORKSPACE   # not 256-byte aligned
+    assert _losa_init(ws_bytes=1 << 10) == _lib.ERR_WORKSPACE
+    if not GPU:
+        assert _losa_init() == _lib.ERR_NO_DEVICE
