@@ -1033,9 +1033,21 @@ int side_stream(SideStream** out) {
   std::lock_guard<std::mutex> lock(g_side_init_mu);
   SideStream& ss = g_side[dev];
   if (ss.s == nullptr) {
-    SP_CUDA(cudaStreamCreateWithFlags(&ss.s, cudaStreamNonBlocking));
-    SP_CUDA(cudaEventCreateWithFlags(&ss.fork, cudaEventDisableTiming));
-    SP_CUDA(cudaEventCreateWithFlags(&ss.join, cudaEventDisableTiming));
+    // all three or none: a failed creation leaves the slot empty for a retry
+    cudaStream_t s = nullptr;
+    cudaEvent_t fork = nullptr, join = nullptr;
+    cudaError_t e = cudaStreamCreateWithFlags(&s, cudaStreamNonBlocking);
+    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&fork, cudaEventDisableTiming);
+    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&join, cudaEventDisableTiming);
+    if (e != cudaSuccess) {
+      if (join) cudaEventDestroy(join);
+      if (fork) cudaEventDestroy(fork);
+      if (s) cudaStreamDestroy(s);
+      return fail_cuda(e);
+    }
+    ss.fork = fork;
+    ss.join = join;
+    ss.s = s;
   }
   *out = &ss;
   return SPARSED_OK;
