@@ -1222,8 +1222,13 @@ int losa_init_impl(const LosaDims& g, const uint16_t* Q, const uint16_t* K, cons
     SP_CUDA(cudaStreamWaitEvent(side->s, side->fork, 0));
     SP_TRY(losa_suffix(g, Q, K, V, scale, O, LSE, side->s));
     SP_CUDA(cudaEventRecord(side->join, side->s));
-    SP_TRY(losa_lists(g, nullptr, nullptr, sel_stride, Q, nullptr, nullptr, ws, st));
-    SP_TRY(losa_prefix_and_merge(g, Kp, Vp, scale, true, o_cache, lse_cache, O, LSE, ws, st, side->join));
+    int rc = losa_lists(g, nullptr, nullptr, sel_stride, Q, nullptr, nullptr, ws, st);
+    if (rc == SPARSED_OK)
+      rc = losa_prefix_and_merge(g, Kp, Vp, scale, true, o_cache, lse_cache, O, LSE, ws, st, side->join);
+    if (rc != SPARSED_OK) {
+      cudaStreamWaitEvent(st, side->join, 0);  // the caller's stream stays ordered after the suffix
+      return rc;
+    }
   }
   float* mass = token_mass ? token_mass : reinterpret_cast<float*>(ws + w.mass);
   SP_TRY(launch_tok_mass(g, Q, Kp, scale, lse_cache, mass, st));
@@ -1252,9 +1257,13 @@ int losa_step_impl(const LosaDims& g, const uint16_t* Q, const uint16_t* K, cons
   SP_TRY(losa_suffix(g, Q, K, V, scale, O, LSE, side->s));
   SP_CUDA(cudaEventRecord(side->join, side->s));
   query_mse_kernel<<<g.B, 256, 0, st>>>(Q, Q_prev, g.H, g.B, g.d, static_cast<double>(tau), act);
-  SP_CUDA(cudaGetLastError());
-  SP_TRY(losa_lists(g, act, sel, sel_stride, Q, union_idx, union_count, ws, st));
-  return losa_prefix_and_merge(g, Kp, Vp, scale, false, o_cache, lse_cache, O, LSE, ws, st, side->join);
+  const cudaError_t e = cudaGetLastError();
+  int rc = e == cudaSuccess ? SPARSED_OK : fail_cuda(e);
+  if (rc == SPARSED_OK) rc = losa_lists(g, act, sel, sel_stride, Q, union_idx, union_count, ws, st);
+  if (rc == SPARSED_OK)
+    rc = losa_prefix_and_merge(g, Kp, Vp, scale, false, o_cache, lse_cache, O, LSE, ws, st, side->join);
+  if (rc != SPARSED_OK) cudaStreamWaitEvent(st, side->join, 0);  // the caller's stream stays ordered after the suffix
+  return rc;
 }
 
 int losa_prepare(int H, int B, int P, int d, int bq, int bk, int n_sel, int splits, float scale, LosaDims* g) {
