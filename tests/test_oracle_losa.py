@@ -258,3 +258,16 @@ def test_block_run_records_and_density_bound():
         assert (r["union_count"][t] <= min(nkb, na * 2)).all()
     ref_o, ref_l = _concat_reference(qs[0], k_pre, v_pre, ks[0], vs[0], 0.4)
     np.testing.assert_allclose(r["o"][0], ref_o, rtol=0, atol=1e-12)
+
+
+def test_block_run_hand_case():
+    c = GOLD["losa_block_three_steps"]
+    r = O.losa_block(np.array(c["qs"]), np.array(c["ks"]), np.array(c["vs"]), np.array(c["k_pre"]),
+                     np.array(c["v_pre"]), c["scale"], c["bk"], c["n_sel"], c["tau"])
+    np.testing.assert_allclose(r["o"][:, 0, 0, 0], c["o"], rtol=0, atol=1e-14)
+    np.testing.assert_allclose(r["lse"][:, 0, 0], c["lse"], rtol=0, atol=1e-14)
+    assert r["active"].tolist() == c["active"]
+    assert r["state"]["sel"][0, 0].tolist() == c["sel"]
+    np.testing.assert_allclose(r["state"]["o_pre"][0, :, 0], c["o_pre_after"], rtol=0, atol=1e-14)
+    np.testing.assert_allclose(r["state"]["lse_pre"][0], c["lse_pre_after"], rtol=0, atol=1e-14)
+    assert r["union_count"].tolist() == [[2], [1], [0]]
