@@ -10,46 +10,50 @@
 // the arithmetic, so a sparse call that keeps every block in ascending order is
 // bitwise equal to the dense call.
 //
-// Persistent CTAs: the grid holds one CTA per SM and CTA b takes the work
-// items b, b + G, b + 2G, ... of the flattened (h, i) order (G = grid size), so
-// the CTAs resident at any moment cover consecutive query blocks of one head
-// and share its K/V tiles in L2. Every pipeline below runs on across item
-// boundaries (the tile counter g counts tiles over all of the CTA's items):
-// the loads, S MMAs and exponentials of item k+1 start while item k's last
-// tiles and its epilogue are still in flight, which matters for the short
-// lists of the sparse steps (a few to a few tens of key blocks per item).
+// Two query tiles per CTA. A CTA works on pairs of work items, (h, 2p) in slot
+// 0 and (h, 2p+1) in slot 1, each slot with its own Q tile, S/P and O in TMEM,
+// its own softmax warpgroup and its own MMA-issuing warp. Per slot the chain
+// is S(t) = Q K_t^T -> softmax -> O += P(t) V_t -> S(t+1); the two slots run
+// it independently, so the tensor core works on one slot's MMAs while the
+// other slot's softmax runs. O += P V is issued in NPV parts, each as soon as
+// the softmax has stored that part of P, so it overlaps the rest of the
+// exponentials. In dense mode both slots read the same K_t / V_t tile; in
+// sparse mode each slot walks its own list and has its own tiles.
+//
+// Persistent CTAs: the grid holds one CTA per SM and CTA b takes the pairs
+// b, b + G, b + 2G, ... of the flattened (h, p) order (G = grid size), so the
+// CTAs resident at any moment cover consecutive query blocks of one head and
+// share its K/V tiles in L2. The pipelines run on across pair boundaries.
 //
 // Warp roles (384 threads):
-//   warps 0-7   softmax. Warp w covers the 16 rows 32*(w%4) + 16*(w/4) + 0..15
-//               of the tile with the "16x32bx2" TMEM access: thread t holds row
-//               t%16 and the column half t/16 of every S tile, so the two
-//               halves of a row meet in one warp (row max / sum by shuffle).
-//   warp 8      TMA producer: Q of each item, K_g / V_g into KS- / VS-deep rings
-//   warp 9      TMEM owner; its lane 0 issues the S = Q K^T MMAs
-//   warp 10     lane 0 issues the O += P V MMAs
+//   warps 0-3   softmax of slot 0: warp w holds rows 32w..32w+31 of the tile,
+//               one full row per thread (row max and sum need no exchange)
+//   warps 4-7   softmax of slot 1, likewise
+//   warp 8      TMA producer: Q of each slot, K/V tiles into one NST-deep ring
+//               in the order the slots consume them
+//   warp 9      TMEM owner; MMA issuer of slot 0
+//   warp 10     MMA issuer of slot 1
 //   warp 11     idle (donates its registers)
-// TMEM (128 lanes): [S0 | S1 | O | P0 | P1] = 2*BK + D + BK fp32 columns. S is
-// double-buffered, so S(g+1) is computed while the softmax works on S(g); P has
-// its own two buffers, so the two issuers never touch the same columns and can
-// run independently (a commit from one thread tracks only its own MMAs):
-//   S issuer : S_b(g) once PV(g-2) is done (which also means the softmax has
-//              read S_b(g-2) and that P_b is free again)       (PVDONE)
-//   softmax  : reads S_b(g), writes P_b(g)                      (SFULL -> PFULL)
-//   PV issuer: O += P_b(g) V_g; the first tile of an item overwrites O, which
-//              the softmax warps have read out before they wrote that P
-//                                                               (PFULL -> PVDONE)
-//   producer : Q of the next item once every S MMA of the current one is
-//              complete                                         (QEMPTY)
-// The lazy rescale keeps O and the running sum on a stale row max until a
-// row's max grows by more than 2^8; both halves of a row see the same max, so
-// they take the same decision, and each rescales its half of O.
-// The epilogue writes O straight from registers to global memory (each thread
-// one contiguous half row), so no shared memory is held across items.
+// The producer and issuers run warp-uniform code and one elected lane issues
+// each copy, MMA and commit.
+// TMEM (128 lanes): [S0 | S1 | O0 | O1] = 2*BK + 2*D fp32 columns. P_s is
+// written as bf16 pairs over the first BK/2 columns of S_s, which PV_s reads
+// before S_s(t+1) overwrites them (MMAs of one thread execute in order).
+// Ordering facts the roles rely on (a slot's MMAs all come from one thread,
+// and a commit tracks every MMA that thread issued before it):
+//   * S_s(t) is issued after PV_s(t-1), so when S_s(t) completes (SFULL_s),
+//     O_s holds every tile before t: the softmax may rescale O_s right away;
+//   * the first part of PV_s(t) waits for the softmax's first PFULL_s(t)
+//     arrival, which follows its rescale of O_s and its epilogue reads of O_s
+//     (the first PV of an item overwrites O_s);
+//   * a ring stage is released by two commits after the MMAs reading it.
+// The lazy rescale keeps O and the running sum on a stale row max until some
+// row of the warp sees its max grow by more than 2^8 (warp-uniform decision).
 // MASS variant (dense only): the pass also yields the block mass of pattern
 // selection. Each tile's probabilities of a row sum to ps = sum_c 2^(s_c*sl2 - m)
 // in the exp pass; times 2^(m - lse2), with lse2 the row's LSE from an earlier
 // full pass of the same inputs, that is the row's mass in the tile, and the
-// warp writes its 16 rows' sum as one of 8 partials per tile.
+// warp writes its 32 rows' sum as one of kMassParts partials per tile.
 // Every wait is bounded (mbarriers only, no named barriers), so a timed-out
 // warp cannot strand the others.
 #pragma once
@@ -57,6 +61,10 @@
 #include "ptx_sm100.cuh"
 
 namespace sparsed {
+
+// Partial block-mass sums per (head, query block, key block) written by the
+// MASS variant: one per softmax warp of a slot.
+constexpr int kMassParts = 4;
 
 struct AttnArgs {
   int H, L, bq, nqb, nkb;
@@ -69,7 +77,7 @@ struct AttnArgs {
   uint16_t* o;               // [H, L, D]
   // block mass from this pass (MASS variant): the LSE of an earlier full pass
   // of the same inputs, and per (head, query block, key block) one partial sum
-  // per softmax warp, [H, nqb, nkb, 8]
+  // per softmax warp, [H, nqb, nkb, kMassParts]
   const float* lse_prev;
   float* mass_part;
   uint64_t timeout_ns;       // bound of every device-side wait
@@ -85,62 +93,52 @@ __device__ __forceinline__ void setmaxnreg_dec_56() {
 template <int D, int BK>
 struct AttnCfg {
   static constexpr int M = 128;
-  static constexpr int HALF = BK / 2;  // S columns per softmax thread
   static constexpr int DCH = D / 64;
-  static constexpr int Q_CHUNK = M * 128;
-  static constexpr int KV_CHUNK = BK * 128;
+  static constexpr int Q_CHUNK = M * 128;    // bytes of one 64-column chunk of a Q tile
+  static constexpr int KV_CHUNK = BK * 128;  // ... of a K or V tile
   static constexpr int Q_BYTES = M * D * 2;
   static constexpr int KV_BYTES = BK * D * 2;
-  static constexpr int KS = 3;
-  // a third V stage when it fits next to Q, three K stages and the barriers
-  static constexpr int VS = (Q_BYTES + 6 * KV_BYTES + 2048) <= 232448 ? 3 : 2;
-  static constexpr int OFF_Q = 0;
-  static constexpr int OFF_K = Q_BYTES;
-  static constexpr int OFF_V = OFF_K + KS * KV_BYTES;
-  static constexpr int OFF_BAR = OFF_V + VS * KV_BYTES;
-  static constexpr int B_QFULL = 0;
-  static constexpr int B_QEMPTY = 1;
-  static constexpr int B_KFULL = 2;
-  static constexpr int B_KEMPTY = B_KFULL + KS;
-  static constexpr int B_VFULL = B_KEMPTY + KS;
-  static constexpr int B_VEMPTY = B_VFULL + VS;
-  static constexpr int B_SFULL = B_VEMPTY + VS;  // [2]
-  static constexpr int B_PFULL = B_SFULL + 2;    // [2] 8 warp arrivals
-  static constexpr int B_PVDONE = B_PFULL + 2;   // [2]
-  static constexpr int B_DRAIN = B_PVDONE + 2;   // [2] per issuer
+  static constexpr int SMEM_LIMIT = 232448;
+  static constexpr int NST_FIT = (SMEM_LIMIT - 1024 - 2 * Q_BYTES - 512) / KV_BYTES;
+  static constexpr int NST = NST_FIT > 8 ? 8 : NST_FIT;  // ring stages (K and V tiles)
+  static constexpr int OFF_Q0 = 0;
+  static constexpr int OFF_Q1 = Q_BYTES;
+  static constexpr int OFF_RING = 2 * Q_BYTES;
+  static constexpr int OFF_BAR = OFF_RING + NST * KV_BYTES;
+  static constexpr int B_QFULL = 0;             // [2]
+  static constexpr int B_QEMPTY = 2;            // [2]
+  static constexpr int B_FULL = 4;              // [NST]
+  static constexpr int B_EMPTY = B_FULL + NST;  // [NST]
+  static constexpr int NPV = 2;                 // parts of P / of the PV MMAs of a tile
+  static constexpr int B_SFULL = B_EMPTY + NST; // [2]
+  static constexpr int B_PFULL = B_SFULL + 2;   // [2][NPV] 4 warp arrivals
+  static constexpr int B_PVDONE = B_PFULL + 2 * NPV;  // [2]
+  static constexpr int B_DRAIN = B_PVDONE + 2;  // [2]
   static constexpr int NUM_BARS = B_DRAIN + 2;
   static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;  // tmem slot, abort flag
   static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;
   static constexpr int TM_S0 = 0;
   static constexpr int TM_S1 = BK;
-  static constexpr int TM_O = 2 * BK;
-  static constexpr int TM_P0 = 2 * BK + D;
-  static constexpr int TM_P1 = TM_P0 + BK / 2;
-  static constexpr int TM_USED = TM_P1 + BK / 2;
+  static constexpr int TM_O0 = 2 * BK;
+  static constexpr int TM_O1 = 2 * BK + D;
+  static constexpr int TM_USED = 2 * BK + 2 * D;
   static constexpr int TM_ALLOC = TM_USED <= 256 ? 256 : 512;
   static constexpr uint32_t IDESC_S = ptx::idesc_bf16_f32(128, BK, 0, 0);
   static constexpr uint32_t IDESC_PV = ptx::idesc_bf16_f32(128, D, 0, 1);
   static constexpr int THREADS = 384;
-  static constexpr int REGS_SOFTMAX = 224;
-  static constexpr int REGS_OTHER = 56;
+  static constexpr int REGS_SOFTMAX = 224;  // warps 0-7
+  static constexpr int REGS_OTHER = 56;     // warps 8-11
+  static_assert(NST >= 4, "ring too shallow");
   static_assert(TM_USED <= 512, "TMEM budget");
-  static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+  static_assert(SMEM_BYTES <= SMEM_LIMIT, "shared memory budget");
 };
 
-// The exp pass of one half row: P = bf16(2^(s*sl2 - m)) for HALF columns into
-// TMEM at p_taddr through the 16x32bx2 access (two columns per 32-bit cell,
-// even column in the low half; the other half row's cells HALF/2 further on),
-// returning the fp32 sum. Column pairs go through packed fp32x2 FMA/ADD.
-template <int HALF>
-__device__ __forceinline__ float softmax_half_exp(const float (&s)[HALF], float sl2, float m, uint32_t p_taddr) {
-  static_assert(HALF == 32 || HALF == 64, "half row of 32 or 64 columns");
-  const uint64_t scale2 = ptx::f32x2(sl2, sl2);
-  const uint64_t negm2 = ptx::f32x2(-m, -m);
-  uint64_t acc0 = ptx::f32x2(0.f, 0.f), acc1 = acc0;
-  constexpr int W = HALF / 2;  // packed cells
-  uint32_t pk[32];
+// The exp pass over 32 columns of a row: P = bf16(2^(s*sl2 - m)) packed in
+// pairs (even column in the low half), the fp32 sums into acc0 / acc1.
+__device__ __forceinline__ void exp_chunk32(const float* s, uint64_t scale2, uint64_t negm2, uint32_t (&pk)[16],
+                                            uint64_t& acc0, uint64_t& acc1) {
 #pragma unroll
-  for (int e = 0; e < W; ++e) {
+  for (int e = 0; e < 16; ++e) {
     float x0, x1;
     ptx::f32x2_split(ptx::fma_f32x2(ptx::f32x2(s[2 * e], s[2 * e + 1]), scale2, negm2), x0, x1);
     const float p0 = ptx::ex2(x0);
@@ -151,54 +149,51 @@ __device__ __forceinline__ float softmax_half_exp(const float (&s)[HALF], float 
       acc0 = ptx::add_f32x2(acc0, ptx::f32x2(p0, p1));
     pk[e] = ptx::pack_bf16x2(p0, p1);
   }
-  // thread t's cells go to column half t/16 of the tile's P cells
-  if constexpr (W == 32) {
-    ptx::tmem_st16x2_32<HALF / 2>(p_taddr, pk);
-  } else {
-    ptx::tmem_st16x2_16<HALF / 2>(p_taddr, pk);
-  }
-  float a0, a1, b0, b1;
-  ptx::f32x2_split(acc0, a0, a1);
-  ptx::f32x2_split(acc1, b0, b1);
-  return (a0 + b0) + (a1 + b1);
 }
 
-// One work item's key-block list.
+// Key-block list of one slot of a pair.
 template <bool SPARSE>
-struct ItemList {
-  int n = 0;
-  const int32_t* list = nullptr;
-  int nkb = 0;
+struct SlotList {
+  int n = 0;                      // blocks to walk (clamped count)
+  int qi = 0;                     // query block
+  const int32_t* list = nullptr;  // sparse mode
   __device__ __forceinline__ int raw(int jj) const {
     if constexpr (SPARSE) return list[jj];
     else return jj;
   }
-  // clamped for addressing: a bad entry (reported by the producer) reads block 0
-  __device__ __forceinline__ int block(int jj) const {
-    const int j = raw(jj);
-    return (j >= 0 && j < nkb) ? j : 0;
-  }
 };
 
-// kv_count of work item w (row h*nqb + i of the [H, nqb] count array); every
-// role reads the next item's count one item ahead, off its critical path
+// Raw kv_count of the two query blocks of pair w (0 for a query block past
+// nqb); every role reads the next pair's counts one pair ahead.
 template <bool SPARSE>
-__device__ __forceinline__ int raw_count(const AttnArgs& a, int w) {
-  if constexpr (SPARSE) return w < a.H * a.nqb ? a.kv_count[w] : 0;
-  else return a.nkb;
+__device__ __forceinline__ int2 pair_raw_counts(const AttnArgs& a, int w, int npairs_h) {
+  int2 c = make_int2(0, 0);
+  if (w >= a.H * npairs_h) return c;
+  const int h = w / npairs_h, p = w - h * npairs_h;
+  const int q0 = 2 * p, q1 = 2 * p + 1;
+  if constexpr (SPARSE) {
+    c.x = a.kv_count[h * a.nqb + q0];
+    c.y = q1 < a.nqb ? a.kv_count[h * a.nqb + q1] : 0;
+  } else {
+    c.x = a.nkb;
+    c.y = q1 < a.nqb ? a.nkb : 0;
+  }
+  return c;
 }
 
 template <bool SPARSE>
-__device__ __forceinline__ ItemList<SPARSE> item_list(const AttnArgs& a, int w, int n_raw) {
-  ItemList<SPARSE> it;
-  it.nkb = a.nkb;
-  it.n = a.nkb;
+__device__ __forceinline__ SlotList<SPARSE> slot_list(const AttnArgs& a, int h, int qi, int n_raw) {
+  SlotList<SPARSE> s;
+  s.qi = qi;
+  if (qi >= a.nqb) return s;
   if constexpr (SPARSE) {
     const int cap = a.kv_stride < a.nkb ? a.kv_stride : a.nkb;
-    it.n = n_raw < 0 ? 0 : (n_raw > cap ? cap : n_raw);  // a bad count is reported by the producer
-    it.list = a.kv_idx + static_cast<long>(w) * a.kv_stride;
+    s.n = n_raw < 0 ? 0 : (n_raw > cap ? cap : n_raw);  // a bad count is reported by the producer
+    s.list = a.kv_idx + (static_cast<long>(h) * a.nqb + qi) * a.kv_stride;
+  } else {
+    s.n = a.nkb;
   }
-  return it;
+  return s;
 }
 
 template <int D, int BK, bool SPARSE, bool MASS = false>
@@ -206,7 +201,7 @@ __global__ void __launch_bounds__(384, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const AttnArgs a) {
   using C = AttnCfg<D, BK>;
-  constexpr int HALF = C::HALF;
+  constexpr int NST = C::NST;
   static_assert(!(MASS && SPARSE), "the block mass comes from a full pass");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -214,28 +209,26 @@ __global__ void __launch_bounds__(384, 1)
   const uint32_t sb = ptx::smem_u32(smem);
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int n_items = a.H * a.nqb;
+  const int npairs_h = (a.nqb + 1) >> 1;
+  const int n_pairs = a.H * npairs_h;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
   auto bar = [&](int idx) -> uint32_t { return sb + C::OFF_BAR + 8 * idx; };
 
   // ---- setup
   if (threadIdx.x == 0) {
-    ptx::mbar_init(bar(C::B_QFULL), 1);
-    ptx::mbar_init(bar(C::B_QEMPTY), 1);
-    for (int s = 0; s < C::KS; ++s) {
-      ptx::mbar_init(bar(C::B_KFULL + s), 1);
-      ptx::mbar_init(bar(C::B_KEMPTY + s), 1);
+    for (int s = 0; s < 2; ++s) {
+      ptx::mbar_init(bar(C::B_QFULL + s), 1);
+      ptx::mbar_init(bar(C::B_QEMPTY + s), 1);
+      ptx::mbar_init(bar(C::B_SFULL + s), 1);
+      for (int q = 0; q < C::NPV; ++q)
+        ptx::mbar_init(bar(C::B_PFULL + s * C::NPV + q), 4);  // one arrival per softmax warp of the slot
+      ptx::mbar_init(bar(C::B_PVDONE + s), 1);
+      ptx::mbar_init(bar(C::B_DRAIN + s), 1);
     }
-    for (int s = 0; s < C::VS; ++s) {
-      ptx::mbar_init(bar(C::B_VFULL + s), 1);
-      ptx::mbar_init(bar(C::B_VEMPTY + s), 1);
-    }
-    for (int b = 0; b < 2; ++b) {
-      ptx::mbar_init(bar(C::B_SFULL + b), 1);
-      ptx::mbar_init(bar(C::B_PFULL + b), 8);  // one arrival per softmax warp
-      ptx::mbar_init(bar(C::B_PVDONE + b), 1);
-      ptx::mbar_init(bar(C::B_DRAIN + b), 1);
+    for (int s = 0; s < NST; ++s) {
+      ptx::mbar_init(bar(C::B_FULL + s), 1);
+      ptx::mbar_init(bar(C::B_EMPTY + s), 2);  // two commits per tile
     }
     *abort_flag = 0;
     ptx::fence_mbar_init();
@@ -251,189 +244,245 @@ __global__ void __launch_bounds__(384, 1)
 
   if (warp >= 8) {
     setmaxnreg_dec_56();
-    if (warp == 8 && lane == 0) {
+    const uint32_t leader = ptx::elect_one();
+    auto wait = [&](int idx, int parity) -> bool {
+      return ptx::mbar_wait_warp(bar(idx), parity & 1, abort_flag, a.timeout_ns, kErrTimeout);
+    };
+    if (warp == 8) {
       // ============================================================ producer
-      ptx::tma_prefetch_desc(&tm_q);
-      ptx::tma_prefetch_desc(&tm_k);
-      ptx::tma_prefetch_desc(&tm_v);
-      int g = 0, iq = 0;  // tile counter, Q tiles loaded so far
-      int issued_k = 0, issued_v = 0;
+      // warp-uniform; one elected lane issues the copies
+      if (leader) {
+        ptx::tma_prefetch_desc(&tm_q);
+        ptx::tma_prefetch_desc(&tm_k);
+        ptx::tma_prefetch_desc(&tm_v);
+      }
+      int seq = 0;               // ring tiles issued
+      int qn0 = 0, qn1 = 0;      // Q tiles issued per slot
       bool ok = true;
-      int n_raw = raw_count<SPARSE>(a, blockIdx.x), n_raw_next = 0;
-      for (int w = blockIdx.x; ok && w < n_items; w += gridDim.x, n_raw = n_raw_next) {
-        n_raw_next = raw_count<SPARSE>(a, w + gridDim.x);
-        const int h = w / a.nqb, qi = w - h * a.nqb;
-        const ItemList<SPARSE> it = item_list<SPARSE>(a, w, n_raw);
-        if (SPARSE && n_raw != it.n) ptx::record_error(kErrBadPattern);
-        if (it.n == 0) continue;
-        // Q of this item once every S MMA of the previous item is complete
-        if (iq > 0 && !ptx::mbar_wait(bar(C::B_QEMPTY), (iq - 1) & 1, abort_flag, a.timeout_ns, kErrTimeout)) {
-          ok = false;
-          break;
-        }
-        ptx::mbar_arrive_expect_tx(bar(C::B_QFULL), C::Q_BYTES);
+      int h = 0;
+      // one K or V tile of key block blk into the next ring stage
+      auto load_tile = [&](const CUtensorMap* tm, int blk) -> bool {
+        const int st = seq % NST;
+        if (seq >= NST && !wait(C::B_EMPTY + st, (seq / NST) - 1)) return false;
+        ptx::mbar_arrive_expect_tx_if(leader, bar(C::B_FULL + st), C::KV_BYTES);
 #pragma unroll
         for (int c = 0; c < C::DCH; ++c)
-          ptx::tma_load_3d(sb + C::OFF_Q + c * C::Q_CHUNK, &tm_q, bar(C::B_QFULL), c * 64, qi * a.bq, h);
-        ++iq;
-        // list entries are read one tile ahead, off the copy-issue path
-        int prev = -1, raw_next = it.raw(0);
-        for (int jj = 0; jj < it.n; ++jj, ++g) {
-          const int raw = raw_next;
-          if (jj + 1 < it.n) raw_next = it.raw(jj + 1);
+          ptx::tma_load_3d_if(leader, sb + C::OFF_RING + st * C::KV_BYTES + c * C::KV_CHUNK, tm, bar(C::B_FULL + st),
+                              c * 64, blk * BK, h);
+        ++seq;
+        return true;
+      };
+      auto load_q = [&](int s, int qi) -> bool {
+        const int qn = s ? qn1 : qn0;
+        if (qn > 0 && !wait(C::B_QEMPTY + s, qn - 1)) return false;
+        ptx::mbar_arrive_expect_tx_if(leader, bar(C::B_QFULL + s), C::Q_BYTES);
+#pragma unroll
+        for (int c = 0; c < C::DCH; ++c)
+          ptx::tma_load_3d_if(leader, sb + (s ? C::OFF_Q1 : C::OFF_Q0) + c * C::Q_CHUNK, &tm_q, bar(C::B_QFULL + s),
+                              c * 64, qi * a.bq, h);
+        if (s) ++qn1;
+        else ++qn0;
+        return true;
+      };
+      // a list entry, validated (out of range or not ascending is reported and
+      // read as block 0)
+      auto checked = [&](int raw, int& prev) -> int {
+        if constexpr (SPARSE) {
+          if (leader && (raw < 0 || raw >= a.nkb || raw <= prev)) ptx::record_error(kErrBadPattern);
+          prev = raw;
+        }
+        return (raw >= 0 && raw < a.nkb) ? raw : 0;
+      };
+      int2 cnt = pair_raw_counts<SPARSE>(a, blockIdx.x, npairs_h), cnt_next;
+      for (int w = blockIdx.x; ok && w < n_pairs; w += gridDim.x, cnt = cnt_next) {
+        cnt_next = pair_raw_counts<SPARSE>(a, w + gridDim.x, npairs_h);
+        h = w / npairs_h;
+        const int p = w - h * npairs_h;
+        const SlotList<SPARSE> l0 = slot_list<SPARSE>(a, h, 2 * p, cnt.x);
+        const SlotList<SPARSE> l1 = slot_list<SPARSE>(a, h, 2 * p + 1, cnt.y);
+        if (SPARSE && leader && (cnt.x != l0.n || (2 * p + 1 < a.nqb && cnt.y != l1.n)))
+          ptx::record_error(kErrBadPattern);
+        if (l0.n == 0 && l1.n == 0) continue;
+        // the next pair's Q rows into L2 while this pair runs
+        if (leader && w + static_cast<int>(gridDim.x) < n_pairs) {
+          const int wn = w + gridDim.x, hn = wn / npairs_h, pn = wn - hn * npairs_h;
+#pragma unroll
+          for (int c = 0; c < C::DCH; ++c) {
+            ptx::tma_prefetch_3d(&tm_q, c * 64, 2 * pn * a.bq, hn);
+            if (2 * pn + 1 < a.nqb) ptx::tma_prefetch_3d(&tm_q, c * 64, (2 * pn + 1) * a.bq, hn);
+          }
+        }
+        const int n = l0.n > l1.n ? l0.n : l1.n;
+        int prev0 = -1, prev1 = -1;
+        int raw0 = l0.n > 0 ? l0.raw(0) : 0, raw1 = l1.n > 0 ? l1.raw(0) : 0;
+        for (int j = 0; ok && j < n; ++j) {
+          const bool a0 = j < l0.n, a1 = j < l1.n;
+          // list entries one tile ahead, off the copy-issue path
+          const int r0 = raw0, r1 = raw1;
+          if (j + 1 < l0.n) raw0 = l0.raw(j + 1);
+          if (j + 1 < l1.n) raw1 = l1.raw(j + 1);
           if constexpr (SPARSE) {
-            if (raw < 0 || raw >= a.nkb || raw <= prev) ptx::record_error(kErrBadPattern);
-            prev = raw;
+            const int j0 = a0 ? checked(r0, prev0) : 0;
+            const int j1 = a1 ? checked(r1, prev1) : 0;
+            if (a0 && j == 0) ok = load_q(0, l0.qi);
+            if (ok && a0) ok = load_tile(&tm_k, j0);
+            if (ok && a1 && j == 0) ok = load_q(1, l1.qi);
+            if (ok && a1) ok = load_tile(&tm_k, j1);
+            if (ok && a0) ok = load_tile(&tm_v, j0);
+            if (ok && a1) ok = load_tile(&tm_v, j1);
+          } else {
+            if (j == 0) ok = load_q(0, l0.qi);
+            if (ok) ok = load_tile(&tm_k, j);
+            if (ok && a1 && j == 0) ok = load_q(1, l1.qi);
+            if (ok) ok = load_tile(&tm_v, j);
           }
-          const int j = (raw >= 0 && raw < a.nkb) ? raw : 0;
-          const int ks = g % C::KS;
-          if (g >= C::KS &&
-              !ptx::mbar_wait(bar(C::B_KEMPTY + ks), (g / C::KS - 1) & 1, abort_flag, a.timeout_ns, kErrTimeout)) {
-            ok = false;
-            break;
-          }
-          ptx::mbar_arrive_expect_tx(bar(C::B_KFULL + ks), C::KV_BYTES);
-#pragma unroll
-          for (int c = 0; c < C::DCH; ++c)
-            ptx::tma_load_3d(sb + C::OFF_K + ks * C::KV_BYTES + c * C::KV_CHUNK, &tm_k, bar(C::B_KFULL + ks),
-                             c * 64, j * BK, h);
-          issued_k = g + 1;
-          const int vs = g % C::VS;
-          if (g >= C::VS &&
-              !ptx::mbar_wait(bar(C::B_VEMPTY + vs), (g / C::VS - 1) & 1, abort_flag, a.timeout_ns, kErrTimeout)) {
-            ok = false;
-            break;
-          }
-          ptx::mbar_arrive_expect_tx(bar(C::B_VFULL + vs), C::KV_BYTES);
-#pragma unroll
-          for (int c = 0; c < C::DCH; ++c)
-            ptx::tma_load_3d(sb + C::OFF_V + vs * C::KV_BYTES + c * C::KV_CHUNK, &tm_v, bar(C::B_VFULL + vs),
-                             c * 64, j * BK, h);
-          issued_v = g + 1;
         }
       }
       if (!ok) {
         // let the copies in flight land before the CTA's shared memory goes
-        // away: the last Q and the last KS / VS tiles
+        // away: the last Q of each slot and the last NST tiles
         const uint64_t short_ns = a.timeout_ns / 4;
         volatile int dummy = 0;
-        if (iq > 0) ptx::mbar_wait(bar(C::B_QFULL), (iq - 1) & 1, &dummy, short_ns, 0);
-        for (int u = (issued_k > C::KS ? issued_k - C::KS : 0); u < issued_k; ++u)
-          ptx::mbar_wait(bar(C::B_KFULL + u % C::KS), (u / C::KS) & 1, &dummy, short_ns, 0);
-        for (int u = (issued_v > C::VS ? issued_v - C::VS : 0); u < issued_v; ++u)
-          ptx::mbar_wait(bar(C::B_VFULL + u % C::VS), (u / C::VS) & 1, &dummy, short_ns, 0);
+        if (qn0 > 0) ptx::mbar_wait(bar(C::B_QFULL + 0), (qn0 - 1) & 1, &dummy, short_ns, 0);
+        if (qn1 > 0) ptx::mbar_wait(bar(C::B_QFULL + 1), (qn1 - 1) & 1, &dummy, short_ns, 0);
+        for (int u = (seq > NST ? seq - NST : 0); u < seq; ++u)
+          ptx::mbar_wait(bar(C::B_FULL + u % NST), (u / NST) & 1, &dummy, short_ns, 0);
+        __syncwarp();
       }
-    } else if (warp == 9 && lane == 0) {
-      // ============================================================ S issuer
+    } else if (warp == 9 || warp == 10) {
+      // ============================================================ MMA issuers
+      // Warp 9 issues slot 0's MMAs, warp 10 slot 1's, so neither slot's chain
+      // (S(t) -> softmax -> PV(t) -> S(t+1)) waits on the other's softmax. The
+      // whole warp runs the loop (warp-uniform control flow, descriptors in
+      // uniform registers); one elected lane issues the MMAs and commits. A
+      // ring stage gets two commits in all (EMPTY counts two): one from each
+      // slot reading a shared dense tile, else two from the slot that owns it.
+      const int s = warp - 9;
       constexpr uint32_t HI = ptx::sdesc_sw128_hi(1024);
-      const uint32_t qlo = ptx::sdesc_sw128_lo(sb + C::OFF_Q, 16);
-      const uint32_t klo = ptx::sdesc_sw128_lo(sb + C::OFF_K, 16);
-      int g = 0, iq = 0;
+      const uint32_t q_lo = ptx::sdesc_sw128_lo(sb + (s ? C::OFF_Q1 : C::OFF_Q0), 16);
+      const uint32_t k_lo = ptx::sdesc_sw128_lo(sb + C::OFF_RING, 16);
+      const uint32_t v_lo = ptx::sdesc_sw128_lo(sb + C::OFF_RING, C::KV_CHUNK);
+      const uint32_t s_tmem = tmem + (s ? C::TM_S1 : C::TM_S0);
+      const uint32_t o_tmem = tmem + (s ? C::TM_O1 : C::TM_O0);
+      constexpr int KPP = BK / 16 / C::NPV;  // PV MMAs per part of P
+      int seq = 0;      // ring tiles (same numbering as the producer)
+      int qn = 0;       // Q tiles consumed
+      int tcnt = 0;     // tiles of this slot (PFULL phases)
       bool ok = true;
-      int n_raw = raw_count<SPARSE>(a, blockIdx.x), n_raw_next = 0;
-      for (int w = blockIdx.x; ok && w < n_items; w += gridDim.x, n_raw = n_raw_next) {
-        n_raw_next = raw_count<SPARSE>(a, w + gridDim.x);
-        const ItemList<SPARSE> it = item_list<SPARSE>(a, w, n_raw);
-        if (it.n == 0) continue;
-        if (!ptx::mbar_wait(bar(C::B_QFULL), iq & 1, abort_flag, a.timeout_ns, kErrTimeout)) {
-          ok = false;
-          break;
-        }
-        for (int jj = 0; jj < it.n; ++jj, ++g) {
-          const int b = g & 1;
-          const int ks = g % C::KS;
-          if (!ptx::mbar_wait(bar(C::B_KFULL + ks), (g / C::KS) & 1, abort_flag, a.timeout_ns, kErrTimeout) ||
-              (g >= 2 &&
-               !ptx::mbar_wait(bar(C::B_PVDONE + b), ((g - 2) >> 1) & 1, abort_flag, a.timeout_ns, kErrTimeout))) {
+      auto commit = [&](int idx) { ptx::umma_commit_if(leader, bar(idx)); };
+      int2 cnt = pair_raw_counts<SPARSE>(a, blockIdx.x, npairs_h), cnt_next;
+      for (int w = blockIdx.x; ok && w < n_pairs; w += gridDim.x, cnt = cnt_next) {
+        cnt_next = pair_raw_counts<SPARSE>(a, w + gridDim.x, npairs_h);
+        const int h = w / npairs_h;
+        const int p = w - h * npairs_h;
+        const int n0 = slot_list<SPARSE>(a, h, 2 * p, cnt.x).n;
+        const int n1 = slot_list<SPARSE>(a, h, 2 * p + 1, cnt.y).n;
+        const int n = n0 > n1 ? n0 : n1;
+        const int nm = s ? n1 : n0;
+        for (int j = 0; j < n; ++j) {
+          const bool a0 = j < n0, a1 = j < n1;
+          int sk, sv;
+          bool sole;  // the tile's two EMPTY commits both come from this slot
+          if constexpr (SPARSE) {
+            const int base = seq;
+            seq += (a0 ? 2 : 0) + (a1 ? 2 : 0);
+            sk = s ? base + (a0 ? 1 : 0) : base;
+            sv = sk + (a0 ? 1 : 0) + (a1 ? 1 : 0);
+            sole = true;
+          } else {
+            sk = seq;
+            sv = seq + 1;
+            seq += 2;
+            sole = !a1;
+          }
+          if (j >= nm) continue;
+          if ((j == 0 && !wait(C::B_QFULL + s, qn++)) || !wait(C::B_FULL + sk % NST, sk / NST)) {
             ok = false;
             break;
           }
           ptx::tc_fence_after();
-          const uint32_t b0 = klo + static_cast<uint32_t>(ks * C::KV_BYTES >> 4);
-          const uint32_t s_tmem = tmem + (b ? C::TM_S1 : C::TM_S0);
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t ao = (kk >> 2) * (C::Q_CHUNK >> 4) + (kk & 3) * 2;
-            const uint32_t bo = (kk >> 2) * (C::KV_CHUNK >> 4) + (kk & 3) * 2;
-            ptx::umma_ss_lohi(s_tmem, qlo + ao, b0 + bo, HI, C::IDESC_S, kk > 0 ? 1u : 0u);
+            constexpr uint32_t QC = C::Q_CHUNK >> 4, KC = C::KV_CHUNK >> 4;
+            const uint32_t ao = (kk >> 2) * QC + (kk & 3) * 2;
+            const uint32_t bo = (kk >> 2) * KC + (kk & 3) * 2;
+            ptx::umma_ss_lohi_if(leader, s_tmem, q_lo + ao,
+                                 k_lo + static_cast<uint32_t>((sk % NST) * C::KV_BYTES >> 4) + bo, HI, C::IDESC_S,
+                                 kk > 0 ? 1u : 0u);
           }
-          ptx::umma_commit(bar(C::B_SFULL + b));
-          ptx::umma_commit(bar(C::B_KEMPTY + ks));
-        }
-        if (!ok) break;
-        // every S MMA of this item read Q: the producer may refill it
-        ptx::umma_commit(bar(C::B_QEMPTY));
-        ++iq;
-      }
-      if (!ok) {
-        ptx::umma_commit(bar(C::B_DRAIN));
-        volatile int dummy = 0;
-        ptx::mbar_wait(bar(C::B_DRAIN), 0, &dummy, a.timeout_ns / 4, 0);
-      }
-    } else if (warp == 10 && lane == 0) {
-      // ============================================================ PV issuer
-      constexpr uint32_t HI = ptx::sdesc_sw128_hi(1024);
-      const uint32_t vlo = ptx::sdesc_sw128_lo(sb + C::OFF_V, C::KV_CHUNK);
-      int g = 0;
-      bool ok = true;
-      int n_raw = raw_count<SPARSE>(a, blockIdx.x), n_raw_next = 0;
-      for (int w = blockIdx.x; ok && w < n_items; w += gridDim.x, n_raw = n_raw_next) {
-        n_raw_next = raw_count<SPARSE>(a, w + gridDim.x);
-        const ItemList<SPARSE> it = item_list<SPARSE>(a, w, n_raw);
-        for (int jj = 0; jj < it.n; ++jj, ++g) {
-          const int b = g & 1;
-          const int vs = g % C::VS;
-          if (!ptx::mbar_wait(bar(C::B_PFULL + b), (g >> 1) & 1, abort_flag, a.timeout_ns, kErrTimeout) ||
-              !ptx::mbar_wait(bar(C::B_VFULL + vs), (g / C::VS) & 1, abort_flag, a.timeout_ns, kErrTimeout)) {
+          commit(C::B_SFULL + s);
+          commit(C::B_EMPTY + sk % NST);
+          if (sole) commit(C::B_EMPTY + sk % NST);
+          if (j == nm - 1) commit(C::B_QEMPTY + s);
+          // O += P V in NPV parts, each issued as soon as the softmax has
+          // stored that part of P
+          if (!wait(C::B_FULL + sv % NST, sv / NST)) {
             ok = false;
             break;
           }
-          ptx::tc_fence_after();
-          const uint32_t b0 = vlo + static_cast<uint32_t>(vs * C::KV_BYTES >> 4);
-          const uint32_t p_tmem = tmem + (b ? C::TM_P1 : C::TM_P0);
+          const uint32_t vb = v_lo + static_cast<uint32_t>((sv % NST) * C::KV_BYTES >> 4);
 #pragma unroll
-          for (int kk = 0; kk < BK / 16; ++kk)
-            ptx::umma_ts_lohi(tmem + C::TM_O, p_tmem + kk * 8, b0 + kk * (2048 >> 4), HI, C::IDESC_PV,
-                              (jj > 0 || kk > 0) ? 1u : 0u);
-          ptx::umma_commit(bar(C::B_VEMPTY + vs));
-          ptx::umma_commit(bar(C::B_PVDONE + b));
+          for (int q = 0; q < C::NPV; ++q) {
+            if (!wait(C::B_PFULL + s * C::NPV + q, tcnt)) {
+              ok = false;
+              break;
+            }
+            ptx::tc_fence_after();
+#pragma unroll
+            for (int u = 0; u < KPP; ++u) {
+              const int kk = q * KPP + u;
+              ptx::umma_ts_lohi_if(leader, o_tmem, s_tmem + kk * 8, vb + kk * (2048 >> 4), HI, C::IDESC_PV,
+                                   (j > 0 || kk > 0) ? 1u : 0u);
+            }
+          }
+          if (!ok) break;
+          commit(C::B_PVDONE + s);
+          commit(C::B_EMPTY + sv % NST);
+          if (sole) commit(C::B_EMPTY + sv % NST);
+          ++tcnt;
         }
       }
       if (!ok) {
-        ptx::umma_commit(bar(C::B_DRAIN + 1));
+        commit(C::B_DRAIN + s);
         volatile int dummy = 0;
-        ptx::mbar_wait(bar(C::B_DRAIN + 1), 0, &dummy, a.timeout_ns / 4, 0);
+        ptx::mbar_wait(bar(C::B_DRAIN + s), 0, &dummy, a.timeout_ns / 4, 0);
+        __syncwarp();
       }
     }
   } else {
     // ================================================================ softmax
     setmaxnreg_inc_224();
-    const int half = lane >> 4;                                        // column half of my row
-    const int r = (warp & 3) * 32 + (warp >> 2) * 16 + (lane & 15);  // row == TMEM lane
-    const uint32_t lane_base = tmem + (static_cast<uint32_t>((warp & 3) * 32 + (warp >> 2) * 16) << 16);
+    const int slot = warp >> 2;
+    const int wq = warp & 3;
+    const int r = wq * 32 + lane;  // row == TMEM lane
+    const uint32_t lane_base = tmem + (static_cast<uint32_t>(wq * 32) << 16);
+    const uint32_t s_col = slot ? C::TM_S1 : C::TM_S0;
+    const uint32_t o_col = slot ? C::TM_O1 : C::TM_O0;
     const float sl2 = a.scale_log2;
-    const int s_off = half * HALF;  // first S column of my half row
-    int g = 0;
+    const uint64_t scale2 = ptx::f32x2(sl2, sl2);
+    int tcount = 0;  // tiles of this slot so far (SFULL / PVDONE phases)
     bool ok = true;
-    int n_raw = raw_count<SPARSE>(a, blockIdx.x), n_raw_next = 0;
-    for (int w = blockIdx.x; ok && w < n_items; w += gridDim.x, n_raw = n_raw_next) {
-      n_raw_next = raw_count<SPARSE>(a, w + gridDim.x);
-      const int h = w / a.nqb, qi = w - h * a.nqb;
-      const ItemList<SPARSE> it = item_list<SPARSE>(a, w, n_raw);
+    int2 cnt = pair_raw_counts<SPARSE>(a, blockIdx.x, npairs_h), cnt_next;
+    for (int w = blockIdx.x; ok && w < n_pairs; w += gridDim.x, cnt = cnt_next) {
+      cnt_next = pair_raw_counts<SPARSE>(a, w + gridDim.x, npairs_h);
+      const int h = w / npairs_h;
+      const int p = w - h * npairs_h;
+      const int qi = 2 * p + slot;
+      if (qi >= a.nqb) continue;
+      const SlotList<SPARSE> it = slot_list<SPARSE>(a, h, qi, slot ? cnt.y : cnt.x);
       const int grow = qi * a.bq + r;
       const bool row_valid = (r < a.bq) && (grow < a.L);
-      // my contiguous half row of O: D/2 bf16 = D bytes
-      uint4* o_dst = reinterpret_cast<uint4*>(a.o + (static_cast<long>(h) * a.L + grow) * D) + half * (D / 16);
+      uint4* o_dst = reinterpret_cast<uint4*>(a.o + (static_cast<long>(h) * a.L + grow) * D);
       if (it.n == 0) {
         if (row_valid) {
 #pragma unroll
-          for (int c = 0; c < D / 16; ++c) o_dst[c] = make_uint4(0, 0, 0, 0);
-          if (half == 0) a.lse[static_cast<long>(h) * a.L + grow] = -__int_as_float(0x7f800000);
+          for (int c = 0; c < D / 8; ++c) o_dst[c] = make_uint4(0, 0, 0, 0);
+          a.lse[static_cast<long>(h) * a.L + grow] = -__int_as_float(0x7f800000);
         }
         continue;
       }
       float m = -__int_as_float(0x7f800000);  // running row max, log2 units (scaled)
-      float l = 0.f;                          // running sum of my half row
+      float l = 0.f;                          // running row sum
       // MASS: my row's LSE (log2 units) from the earlier full pass
       float lse2_prev = 0.f;
       if constexpr (MASS)
@@ -441,105 +490,123 @@ __global__ void __launch_bounds__(384, 1)
       // only a list that can hold the ragged last key block needs its entries
       // here; they are read one tile ahead, off the critical path
       const bool ragged = SPARSE && (a.Lk % BK) != 0;
-      int blk_next = ragged ? it.block(0) : 0;
-      for (int jj = 0; jj < it.n; ++jj, ++g) {
+      int blk_next = 0;
+      if (ragged) {
+        const int b0 = it.raw(0);
+        blk_next = (b0 >= 0 && b0 < a.nkb) ? b0 : 0;
+      }
+      for (int jj = 0; jj < it.n; ++jj, ++tcount) {
         int blk = jj;
         if (ragged) {
           blk = blk_next;
-          if (jj + 1 < it.n) blk_next = it.block(jj + 1);
+          if (jj + 1 < it.n) {
+            const int bn = it.raw(jj + 1);
+            blk_next = (bn >= 0 && bn < a.nkb) ? bn : 0;
+          }
         }
-        const int b = g & 1;
-        if (!ptx::mbar_wait_warp(bar(C::B_SFULL + b), (g >> 1) & 1, abort_flag, a.timeout_ns, kErrTimeout)) {
+        if (!ptx::mbar_wait_warp(bar(C::B_SFULL + slot), tcount & 1, abort_flag, a.timeout_ns, kErrTimeout)) {
           ok = false;
           break;
         }
         ptx::tc_fence_after();
-        float s[HALF];
+        float s[BK];
         {
-          uint32_t raw[HALF / 32][32];
+          uint32_t raw[BK / 32][32];
 #pragma unroll
-          for (int c = 0; c < HALF / 32; ++c)
-            ptx::tmem_ld16x2_32<HALF>(lane_base + (b ? C::TM_S1 : C::TM_S0) + c * 32, raw[c]);
+          for (int c = 0; c < BK / 32; ++c) ptx::tmem_ld32(lane_base + s_col + c * 32, raw[c]);
           ptx::tmem_wait_ld();
 #pragma unroll
-          for (int c = 0; c < HALF / 32; ++c) {
+          for (int c = 0; c < BK / 32; ++c) {
             ptx::reg_fence32(raw[c]);
 #pragma unroll
             for (int e = 0; e < 32; ++e) s[c * 32 + e] = __uint_as_float(raw[c][e]);
           }
         }
-        // ragged last key block: keys past L do not exist
-        const int valid = a.Lk - blk * BK - s_off;
-        if (valid < HALF) {
+        // ragged last key block: keys past Lk do not exist
+        const int valid = a.Lk - blk * BK;
+        if (valid < BK) {
 #pragma unroll
-          for (int c = 0; c < HALF; ++c)
+          for (int c = 0; c < BK; ++c)
             if (c >= valid) s[c] = -__int_as_float(0x7f800000);
         }
-        float mx0 = s[0], mx1 = s[1];
+        float mx0 = s[0], mx1 = s[1], mx2 = s[2], mx3 = s[3];
 #pragma unroll
-        for (int c = 2; c < HALF; c += 4) {
+        for (int c = 4; c < BK; c += 8) {
           mx0 = ptx::max3(mx0, s[c], s[c + 1]);
-          if (c + 3 < HALF) mx1 = ptx::max3(mx1, s[c + 2], s[c + 3]);
+          mx1 = ptx::max3(mx1, s[c + 2], s[c + 3]);
+          if (c + 4 < BK) {
+            mx2 = ptx::max3(mx2, s[c + 4], s[c + 5]);
+            mx3 = ptx::max3(mx3, s[c + 6], s[c + 7]);
+          }
         }
-        float mx = fmaxf(mx0, mx1);
-        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));  // the other half of my row
+        const float mx = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3));
         const float m_new = fmaxf(m, mx * sl2);
         if (jj == 0) {
           m = m_new;
         } else if (__any_sync(0xffffffffu, m_new > m + 8.0f)) {
-          // O holds this item's tiles before g-1 plus PV(g-1): wait for it,
-          // rescale my half
-          if (!ptx::mbar_wait_warp(bar(C::B_PVDONE + ((g - 1) & 1)), ((g - 1) >> 1) & 1, abort_flag,
-                                   a.timeout_ns, kErrTimeout)) {
-            ok = false;
-            break;
-          }
-          ptx::tc_fence_after();
+          // O_s holds every earlier tile of this item (S_s(t) was issued after
+          // PV_s(t-1)): rescale my row
           const float alpha = ptx::ex2(m - m_new);
 #pragma unroll
-          for (int c = 0; c < D / 64; ++c) {
+          for (int c = 0; c < D / 32; ++c) {
             uint32_t raw[32];
-            ptx::tmem_ld16x2_32<D / 2>(lane_base + C::TM_O + c * 32, raw);
+            ptx::tmem_ld32(lane_base + o_col + c * 32, raw);
             ptx::tmem_wait_ld();
             ptx::reg_fence32(raw);
 #pragma unroll
             for (int e = 0; e < 32; ++e) raw[e] = __float_as_uint(__uint_as_float(raw[e]) * alpha);
-            ptx::tmem_st16x2_32<D / 2>(lane_base + C::TM_O + c * 32, raw);
+            ptx::tmem_st32(lane_base + o_col + c * 32, raw);
           }
-          ptx::tmem_wait_st();
           l *= alpha;
           m = m_new;
         }
-        // P_b is free: S_b(g) was issued only after PV(g-2) completed
-        const float ps = softmax_half_exp<HALF>(s, sl2, m, lane_base + (b ? C::TM_P1 : C::TM_P0));
+        // P_s over the first BK/2 columns of S_s (read out above)
+        const uint64_t negm2 = ptx::f32x2(-m, -m);
+        uint64_t acc0 = ptx::f32x2(0.f, 0.f), acc1 = acc0;
+        constexpr int CPP = BK / 32 / C::NPV;  // 32-column chunks per part of P
+#pragma unroll
+        for (int c = 0; c < BK / 32; ++c) {
+          uint32_t pk[16];
+          exp_chunk32(s + 32 * c, scale2, negm2, pk, acc0, acc1);
+          ptx::tmem_st32_16(lane_base + s_col + c * 16, pk);
+          if ((c + 1) % CPP == 0 && c + 1 < BK / 32) {
+            // this part of P is in TMEM: its PV MMAs may start
+            ptx::tmem_wait_st();
+            ptx::tc_fence_before();
+            __syncwarp();
+            if (lane == 0) ptx::mbar_arrive(bar(C::B_PFULL + slot * C::NPV + c / CPP));
+          }
+        }
+        float a0, a1, b0, b1;
+        ptx::f32x2_split(acc0, a0, a1);
+        ptx::f32x2_split(acc1, b0, b1);
+        const float ps = (a0 + b0) + (a1 + b1);
         l += ps;
         if constexpr (MASS) {
-          // this tile's probability mass of my half row is ps * 2^(m - lse2);
-          // the warp's 16 rows x 2 halves summed by a fixed shuffle tree
-          float c = row_valid ? ps * ptx::ex2(m - lse2_prev) : 0.f;
+          // this tile's probability mass of my row is ps * 2^(m - lse2); the
+          // warp's 32 rows summed by a fixed shuffle tree
+          float cm = row_valid ? ps * ptx::ex2(m - lse2_prev) : 0.f;
 #pragma unroll
-          for (int off = 16; off > 0; off >>= 1) c += __shfl_xor_sync(0xffffffffu, c, off);
-          if (lane == 0) a.mass_part[((static_cast<long>(h) * a.nqb + qi) * a.nkb + jj) * 8 + warp] = c;
+          for (int off = 16; off > 0; off >>= 1) cm += __shfl_xor_sync(0xffffffffu, cm, off);
+          if (lane == 0) a.mass_part[((static_cast<long>(h) * a.nqb + qi) * a.nkb + jj) * kMassParts + wq] = cm;
         }
         ptx::tmem_wait_st();
         ptx::tc_fence_before();
         __syncwarp();
-        if (lane == 0) ptx::mbar_arrive(bar(C::B_PFULL + b));
+        if (lane == 0) ptx::mbar_arrive(bar(C::B_PFULL + slot * C::NPV + C::NPV - 1));
       }
       if (!ok) break;
       // ---- epilogue: every PV of the item is done -> O / l -> bf16 -> global; LSE
-      if (!ptx::mbar_wait_warp(bar(C::B_PVDONE + ((g - 1) & 1)), ((g - 1) >> 1) & 1, abort_flag, a.timeout_ns,
-                               kErrTimeout)) {
+      if (!ptx::mbar_wait_warp(bar(C::B_PVDONE + slot), (tcount - 1) & 1, abort_flag, a.timeout_ns, kErrTimeout)) {
         ok = false;
         break;
       }
       ptx::tc_fence_after();
-      const float lt = l + __shfl_xor_sync(0xffffffffu, l, 16);
-      const float inv_l = 1.0f / lt;
+      const float inv_l = 1.0f / l;
 #pragma unroll
-      for (int c = 0; c < D / 64; ++c) {
+      for (int c = 0; c < D / 32; ++c) {
         uint32_t raw[32];
-        ptx::tmem_ld16x2_32<D / 2>(lane_base + C::TM_O + c * 32, raw);
+        ptx::tmem_ld32(lane_base + o_col + c * 32, raw);
         ptx::tmem_wait_ld();
         ptx::reg_fence32(raw);
         uint32_t pk[16];
@@ -552,9 +619,8 @@ __global__ void __launch_bounds__(384, 1)
             o_dst[c * 4 + u] = make_uint4(pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
         }
       }
-      if (row_valid && half == 0)
-        a.lse[static_cast<long>(h) * a.L + grow] = (m + ptx::lg2(lt)) * 0.69314718055994530942f;
-      // the next item's first PV overwrites O only after this warp's next
+      if (row_valid) a.lse[static_cast<long>(h) * a.L + grow] = (m + ptx::lg2(l)) * 0.69314718055994530942f;
+      // the next item's first PV overwrites O_s only after this warp's next
       // PFULL arrival, which follows the loads above (tcgen05.wait::ld)
     }
   }

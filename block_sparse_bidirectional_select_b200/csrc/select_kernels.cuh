@@ -215,14 +215,14 @@ __global__ void __launch_bounds__(256, 1)
 // ---------------------------------------------------------------- fused mass
 
 // Block mass from the partial sums the attention kernel's MASS variant wrote
-// during its full pass: mass[e] = sum of the 8 softmax warps' partials of tile
+// during its full pass: mass[e] = sum of the 4 softmax warps' partials of tile
 // e = (h, i, j), in a fixed order.
 __global__ void __launch_bounds__(256)
     mass_from_parts_kernel(const float4* __restrict__ part, long n, float* __restrict__ mass) {
   const long e = static_cast<long>(blockIdx.x) * blockDim.x + threadIdx.x;
   if (e >= n) return;
-  const float4 a = part[2 * e], b = part[2 * e + 1];
-  mass[e] = ((a.x + a.y) + (a.z + a.w)) + ((b.x + b.y) + (b.z + b.w));
+  const float4 a = part[e];
+  mass[e] = (a.x + a.y) + (a.z + a.w);
 }
 
 // ---------------------------------------------------------------- top-k

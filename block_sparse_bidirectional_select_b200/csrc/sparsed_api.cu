@@ -64,6 +64,34 @@ int get_encoder() {
   return SPARSED_OK;
 }
 
+// Process-unique id of the CUDA context current on this thread (0 when none
+// is current yet). Device-side addresses and library-owned streams belong to
+// a context: caches of them are keyed on this id, so that a context created
+// after cudaDeviceReset never sees the handles of the one before.
+PFN_cuCtxGetCurrent_v4000 g_ctx_current = nullptr;
+PFN_cuCtxGetId_v12000 g_ctx_id = nullptr;
+std::once_flag g_ctx_once;
+
+int context_id(unsigned long long* id) {
+  std::call_once(g_ctx_once, [] {
+    cudaDriverEntryPointQueryResult q;
+    void* fn = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &fn, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      g_ctx_current = reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(fn);
+    fn = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &fn, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      g_ctx_id = reinterpret_cast<PFN_cuCtxGetId_v12000>(fn);
+  });
+  if (!g_ctx_current || !g_ctx_id) return fail_cuda(cudaErrorSymbolNotFound);
+  CUcontext ctx = nullptr;
+  if (g_ctx_current(&ctx) != CUDA_SUCCESS) return fail_cuda(cudaErrorContextIsDestroyed);
+  *id = 0;
+  if (ctx && g_ctx_id(ctx, id) != CUDA_SUCCESS) return fail_cuda(cudaErrorContextIsDestroyed);
+  return SPARSED_OK;
+}
+
 int require_sm100() {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
@@ -171,7 +199,7 @@ int launch_attn_t(const Problem& p, const int32_t* kv_idx, const int32_t* kv_cou
     SP_CUDA(cudaFuncGetAttributes(&fa, kern));
     regs = fa.numRegs;
   }
-  if (regs * C::THREADS < C::REGS_SOFTMAX * 256 + C::REGS_OTHER * 128) return SPARSED_ERR_UNSUPPORTED;
+  if (regs * C::THREADS < C::REGS_SOFTMAX * 256 + C::REGS_OTHER * (C::THREADS - 256)) return SPARSED_ERR_UNSUPPORTED;
   CUtensorMap tq, tk, tv;
   SP_TRY(make_map(&tq, p.Q, p.H, p.L, D, 128));
   SP_TRY(make_map(&tk, p.K, p.H, p.Lk, D, BK));
@@ -195,10 +223,10 @@ int launch_attn_t(const Problem& p, const int32_t* kv_idx, const int32_t* kv_cou
   int sms = 0;
   SP_TRY(sm_count(&sms));
   SP_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES));
-  // persistent: one CTA per SM (shared memory admits one), each walking items
-  // blockIdx.x, blockIdx.x + gridDim.x, ...
-  const long items = static_cast<long>(p.H) * p.nqb;
-  const int grid = static_cast<int>(items < sms ? items : sms);
+  // persistent: one CTA per SM (its registers admit one), each walking the
+  // pairs of query blocks blockIdx.x, blockIdx.x + gridDim.x, ...
+  const long pairs = static_cast<long>(p.H) * ((p.nqb + 1) / 2);
+  const int grid = static_cast<int>(pairs < sms ? pairs : sms);
   kern<<<grid, C::THREADS, C::SMEM_BYTES, st>>>(tq, tk, tv, a);
   SP_CUDA(cudaGetLastError());
   return SPARSED_OK;
@@ -398,7 +426,7 @@ struct FusedWorkspace {
 FusedWorkspace fused_ws_layout(int H, int L, int nqb, int nkb) {
   FusedWorkspace f;
   f.part = ws_layout(H, nqb, nkb).total;
-  f.lse_prev = f.part + align256(static_cast<size_t>(H) * nqb * nkb * 8 * sizeof(float));
+  f.lse_prev = f.part + align256(static_cast<size_t>(H) * nqb * nkb * kMassParts * sizeof(float));
   f.total = f.lse_prev + align256(static_cast<size_t>(H) * L * sizeof(float));
   return f;
 }
@@ -641,7 +669,7 @@ int sparsed_run_steps_span(const uint16_t* Q, const uint16_t* K, const uint16_t*
   // fused selection when the workspace has room for it (see the header)
   const bool fused = any_select && workspace &&
                      workspace_bytes >= fused_ws_layout(p.H, p.L, p.nqb, p.nkb).total &&
-                     static_cast<long long>(p.H) * p.nqb * p.nkb * 8 < (1ll << 31);
+                     static_cast<long long>(p.H) * p.nqb * p.nkb * kMassParts < (1ll << 31);
   bool have_lse = false;  // a full pass of this call left its LSE in the workspace
   std::vector<cudaEvent_t> ev;
   if (step_ms && start_step < end_step) {
@@ -893,24 +921,34 @@ static __device__ __align__(256) unsigned char g_noalloc_scratch[SPARSED_NOALLOC
 namespace {
 
 constexpr int kNoAllocMaxDevices = 64;
+struct NoAllocAddr {
+  unsigned long long ctx = 0;  // context id (0: slot unused)
+  void* addr = nullptr;
+};
 std::mutex g_noalloc_mu;
-void* g_noalloc_addr[kNoAllocMaxDevices] = {};
+NoAllocAddr g_noalloc_addr[kNoAllocMaxDevices];
 
-// Device address of g_noalloc_scratch on the current device. In host code the
-// array's name is only a host-side stand-in, so the address is resolved with
-// cudaGetSymbolAddress once per device (the first call on that device) and
-// cached.
+// Device address of g_noalloc_scratch in the current device's context. In
+// host code the array's name is only a host-side stand-in, so the address is
+// looked up with cudaGetSymbolAddress, once per context (the first call on a
+// device, with that device current), and cached under the context's id: a
+// context created after cudaDeviceReset gets its own lookup.
 int noalloc_scratch_address(void** out) {
   int dev = 0;
   SP_CUDA(cudaGetDevice(&dev));
   if (dev < 0 || dev >= kNoAllocMaxDevices) return SPARSED_ERR_UNSUPPORTED;
+  unsigned long long ctx = 0;
+  SP_TRY(context_id(&ctx));
   std::lock_guard<std::mutex> lock(g_noalloc_mu);
-  if (g_noalloc_addr[dev] == nullptr) {
+  NoAllocAddr& slot = g_noalloc_addr[dev];
+  if (ctx == 0 || slot.ctx != ctx) {
     void* addr = nullptr;
-    SP_CUDA(cudaGetSymbolAddress(&addr, g_noalloc_scratch));
-    g_noalloc_addr[dev] = addr;
+    SP_CUDA(cudaGetSymbolAddress(&addr, g_noalloc_scratch));  // makes the primary context current if none was
+    SP_TRY(context_id(&ctx));
+    slot.ctx = ctx;
+    slot.addr = addr;
   }
-  *out = g_noalloc_addr[dev];
+  *out = slot.addr;
   return SPARSED_OK;
 }
 
@@ -1018,6 +1056,7 @@ LosaWorkspace losa_ws_layout(const LosaDims& g) {
 // takes both branches). Created at the first use on a device; the lock keeps
 // the fork / join of concurrent callers apart.
 struct SideStream {
+  unsigned long long ctx = 0;  // id of the context the handles belong to
   cudaStream_t s = nullptr;
   cudaEvent_t fork = nullptr, join = nullptr;
   std::mutex mu;
@@ -1032,6 +1071,11 @@ int side_stream(SideStream** out) {
   if (dev < 0 || dev >= kSideMaxDevices) return SPARSED_ERR_UNSUPPORTED;
   std::lock_guard<std::mutex> lock(g_side_init_mu);
   SideStream& ss = g_side[dev];
+  unsigned long long ctx = 0;
+  SP_TRY(context_id(&ctx));
+  // handles created in a context that has since gone (cudaDeviceReset) are
+  // not valid any more: make new ones in the current context
+  if (ss.s != nullptr && (ctx == 0 || ss.ctx != ctx)) ss.s = nullptr;
   if (ss.s == nullptr) {
     // all three or none: a failed creation leaves the slot empty for a retry
     cudaStream_t s = nullptr;
@@ -1045,12 +1089,37 @@ int side_stream(SideStream** out) {
       if (s) cudaStreamDestroy(s);
       return fail_cuda(e);
     }
+    SP_TRY(context_id(&ctx));
+    ss.ctx = ctx;
     ss.fork = fork;
     ss.join = join;
     ss.s = s;
   }
   *out = &ss;
   return SPARSED_OK;
+}
+
+// Fork: the side stream waits for everything issued on st so far. Nothing is
+// forked when this fails.
+int fork_side(SideStream* side, cudaStream_t st) {
+  SP_CUDA(cudaEventRecord(side->fork, st));
+  SP_CUDA(cudaStreamWaitEvent(side->s, side->fork, 0));
+  return SPARSED_OK;
+}
+
+int record_join(SideStream* side) {
+  SP_CUDA(cudaEventRecord(side->join, side->s));
+  return SPARSED_OK;
+}
+
+// Any failure after a fork: record the join on the side stream (best effort;
+// it may already be recorded) and make st wait for it, so the caller's stream
+// stays ordered after the side work and a stream capture of st never ends
+// with the side stream left unjoined. Returns rc.
+int rejoin_after_error(SideStream* side, cudaStream_t st, int rc) {
+  cudaEventRecord(side->join, side->s);
+  cudaStreamWaitEvent(st, side->join, 0);
+  return rc;
 }
 
 int losa_check_ws(const LosaDims& g, const void* workspace, size_t ws_bytes) {
@@ -1218,17 +1287,13 @@ int losa_init_impl(const LosaDims& g, const uint16_t* Q, const uint16_t* K, cons
   SP_TRY(side_stream(&side));
   {
     std::lock_guard<std::mutex> lock(side->mu);
-    SP_CUDA(cudaEventRecord(side->fork, st));
-    SP_CUDA(cudaStreamWaitEvent(side->s, side->fork, 0));
-    SP_TRY(losa_suffix(g, Q, K, V, scale, O, LSE, side->s));
-    SP_CUDA(cudaEventRecord(side->join, side->s));
-    int rc = losa_lists(g, nullptr, nullptr, sel_stride, Q, nullptr, nullptr, ws, st);
+    SP_TRY(fork_side(side, st));
+    int rc = losa_suffix(g, Q, K, V, scale, O, LSE, side->s);
+    if (rc == SPARSED_OK) rc = record_join(side);
+    if (rc == SPARSED_OK) rc = losa_lists(g, nullptr, nullptr, sel_stride, Q, nullptr, nullptr, ws, st);
     if (rc == SPARSED_OK)
       rc = losa_prefix_and_merge(g, Kp, Vp, scale, true, o_cache, lse_cache, O, LSE, ws, st, side->join);
-    if (rc != SPARSED_OK) {
-      cudaStreamWaitEvent(st, side->join, 0);  // the caller's stream stays ordered after the suffix
-      return rc;
-    }
+    if (rc != SPARSED_OK) return rejoin_after_error(side, st, rc);
   }
   float* mass = token_mass ? token_mass : reinterpret_cast<float*>(ws + w.mass);
   SP_TRY(launch_tok_mass(g, Q, Kp, scale, lse_cache, mass, st));
@@ -1252,17 +1317,18 @@ int losa_step_impl(const LosaDims& g, const uint16_t* Q, const uint16_t* K, cons
   SideStream* side = nullptr;
   SP_TRY(side_stream(&side));
   std::lock_guard<std::mutex> lock(side->mu);
-  SP_CUDA(cudaEventRecord(side->fork, st));
-  SP_CUDA(cudaStreamWaitEvent(side->s, side->fork, 0));
-  SP_TRY(losa_suffix(g, Q, K, V, scale, O, LSE, side->s));
-  SP_CUDA(cudaEventRecord(side->join, side->s));
-  query_mse_kernel<<<g.B, 256, 0, st>>>(Q, Q_prev, g.H, g.B, g.d, static_cast<double>(tau), act);
-  const cudaError_t e = cudaGetLastError();
-  int rc = e == cudaSuccess ? SPARSED_OK : fail_cuda(e);
+  SP_TRY(fork_side(side, st));
+  int rc = losa_suffix(g, Q, K, V, scale, O, LSE, side->s);
+  if (rc == SPARSED_OK) rc = record_join(side);
+  if (rc == SPARSED_OK) {
+    query_mse_kernel<<<g.B, 256, 0, st>>>(Q, Q_prev, g.H, g.B, g.d, static_cast<double>(tau), act);
+    const cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) rc = fail_cuda(e);
+  }
   if (rc == SPARSED_OK) rc = losa_lists(g, act, sel, sel_stride, Q, union_idx, union_count, ws, st);
   if (rc == SPARSED_OK)
     rc = losa_prefix_and_merge(g, Kp, Vp, scale, false, o_cache, lse_cache, O, LSE, ws, st, side->join);
-  if (rc != SPARSED_OK) cudaStreamWaitEvent(st, side->join, 0);  // the caller's stream stays ordered after the suffix
+  if (rc != SPARSED_OK) return rejoin_after_error(side, st, rc);
   return rc;
 }
 
@@ -1280,7 +1346,7 @@ int sparsed_losa_splits(int H, int B, int bq, int P, int bk, int sm_count, int* 
   if (!splits || H < 1 || B < 1 || P < 1 || sm_count < 1) return SPARSED_ERR_INVALID_ARG;
   if ((bq != 64 && bq != 128) || (bk != 64 && bk != 128)) return SPARSED_ERR_UNSUPPORTED;
   const long per_split = static_cast<long>(H) * cdiv(B, bq);  // work items of one split
-  long s = sm_count / per_split;
+  long s = 2L * sm_count / per_split;  // the attention kernel runs two work items per SM
   if (s < 1) s = 1;
   long s_max = cdiv(cdiv(P, bk), kLosaMinChunk);
   if (s_max > kLosaMaxSplits) s_max = kLosaMaxSplits;
@@ -1322,6 +1388,10 @@ int sparsed_losa_step(const uint16_t* Q, const uint16_t* K, const uint16_t* V, c
   SP_TRY(losa_check_ptrs(Q, K, V, K_prefix, V_prefix, o_cache, lse_cache, sel, O, LSE));
   if (!Q_prev || !aligned16(Q_prev)) return SPARSED_ERR_INVALID_ARG;
   if (!std::isfinite(tau) || tau < 0.f) return SPARSED_ERR_INVALID_ARG;
+  // the optional int32 outputs are stored by the kernels as int32
+  for (const int32_t* ptr : {static_cast<const int32_t*>(active), static_cast<const int32_t*>(union_idx),
+                             static_cast<const int32_t*>(union_count)})
+    if (ptr && (reinterpret_cast<uintptr_t>(ptr) & 3u)) return SPARSED_ERR_INVALID_ARG;
   SP_TRY(losa_check_ws(g, workspace, workspace_bytes));
   SP_TRY(require_sm100());
   SP_TRY(get_encoder());

@@ -160,7 +160,7 @@ int sparsed_select_pattern(const uint16_t* Q, const uint16_t* K, const uint16_t*
 
 /* Workspace bytes with which sparsed_run_steps fuses the block mass into
  * the full pass of its SELECT steps: sparsed_workspace_bytes plus the
- * per-warp mass partials [H, nqb, nkb, 8] fp32 and one [H, L] fp32 LSE copy,
+ * per-warp mass partials [H, nqb, nkb, 4] fp32 and one [H, L] fp32 LSE copy,
  * every part 256-byte aligned. */
 int sparsed_run_steps_workspace_bytes(int H, int L, int bq, int bk, size_t* bytes);
 
@@ -331,8 +331,10 @@ int sparsed_run_steps_columns(const uint16_t* Q, const uint16_t* K, const uint16
  *     (sparsed_workspace_bytes(H, L, bq, bk) > SPARSED_NOALLOC_SCRATCH_BYTES;
  *     e.g. H=32, L=32768, bq=bk=128 fits, L=65536 does not).
  *   - The first call on each device looks up the array's device address
- *     (cudaGetSymbolAddress) with that device current and caches it; make that
- *     first call before any stream capture.
+ *     (cudaGetSymbolAddress) with that device current and caches it under the
+ *     device's CUDA context (a context created after cudaDeviceReset gets a
+ *     fresh lookup on its first call); make that first call before any stream
+ *     capture.
  *   - Every call on a device shares the one array, which keeps the previous
  *     call's contents; each call overwrites all scratch it reads, so nothing
  *     needs clearing. Calls that overlap on the GPU race on the array: issue
@@ -397,8 +399,9 @@ int sparsed_select_pattern_noalloc(const uint16_t* Q, const uint16_t* K, const u
  * outside a graph capture (it creates that stream and its two events). */
 
 /* Splits for a step of these sizes on a GPU with sm_count SMs: as many as
- * keep one split's H*ceil(B/bq) work items per SM at most
- * (floor(sm_count / (H*ceil(B/bq))), at least 1, at most min(32, ceil(nkb/4))). */
+ * keep two work items per SM at most (the attention kernel runs two query
+ * tiles per SM), one split having H*ceil(B/bq) work items
+ * (floor(2*sm_count / (H*ceil(B/bq))), at least 1, at most min(32, ceil(nkb/4))). */
 int sparsed_losa_splits(int H, int B, int bq, int P, int bk, int sm_count, int* splits);
 
 /* Workspace bytes of sparsed_losa_init / _step / _block for these sizes:

@@ -170,9 +170,9 @@ def _losa_splits(H=32, B=64, bq=64, P_=32768, bk=64, sms=148):
 
 
 def test_losa_splits():
-    assert _losa_splits() == (_lib.OK, 4)                      # 148 SMs / 32 work items per split
-    assert _losa_splits(B=128) == (_lib.OK, 2)                 # two query tiles per split
-    assert _losa_splits(H=200) == (_lib.OK, 1)                 # at least one split
+    assert _losa_splits() == (_lib.OK, 9)                      # 2 x 148 work items / 32 per split
+    assert _losa_splits(B=128) == (_lib.OK, 4)                 # two query tiles per split
+    assert _losa_splits(H=400) == (_lib.OK, 1)                 # at least one split
     assert _losa_splits(H=1, P_=100) == (_lib.OK, 1)           # at most ceil(nkb / 4): nkb = 2
     assert _losa_splits(H=1, P_=64 * 40) == (_lib.OK, 10)      # nkb = 40 -> at most 10
     assert _losa_splits(H=1, P_=64 * 1000) == (_lib.OK, 32)    # never more than 32
@@ -201,9 +201,10 @@ def test_losa_workspace_bytes():
     assert _losa_ws(P_=64 * 32768 + 1, H=1, d=64)[0] == _lib.ERR_UNSUPPORTED  # nkb > 32768
 
 
-def _losa_step(tau=0.01, ws=P, ws_bytes=1 << 30, qprev=P, sel=P, n_sel=2, B=64):
+def _losa_step(tau=0.01, ws=P, ws_bytes=1 << 30, qprev=P, sel=P, n_sel=2, B=64, active=None, uidx=None,
+               ucount=None):
     return lib.sparsed_losa_step(P, P, P, qprev, P, P, 2, B, 4096, 128, 0.088, 64, 64, n_sel, tau, 2,
-                                 P, P, sel, P, P, None, None, None, ws, ws_bytes, None)
+                                 P, P, sel, P, P, active, uidx, ucount, ws, ws_bytes, None)
 
 
 def test_losa_step_validation():
@@ -216,8 +217,15 @@ def test_losa_step_validation():
     assert _losa_step(ws=None) == _lib.ERR_WORKSPACE
     assert _losa_step(ws_bytes=4096) == _lib.ERR_WORKSPACE
     assert _losa_step(B=2000) == _lib.ERR_UNSUPPORTED
+    # the optional int32 outputs must be 4-byte aligned
+    odd = ctypes.c_void_p(0x10002)
+    assert _losa_step(active=odd) == _lib.ERR_INVALID_ARG
+    assert _losa_step(uidx=odd) == _lib.ERR_INVALID_ARG
+    assert _losa_step(ucount=odd) == _lib.ERR_INVALID_ARG
     if not GPU:
         assert _losa_step() == _lib.ERR_NO_DEVICE
+        assert _losa_step(active=P, uidx=ctypes.c_void_p(0x10004), ucount=ctypes.c_void_p(0x10008)) == \
+            _lib.ERR_NO_DEVICE
 
 
 def test_losa_block_validation():
