@@ -379,19 +379,10 @@ __host__ __device__ inline void allocate_budget(const double* E, int H, int nkb,
       mark[best] = 1.0;
       --rem;
     }
-    while (rem < 0) {  // only reachable through fp64 rounding of the quotas
-      int best = -1;
-      double bf = 2.0;
-      for (int h = 0; h < H; ++h) {
-        if (quota[h] < 0.0 || mark[h] != 0.0 || extra[h] <= 0.0) continue;
-        const double f = quota[h] - floor(quota[h]);
-        if (f <= bf) { bf = f; best = h; }
-      }
-      if (best < 0) break;
-      extra[best] -= 1.0;
-      mark[best] = 1.0;
-      ++rem;
-    }
+    // (the floors never sum above Xf: quotas that sum to Xf up to a few ulps
+    // can cross an integer from below only with fractional parts within an
+    // ulp of 1, and one crossing more than the fractional parts add up to is
+    // impossible, so rem >= 0)
     break;
   }
   for (int h = 0; h < H; ++h) head_k[h] = 1 + static_cast<int32_t>(extra[h]);

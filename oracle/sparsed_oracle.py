@@ -177,7 +177,14 @@ def head_entropy(M):
 def largest_remainder(total, weights):
     """Split integer ``total`` in proportion to ``weights``: floor of each quota,
     then one more unit to the largest fractional parts (ties: lower position).
-    All-zero weights split evenly by the same rule."""
+    All-zero weights split evenly by the same rule.
+
+    The floors never sum above ``total``: the quotas sum to ``total`` up to a
+    relative error of a few ulps, so the fractional parts sum to an integer m
+    (up to that error), and a computed quota can cross an integer from below
+    only when its exact fractional part is within an ulp of 1; m + 1 such
+    crossings would need fractional parts summing to about m + 1 > m. The
+    remainder is therefore never negative (asserted)."""
     w = [float(x) for x in weights]
     sw = sum(w)
     if sw <= 0.0:
@@ -186,17 +193,10 @@ def largest_remainder(total, weights):
     quota = [total * x / sw for x in w]
     base = [math.floor(x) for x in quota]
     rem = total - sum(base)
-    if rem >= 0:
-        order = sorted(range(len(w)), key=lambda a: (-(quota[a] - base[a]), a))
-        for a in order[:rem]:
-            base[a] += 1
-    else:
-        # only reachable when fp64 rounding pushes a quota across an integer:
-        # take units back from the smallest fractions (ties: higher position)
-        order = sorted((a for a in range(len(w)) if base[a] > 0),
-                       key=lambda a: (quota[a] - base[a], -a))
-        for a in order[:-rem]:
-            base[a] -= 1
+    assert rem >= 0, "floors of the quotas exceed the total"
+    order = sorted(range(len(w)), key=lambda a: (-(quota[a] - base[a]), a))
+    for a in order[:rem]:
+        base[a] += 1
     return base, quota
 
 

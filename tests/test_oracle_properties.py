@@ -83,6 +83,34 @@ def test_entropy_budget_invariants(H, nkb, keep, ent):
 
 
 @SETTINGS
+@given(total=st.integers(0, 5000), w=st.lists(st.one_of(st.floats(0.0, 10.0), st.sampled_from([0.1, 1 / 3, 0.7, 1.0])),
+                                                min_size=1, max_size=40))
+def test_largest_remainder_against_exact_rationals(total, w):
+    """Largest remainder against the same split in exact rational arithmetic
+    (fractions.Fraction of the same fp64 weights): every head gets the floor
+    or the ceiling of its exact quota, the shares sum to the total, and where
+    the exact fractional parts at the cut are separated the two agree."""
+    from fractions import Fraction
+    base, quota = O.largest_remainder(total, w)
+    wf = [Fraction(x) for x in w]
+    if sum(wf) == 0:
+        wf = [Fraction(1)] * len(w)
+    qf = [total * x / sum(wf) for x in wf]
+    fl = [math.floor(x) for x in qf]
+    rem = total - sum(fl)
+    assert sum(base) == total
+    assert all(b in (f, f + 1) for b, f in zip(base, fl))
+    order = sorted(range(len(w)), key=lambda a: (-(qf[a] - fl[a]), a))
+    fr = sorted((qf[a] - fl[a] for a in range(len(w))), reverse=True)
+    separated = rem == 0 or rem == len(w) or fr[rem - 1] - fr[rem] > Fraction(1, 10 ** 9)
+    if separated and all(abs(Fraction(q) - x) < Fraction(1, 10 ** 6) for q, x in zip(quota, qf)):
+        exact = list(fl)
+        for a in order[:rem]:
+            exact[a] += 1
+        assert base == exact, (total, w)
+
+
+@SETTINGS
 @given(seed=st.integers(0, 2 ** 31 - 1), n=st.integers(1, 40), k=st.integers(1, 40), levels=st.integers(1, 6))
 def test_topk_blocks_is_the_head_of_the_order(seed, n, k, levels):
     rng = np.random.default_rng(seed)
