@@ -13,8 +13,11 @@ a sparse step (the block-mass pass of a selecting step is overhead, not counted)
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
-With N > 1 (launched by torchrun) every rank runs its own independent layer
-(weak scaling, no data-path collective); the time is the max over ranks.
+With N > 1 (launched by torchrun) the layer's heads are split evenly over the
+ranks (strong scaling): a uniform budget needs no exchange, an entropy budget
+all-gathers the H per-head entropies at each selecting step (NCCL). The time
+is the max over ranks and the value the whole layer's flops over that time.
+(--path losa runs an independent block per rank.)
 --impl reference times the fp64 CPU oracle on this host's cores on a bounded
 sample of the same workload (rank 0 only).
 """
@@ -200,9 +203,14 @@ def cpu_oracle_sample(wl, q, k, v, budget_s, rng_seed=0):
 
 # ----------------------------------------------------------------- ranks
 
-def rank_workload(wl, rank):
-    """Each rank runs its own independent layer: same shapes, its own seed."""
-    return wl.scaled(seed=wl.seed + rank)
+def head_range(H, world, rank):
+    """The heads [h0, h1) of the layer this rank holds: the layer's heads split
+    evenly over the ranks in rank order (every head's work is independent; an
+    entropy budget only exchanges the per-head entropies)."""
+    if H % world:
+        raise SystemExit(f"--gpus {world} must divide the {H} heads of the layer")
+    n = H // world
+    return rank * n, (rank + 1) * n
 
 
 def reduce_max(x, world, device):
@@ -215,10 +223,21 @@ def reduce_max(x, world, device):
     return float(t.item())
 
 
-def job_value(flops_per_step, steps, world, total_ms):
-    """Whole-job throughput in TFLOP/s: every rank's steps over the slowest
-    rank's time (weak scaling: each rank does the same work)."""
-    return flops_per_step * steps * world / (total_ms * 1e-3) / 1e12
+def reduce_sum(x, world, device):
+    """Sum of a host float over all ranks (identity for one rank)."""
+    if world == 1:
+        return float(x)
+    import torch.distributed as dist
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return float(t.item())
+
+
+def job_value(layer_flops_per_step, steps, total_ms):
+    """Whole-job throughput in TFLOP/s: the layer's flops (all ranks' heads
+    together) over the slowest rank's time (strong scaling: the layer is
+    fixed, its heads split over the ranks)."""
+    return layer_flops_per_step * steps / (total_ms * 1e-3) / 1e12
 
 
 def run_reference(args, rank, world):
@@ -326,19 +345,27 @@ def main():
         return run_columns(args, wl, dev, rank, world, barrier, max_over_ranks)
     if args.path == "losa":
         return run_losa(args, dev, rank, world, barrier, max_over_ranks)
-    log(f"[rank {rank}] inputs for {wl.name}")
-    q_cpu, k_cpu, v_cpu = make_inputs(rank_workload(wl, rank))
+    h0, h1 = head_range(wl.H, world, rank)
+    log(f"[rank {rank}] inputs for {wl.name}, heads {h0}..{h1 - 1}")
+    q_cpu, k_cpu, v_cpu = (t[h0:h1].contiguous() for t in make_inputs(wl))
     q, k, v = (t.to(dev) for t in (q_cpu, k_cpu, v_cpu))
     stream = torch.cuda.current_stream()
     peaks, peak_src = load_peaks()
 
-    H, L, d = wl.H, wl.L, wl.d
-    nqb = -(-L // wl.bq)
+    H, L, d = h1 - h0, wl.L, wl.d
+    wl_local = wl.scaled(H=H)
     ws = torch.empty(sp.run_steps_workspace_bytes(H, L, wl.bq, wl.bk), dtype=torch.uint8, device=dev)
     o = torch.empty_like(q)
     lse = torch.empty((H, L), dtype=torch.float32, device=dev)
+    group = dist.group.WORLD if world > 1 else None
 
     def one_run(time_steps=False):
+        if world > 1:
+            # this rank's heads; an entropy budget all-gathers the per-head
+            # entropies at every selecting step (the loop's only exchange)
+            return sp.run_steps_sharded(q, k, v, wl.T, wl.warmup_frac, keep=wl.keep, budget=wl.budget,
+                                        refresh_every=wl.refresh_every, group=group, bq=wl.bq, bk=wl.bk,
+                                        out=o, lse=lse, workspace=ws)
         return sp.run_steps(q, k, v, wl.T, wl.warmup_frac, keep=wl.keep, budget=wl.budget,
                             refresh_every=wl.refresh_every, bq=wl.bq, bk=wl.bk, out=o, lse=lse,
                             workspace=ws, time_steps=time_steps)
@@ -349,7 +376,8 @@ def main():
     sp.device_check()
     kinds = res.kinds
     kv_sum = int(res.kv_count.sum().item())
-    acc = run_accounting(wl, kinds, kv_sum)
+    acc = run_accounting(wl_local, kinds, kv_sum)
+    layer_flops = reduce_sum(acc["flops"], world, dev)
 
     # ---------------- timed region: K full runs
     torch.cuda.synchronize()
@@ -361,8 +389,9 @@ def main():
     e_ev = torch.cuda.Event(enable_timing=True)
     s_ev.record(stream)
     for _ in range(args.steps):
-        r = one_run(time_steps=True)
-        step_ms.append(r.step_ms)
+        r = one_run(time_steps=world == 1)
+        if r.step_ms is not None:
+            step_ms.append(r.step_ms)
     e_ev.record(stream)
     e_ev.synchronize()
     torch.cuda.synchronize()
@@ -371,7 +400,7 @@ def main():
     total_ms = max_over_ranks(s_ev.elapsed_time(e_ev))
     sp.device_check()
     ms_per_step = total_ms / args.steps
-    value = job_value(acc["flops"], args.steps, world, total_ms)
+    value = job_value(layer_flops, args.steps, total_ms)
 
     per_kind = {0: [], 1: [], 2: []}
     for run in step_ms:
@@ -439,8 +468,13 @@ def main():
             qd.copy_(qh, non_blocking=True)
             kd.copy_(kh, non_blocking=True)
             vd.copy_(vh, non_blocking=True)
-            sp.run_steps(qd, kd, vd, wl.T, wl.warmup_frac, keep=wl.keep, budget=wl.budget,
-                         refresh_every=wl.refresh_every, bq=wl.bq, bk=wl.bk, out=o, lse=lse, workspace=ws)
+            if world > 1:
+                sp.run_steps_sharded(qd, kd, vd, wl.T, wl.warmup_frac, keep=wl.keep, budget=wl.budget,
+                                     refresh_every=wl.refresh_every, group=group, bq=wl.bq, bk=wl.bk, out=o,
+                                     lse=lse, workspace=ws)
+            else:
+                sp.run_steps(qd, kd, vd, wl.T, wl.warmup_frac, keep=wl.keep, budget=wl.budget,
+                             refresh_every=wl.refresh_every, bq=wl.bq, bk=wl.bk, out=o, lse=lse, workspace=ws)
             oh.copy_(o, non_blocking=True)
             lh.copy_(lse, non_blocking=True)
 
@@ -450,7 +484,7 @@ def main():
         torch.cuda.synchronize()
         bi = 3 * q.numel() * q.element_size()
         bo = o.numel() * o.element_size() + lse.numel() * lse.element_size()
-        e2e = {"value": job_value(acc["flops"], args.steps, world, e2e_ms), "unit": UNIT,
+        e2e = {"value": job_value(layer_flops, args.steps, e2e_ms), "unit": UNIT,
                "h2d_bytes_per_step": bi, "d2h_bytes_per_step": bo, "ms_per_step": e2e_ms / args.steps}
 
     cpu = None
@@ -460,14 +494,18 @@ def main():
 
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "strong",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": dict(workload_config(wl), parallelism=f"replicas x{world}" if world > 1 else "single"),
+        "config": dict(workload_config(wl), parallelism=f"heads x{world}" if world > 1 else "single",
+                       step="one complete T-step denoising run of the layer"),
         "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": acc["launches"] * args.steps,
         "clocks": clk,
         "pct_of_peak": {"value_vs_burst": value / world / peak_burst, "value_vs_sustained": value / world / peak_tc,
                         "value_vs_datasheet_dense_bf16": value / world / DATASHEET_BF16_TFLOPS,
                         "peak_source": peak_src},
+        # per GPU and per GHz of the median SM clock sampled in the timed
+        # region: the run's throughput with the power-capped clock divided out
+        "tflops_per_gpu_per_ghz": (value / world / (clk["sm_mhz"] / 1000.0)) if clk.get("sm_mhz") else None,
         "ms_per_denoise_step": ms_per_step / wl.T,
         "steps_breakdown": {"dense_ms": dense_ms, "select_ms": select_ms, "sparse_ms": sparse_ms,
                             "n_dense": acc["n_dense"], "n_select": acc["n_select"], "n_sparse": acc["n_sparse"]},
@@ -534,9 +572,10 @@ def run_columns(args, wl, dev, rank, world, barrier, max_over_ranks):
     warm-up, column selection at the switch, attention over the kept columns.
     Effective flops count 4*L*kc*d per head for a sparse step."""
     import block_sparse_bidirectional_select_b200 as sp
-    q, k, v = (t.to(dev) for t in make_inputs(rank_workload(wl, rank)))
+    h0, h1 = head_range(wl.H, world, rank)  # this rank's heads of the layer (no exchange: columns are per head)
+    q, k, v = (t[h0:h1].contiguous().to(dev) for t in make_inputs(wl))
     stream = torch.cuda.current_stream()
-    H, L, d = wl.H, wl.L, wl.d
+    H, L, d = h1 - h0, wl.L, wl.d
     kc = sp.column_keep(L, wl.keep)
     ws = torch.empty(sp.column_workspace_bytes(H, L, d, kc), dtype=torch.uint8, device=dev)
     o = torch.empty_like(q)
@@ -581,11 +620,14 @@ def run_columns(args, wl, dev, rank, world, barrier, max_over_ranks):
     ms_alone = median_time(fn, stream, 20)
     peaks, peak_src = load_peaks()
     peak_burst = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
+    layer_flops = reduce_sum(flops, world, dev)
     line = {"metric": "column-sparse attn effective TFLOP/s & ms/step at 64k", "value":
-            job_value(flops, args.steps, world, total_ms), "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            job_value(layer_flops, args.steps, total_ms), "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": dict(workload_config(wl), path="columns", kept_columns_per_head=kc),
+            "scaling": "strong", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": dict(workload_config(wl), path="columns", kept_columns_per_head=kc,
+                           parallelism=f"heads x{world}" if world > 1 else "single",
+                           step="one complete T-step denoising run of the layer"),
             "ms_per_denoise_step": total_ms / args.steps / wl.T,
             "steps_breakdown": {"dense_ms": mean(per_kind[0]), "select_ms": mean(per_kind[1]),
                                 "sparse_ms": mean(per_kind[2]), "n_dense": n_dense, "n_select": n_select,
@@ -690,7 +732,8 @@ def run_losa(args, dev, rank, world, barrier, max_over_ranks):
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
             "config": {"workload": wl.name, "H": wl.H, "prefix": wl.P, "block": wl.B, "d": wl.d, "bq": wl.bq,
                        "bk": wl.bk, "blocks_per_token": wl.n_sel, "T": wl.T, "tau": wl.tau, "splits": splits,
-                       "l2": "flushed before every timed run"},
+                       "l2": "flushed before every timed run",
+                       "parallelism": f"independent blocks x{world}" if world > 1 else "single"},
             "ms_per_denoise_step": total_ms / args.steps / wl.T,
             "first_step_ms": first_ms, "later_step_ms": step_ms,
             "active_tokens_per_step": float(n_active[1:].mean()) if wl.T > 1 else None,

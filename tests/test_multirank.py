@@ -1,8 +1,9 @@
 """Host logic of the N-GPU benchmark on CPU: two gloo ranks on 127.0.0.1.
 
-bench.py --gpus N runs N independent layers (weak scaling, no data-path
-collective); the only cross-rank steps are the timing barrier and the max of
-the ranks' times. These tests run that host logic with the gloo backend.
+bench.py --gpus N splits one layer's heads evenly over N ranks (strong
+scaling); the cross-rank steps are the timing barrier, the max of the ranks'
+times, the sum of the ranks' flops, and (entropy budget) the all-gather of the
+per-head entropies. These tests run that host logic with the gloo backend.
 """
 import os
 import socket
@@ -35,17 +36,18 @@ def _worker(rank, world, port, out):
         mine = 10.0 + 5.0 * rank
         dist.barrier()
         got = bench.reduce_max(mine, world, torch.device("cpu"))
-        # each rank's layer has its own seed, so its own inputs
-        wl = bench.rank_workload(WORKLOADS["tiny"].scaled(H=1, L=128), rank)
+        # the ranks hold disjoint heads of one layer (same seed, same inputs)
+        wl = WORKLOADS["tiny"].scaled(L=128)
+        h0, h1 = bench.head_range(wl.H, world, rank)
         q, _, _ = make_inputs(wl)
-        sums = [torch.zeros(1, dtype=torch.float64) for _ in range(world)]
-        dist.all_gather(sums, q.double().sum().reshape(1))
-        out[rank] = (got, wl.seed, [float(x) for x in sums])
+        part = q[h0:h1].double().sum()
+        total = bench.reduce_sum(float(part), world, torch.device("cpu"))
+        out[rank] = (got, (h0, h1), total, float(q.double().sum()))
     finally:
         dist.destroy_process_group()
 
 
-def test_two_gloo_ranks_take_the_max_time_and_run_distinct_layers():
+def test_two_gloo_ranks_take_the_max_time_and_split_one_layer():
     world = 2
     ctx = mp.get_context("spawn")
     with ctx.Manager() as m:
@@ -59,15 +61,19 @@ def test_two_gloo_ranks_take_the_max_time_and_run_distinct_layers():
             assert p.exitcode == 0
         res = dict(out)
     assert res[0][0] == res[1][0] == 15.0
-    assert res[0][1] != res[1][1]
-    assert res[0][2] == res[1][2] and res[0][2][0] != res[0][2][1]
+    assert res[0][1] == (0, 2) and res[1][1] == (2, 4)      # tiny has H = 4
+    assert res[0][2] == pytest.approx(res[0][3]) and res[1][2] == pytest.approx(res[1][3])
 
 
-def test_job_value_counts_every_rank_over_the_slowest_time():
+def test_job_value_is_the_layer_over_the_slowest_time():
     import bench
-    # 2 ranks x 3 steps x 1e12 flop in 1.5 s -> 4 TFLOP/s of whole-job throughput
-    assert bench.job_value(1e12, 3, 2, 1500.0) == pytest.approx(4.0)
+    # the layer's 3e12 flop per step x 2 steps in 1.5 s -> 4 TFLOP/s
+    assert bench.job_value(3e12, 2, 1500.0) == pytest.approx(4.0)
     assert bench.reduce_max(7.5, 1, torch.device("cpu")) == 7.5
+    assert bench.reduce_sum(7.5, 1, torch.device("cpu")) == 7.5
+    assert bench.head_range(32, 8, 3) == (12, 16)
+    with pytest.raises(SystemExit):
+        bench.head_range(32, 3, 0)
 
 
 def test_reference_arm_runs_on_rank_zero_only(capsys):

@@ -187,3 +187,67 @@ def test_sharded_denoising_loop_two_shards_in_two_threads():
         o_ref, l_ref = O.masked_attention(qh[h], kh[h], vh[h], wl.scale, lists, cnt[h], 128, 128)
         assert np.abs(full.o[h].float().cpu().numpy() - o_ref).max() <= 2e-2
         assert np.abs(full.lse[h].cpu().numpy() - l_ref).max() <= 1e-3
+
+
+def _gpu_shard_worker(rank, world, port, out):
+    """One rank of a two-process head-sharded loop on cuda:0: its half of the
+    heads, the per-head entropies all-gathered over a gloo group on the host
+    (no kernel of one process waits on the other's)."""
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    sys.path.insert(0, ROOT)
+    import datetime
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=120))
+    try:
+        import block_sparse_bidirectional_select_b200 as spw
+        from block_sparse_bidirectional_select_b200.inputs import WORKLOADS, make_inputs
+        torch.cuda.set_device(0)
+        wl = WORKLOADS["tiny"].scaled(H=4, L=1024, d=128, bq=128, bk=128, seed=505, structure="band")
+        q, k, v = make_inputs(wl)
+        sl = slice(2 * rank, 2 * rank + 2)
+        qs, ks, vs = (t[sl].contiguous().cuda() for t in (q, k, v))
+        res = spw.run_steps_sharded(qs, ks, vs, 8, 0.3, 0.2, "entropy", 2, group=dist.group.WORLD)
+        torch.cuda.synchronize()
+        spw.device_check()
+        out[rank] = (res.kinds, res.kv_idx.cpu().numpy(), res.kv_count.cpu().numpy(),
+                     res.o.view(torch.int16).cpu().numpy(), res.lse.cpu().numpy())
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.gpu
+def test_sharded_denoising_loop_two_processes_gloo():
+    """Two processes on one GPU, a gloo group between them, each running the
+    head-sharded loop (entropy budget, anchors) on its half of the heads: each
+    rank's heads equal the unsharded loop's bit for bit."""
+    from block_sparse_bidirectional_select_b200.inputs import WORKLOADS, make_inputs
+    world = 2
+    ctx = mp.get_context("spawn")
+    with ctx.Manager() as m:
+        out = m.dict()
+        port = _free_port()
+        procs = [ctx.Process(target=_gpu_shard_worker, args=(r, world, port, out)) for r in range(world)]
+        for p in procs:
+            p.start()
+        for p in procs:
+            p.join(300)
+            assert p.exitcode == 0
+        res = dict(out)
+    wl = WORKLOADS["tiny"].scaled(H=4, L=1024, d=128, bq=128, bk=128, seed=505, structure="band")
+    q, k, v = (t.cuda() for t in make_inputs(wl))
+    full = sp.run_steps_sharded(q, k, v, 8, 0.3, 0.2, "entropy", 2)
+    sp.device_check()
+    assert full.kinds.count(sp.STEP_SELECT) == 3
+    idx, cnt = full.kv_idx.cpu().numpy(), full.kv_count.cpu().numpy()
+    o16, lse = full.o.view(torch.int16).cpu().numpy(), full.lse.cpu().numpy()
+    for rank in range(world):
+        kinds, r_idx, r_cnt, r_o16, r_lse = res[rank]
+        sl = slice(2 * rank, 2 * rank + 2)
+        assert kinds == full.kinds
+        assert (r_cnt == cnt[sl]).all()
+        for h in range(2):
+            for i in range(r_cnt.shape[1]):
+                c = int(r_cnt[h, i])
+                assert (r_idx[h, i, :c] == idx[sl][h, i, :c]).all()
+        assert (r_o16 == o16[sl]).all()
+        assert (r_lse == lse[sl]).all()
