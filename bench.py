@@ -426,7 +426,7 @@ def main():
                 "units_per_launch": units, "traffic": traffic.get(kernel)}
 
     dense_name = f"attn_fwd_kernel<{d},{wl.bk},dense>"
-    sparse_name = f"attn_fwd_kernel<{d},{wl.bk},sparse>"
+    sparse_name = f"attn_list_kernel<{d},{wl.bk}>"
     roof_dense = roof(dense_name, d_ach, f"{H}x{L}x{L} score tiles, 4*H*L^2*d flops")
     roof_sparse = roof(sparse_name, s_ach, f"{kv_sum} kept blocks, 4*bq*bk*d flops each")
     roofline = roof_dense if dominant == "dense" else roof_sparse
@@ -765,20 +765,29 @@ def code_signature(src):
     return "\n".join(lines)
 
 
+def kernel_signature():
+    """sha256 of the two attention kernels' code (comments and blank lines
+    removed): the dense two-tile kernel and the block-sparse one-tile kernel."""
+    import hashlib
+    csrc = os.path.join(ROOT, "block_sparse_bidirectional_select_b200", "csrc")
+    parts = []
+    for name in ("attn_kernel.cuh", "attn_list_kernel.cuh"):
+        with open(os.path.join(csrc, name)) as f:
+            parts.append(code_signature(f.read()))
+    return hashlib.sha256("\n".join(parts).encode()).hexdigest()
+
+
 def load_traffic(workload):
     """DRAM bytes per launch from the committed ncu capture (profiles/traffic.json),
-    used only while the attention kernel source is the one that was captured."""
-    import hashlib
+    used only while the attention kernels' source is the one that was captured."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
-    src = os.path.join(ROOT, "block_sparse_bidirectional_select_b200", "csrc", "attn_kernel.cuh")
     try:
         with open(path) as f:
             t = json.load(f)
-        with open(src) as f:
-            sha = hashlib.sha256(code_signature(f.read()).encode()).hexdigest()
+        sha = kernel_signature()
     except (OSError, ValueError):
         return {}
-    if t.get("attn_kernel_sha256") != sha:
+    if t.get("attn_kernels_sha256") != sha:
         return {}
     return t.get(workload, {})
 

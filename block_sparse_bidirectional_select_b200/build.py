@@ -12,7 +12,7 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libsparsed.so")
 SOURCES = ["sparsed_api.cu"]
-DEPS = ["sparsed_api.cu", "attn_kernel.cuh", "select_kernels.cuh", "column_kernels.cuh", "losa_kernels.cuh",
+DEPS = ["sparsed_api.cu", "attn_kernel.cuh", "attn_list_kernel.cuh", "select_kernels.cuh", "column_kernels.cuh", "losa_kernels.cuh",
         "ptx_sm100.cuh"]
 
 

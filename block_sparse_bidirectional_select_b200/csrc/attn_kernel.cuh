@@ -1,24 +1,21 @@
-// Flash-style bidirectional attention for sm_100a, dense or block-sparse.
+// Dense bidirectional attention for sm_100a, two query tiles per CTA.
 //
 // Work item (h, i): one head h and one query block i of up to 128 rows,
-//   O = softmax(scale * Q_i K^T) V over the key blocks of its list, and the
-//   fp32 natural-log LSE of every row.
-// Dense mode walks key blocks 0..nkb-1 (SparseD abstract: full attention in the
-// early denoising steps; Step-dLLM abstract: the full map is recomputed at every
-// step). Sparse mode walks kv_idx[h,i,0..kv_count) (Step-dLLM abstract:
-// block-sparse attention over a reused mask). Both modes share every line of
-// the arithmetic, so a sparse call that keeps every block in ascending order is
-// bitwise equal to the dense call.
+//   O = softmax(scale * Q_i K^T) V over every key block 0..nkb-1, and the
+//   fp32 natural-log LSE of every row (SparseD abstract: full attention in the
+//   early denoising steps; Step-dLLM abstract: the full map is recomputed at
+//   every step). Block-sparse passes, whose query tiles each walk their own
+//   list, run in the one-tile kernel of attn_list_kernel.cuh.
 //
-// Two query tiles per CTA. A CTA works on pairs of work items, (h, 2p) in slot
-// 0 and (h, 2p+1) in slot 1, each slot with its own Q tile, S/P and O in TMEM,
-// its own softmax warpgroup and its own MMA-issuing warp. Per slot the chain
-// is S(t) = Q K_t^T -> softmax -> O += P(t) V_t -> S(t+1); the two slots run
-// it independently, so the tensor core works on one slot's MMAs while the
-// other slot's softmax runs. O += P V is issued in NPV parts, each as soon as
-// the softmax has stored that part of P, so it overlaps the rest of the
-// exponentials. In dense mode both slots read the same K_t / V_t tile; in
-// sparse mode each slot walks its own list and has its own tiles.
+// A CTA works on pairs of work items, (h, 2p) in slot 0 and (h, 2p+1) in
+// slot 1. Each slot has its own Q tile, S/P and O in TMEM, its own softmax
+// warpgroup and its own MMA-issuing warp. Both slots read the same K_t / V_t
+// tiles, so a tile is loaded once for two query tiles. Per slot the chain is
+// S(t) = Q K_t^T -> softmax -> O += P(t) V_t -> S(t+1). The two slots run it
+// independently, so the tensor core works on one slot's MMAs while the other
+// slot's softmax runs. O += P V is issued in NPV parts, each as soon as the
+// softmax has stored that part of P, so it overlaps the rest of the
+// exponentials.
 //
 // Persistent CTAs: the grid holds one CTA per SM and CTA b takes the pairs
 // b, b + G, b + 2G, ... of the flattened (h, p) order (G = grid size), so the
@@ -29,8 +26,7 @@
 //   warps 0-3   softmax of slot 0: warp w holds rows 32w..32w+31 of the tile,
 //               one full row per thread (row max and sum need no exchange)
 //   warps 4-7   softmax of slot 1, likewise
-//   warp 8      TMA producer: Q of each slot, K/V tiles into one NST-deep ring
-//               in the order the slots consume them
+//   warp 8      TMA producer: Q of each slot, K_t and V_t into one NST-deep ring
 //   warp 9      TMEM owner; MMA issuer of slot 0
 //   warp 10     MMA issuer of slot 1
 //   warp 11     idle (donates its registers)
@@ -46,14 +42,15 @@
 //   * the first part of PV_s(t) waits for the softmax's first PFULL_s(t)
 //     arrival, which follows its rescale of O_s and its epilogue reads of O_s
 //     (the first PV of an item overwrites O_s);
-//   * a ring stage is released by two commits after the MMAs reading it.
+//   * a ring stage is released by two commits after the MMAs reading it, one
+//     from each slot (two from slot 0 when the pair has no second query block).
 // The lazy rescale keeps O and the running sum on a stale row max until some
 // row of the warp sees its max grow by more than 2^8 (warp-uniform decision).
-// MASS variant (dense only): the pass also yields the block mass of pattern
-// selection. Each tile's probabilities of a row sum to ps = sum_c 2^(s_c*sl2 - m)
-// in the exp pass; times 2^(m - lse2), with lse2 the row's LSE from an earlier
-// full pass of the same inputs, that is the row's mass in the tile, and the
-// warp writes its 32 rows' sum as one of kMassParts partials per tile.
+// MASS variant: the pass also yields the block mass of pattern selection.
+// Each tile's probabilities of a row sum to ps = sum_c 2^(s_c*sl2 - m) in the
+// exp pass; times 2^(m - lse2), with lse2 the row's LSE from an earlier full
+// pass of the same inputs, that is the row's mass in the tile, and the warp
+// writes its 32 rows' sum as one of kMassParts partials per tile.
 // Every wait is bounded (mbarriers only, no named barriers), so a timed-out
 // warp cannot strand the others.
 #pragma once
@@ -70,8 +67,8 @@ struct AttnArgs {
   int H, L, bq, nqb, nkb;
   int Lk;                    // keys (== L, except over the gathered columns of a column pattern)
   float scale_log2;          // scale * log2(e)
-  const int32_t* kv_idx;     // sparse mode only
-  const int32_t* kv_count;   // sparse mode only
+  const int32_t* kv_idx;     // block-sparse passes (attn_list_kernel) only
+  const int32_t* kv_count;   // block-sparse passes only
   int kv_stride;
   float* lse;                // [H, L]
   uint16_t* o;               // [H, L, D]
@@ -151,58 +148,28 @@ __device__ __forceinline__ void exp_chunk32(const float* s, uint64_t scale2, uin
   }
 }
 
-// Key-block list of one slot of a pair.
-template <bool SPARSE>
-struct SlotList {
-  int n = 0;                      // blocks to walk (clamped count)
-  int qi = 0;                     // query block
-  const int32_t* list = nullptr;  // sparse mode
-  __device__ __forceinline__ int raw(int jj) const {
-    if constexpr (SPARSE) return list[jj];
-    else return jj;
-  }
+// Query blocks of pair w: (h, 2p) and (h, 2p+1), the second absent when nqb
+// is odd and p is the head's last pair.
+struct Pair {
+  int h, q0;
+  bool has1;
 };
 
-// Raw kv_count of the two query blocks of pair w (0 for a query block past
-// nqb); every role reads the next pair's counts one pair ahead.
-template <bool SPARSE>
-__device__ __forceinline__ int2 pair_raw_counts(const AttnArgs& a, int w, int npairs_h) {
-  int2 c = make_int2(0, 0);
-  if (w >= a.H * npairs_h) return c;
-  const int h = w / npairs_h, p = w - h * npairs_h;
-  const int q0 = 2 * p, q1 = 2 * p + 1;
-  if constexpr (SPARSE) {
-    c.x = a.kv_count[h * a.nqb + q0];
-    c.y = q1 < a.nqb ? a.kv_count[h * a.nqb + q1] : 0;
-  } else {
-    c.x = a.nkb;
-    c.y = q1 < a.nqb ? a.nkb : 0;
-  }
-  return c;
+__device__ __forceinline__ Pair pair_of(const AttnArgs& a, int w, int npairs_h) {
+  Pair r;
+  r.h = w / npairs_h;
+  const int p = w - r.h * npairs_h;
+  r.q0 = 2 * p;
+  r.has1 = r.q0 + 1 < a.nqb;
+  return r;
 }
 
-template <bool SPARSE>
-__device__ __forceinline__ SlotList<SPARSE> slot_list(const AttnArgs& a, int h, int qi, int n_raw) {
-  SlotList<SPARSE> s;
-  s.qi = qi;
-  if (qi >= a.nqb) return s;
-  if constexpr (SPARSE) {
-    const int cap = a.kv_stride < a.nkb ? a.kv_stride : a.nkb;
-    s.n = n_raw < 0 ? 0 : (n_raw > cap ? cap : n_raw);  // a bad count is reported by the producer
-    s.list = a.kv_idx + (static_cast<long>(h) * a.nqb + qi) * a.kv_stride;
-  } else {
-    s.n = a.nkb;
-  }
-  return s;
-}
-
-template <int D, int BK, bool SPARSE, bool MASS = false>
+template <int D, int BK, bool MASS = false>
 __global__ void __launch_bounds__(384, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const AttnArgs a) {
   using C = AttnCfg<D, BK>;
   constexpr int NST = C::NST;
-  static_assert(!(MASS && SPARSE), "the block mass comes from a full pass");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -284,58 +251,24 @@ __global__ void __launch_bounds__(384, 1)
         else ++qn0;
         return true;
       };
-      // a list entry, validated (out of range or not ascending is reported and
-      // read as block 0)
-      auto checked = [&](int raw, int& prev) -> int {
-        if constexpr (SPARSE) {
-          if (leader && (raw < 0 || raw >= a.nkb || raw <= prev)) ptx::record_error(kErrBadPattern);
-          prev = raw;
-        }
-        return (raw >= 0 && raw < a.nkb) ? raw : 0;
-      };
-      int2 cnt = pair_raw_counts<SPARSE>(a, blockIdx.x, npairs_h), cnt_next;
-      for (int w = blockIdx.x; ok && w < n_pairs; w += gridDim.x, cnt = cnt_next) {
-        cnt_next = pair_raw_counts<SPARSE>(a, w + gridDim.x, npairs_h);
-        h = w / npairs_h;
-        const int p = w - h * npairs_h;
-        const SlotList<SPARSE> l0 = slot_list<SPARSE>(a, h, 2 * p, cnt.x);
-        const SlotList<SPARSE> l1 = slot_list<SPARSE>(a, h, 2 * p + 1, cnt.y);
-        if (SPARSE && leader && (cnt.x != l0.n || (2 * p + 1 < a.nqb && cnt.y != l1.n)))
-          ptx::record_error(kErrBadPattern);
-        if (l0.n == 0 && l1.n == 0) continue;
+      for (int w = blockIdx.x; ok && w < n_pairs; w += gridDim.x) {
+        const Pair pr = pair_of(a, w, npairs_h);
+        h = pr.h;
         // the next pair's Q rows into L2 while this pair runs
         if (leader && w + static_cast<int>(gridDim.x) < n_pairs) {
-          const int wn = w + gridDim.x, hn = wn / npairs_h, pn = wn - hn * npairs_h;
+          const Pair pn = pair_of(a, w + gridDim.x, npairs_h);
 #pragma unroll
           for (int c = 0; c < C::DCH; ++c) {
-            ptx::tma_prefetch_3d(&tm_q, c * 64, 2 * pn * a.bq, hn);
-            if (2 * pn + 1 < a.nqb) ptx::tma_prefetch_3d(&tm_q, c * 64, (2 * pn + 1) * a.bq, hn);
+            ptx::tma_prefetch_3d(&tm_q, c * 64, pn.q0 * a.bq, pn.h);
+            if (pn.has1) ptx::tma_prefetch_3d(&tm_q, c * 64, (pn.q0 + 1) * a.bq, pn.h);
           }
         }
-        const int n = l0.n > l1.n ? l0.n : l1.n;
-        int prev0 = -1, prev1 = -1;
-        int raw0 = l0.n > 0 ? l0.raw(0) : 0, raw1 = l1.n > 0 ? l1.raw(0) : 0;
-        for (int j = 0; ok && j < n; ++j) {
-          const bool a0 = j < l0.n, a1 = j < l1.n;
-          // list entries one tile ahead, off the copy-issue path
-          const int r0 = raw0, r1 = raw1;
-          if (j + 1 < l0.n) raw0 = l0.raw(j + 1);
-          if (j + 1 < l1.n) raw1 = l1.raw(j + 1);
-          if constexpr (SPARSE) {
-            const int j0 = a0 ? checked(r0, prev0) : 0;
-            const int j1 = a1 ? checked(r1, prev1) : 0;
-            if (a0 && j == 0) ok = load_q(0, l0.qi);
-            if (ok && a0) ok = load_tile(&tm_k, j0);
-            if (ok && a1 && j == 0) ok = load_q(1, l1.qi);
-            if (ok && a1) ok = load_tile(&tm_k, j1);
-            if (ok && a0) ok = load_tile(&tm_v, j0);
-            if (ok && a1) ok = load_tile(&tm_v, j1);
-          } else {
-            if (j == 0) ok = load_q(0, l0.qi);
-            if (ok) ok = load_tile(&tm_k, j);
-            if (ok && a1 && j == 0) ok = load_q(1, l1.qi);
-            if (ok) ok = load_tile(&tm_v, j);
-          }
+        // in the order the slots consume them: Q0, K_0, Q1, V_0, K_1, V_1, ...
+        for (int j = 0; ok && j < a.nkb; ++j) {
+          if (j == 0) ok = load_q(0, pr.q0);
+          if (ok) ok = load_tile(&tm_k, j);
+          if (ok && pr.has1 && j == 0) ok = load_q(1, pr.q0 + 1);
+          if (ok) ok = load_tile(&tm_v, j);
         }
       }
       if (!ok) {
@@ -355,8 +288,8 @@ __global__ void __launch_bounds__(384, 1)
       // (S(t) -> softmax -> PV(t) -> S(t+1)) waits on the other's softmax. The
       // whole warp runs the loop (warp-uniform control flow, descriptors in
       // uniform registers); one elected lane issues the MMAs and commits. A
-      // ring stage gets two commits in all (EMPTY counts two): one from each
-      // slot reading a shared dense tile, else two from the slot that owns it.
+      // ring stage gets two commits (EMPTY counts two): one from each slot, or
+      // both from slot 0 when the pair has no second query block.
       const int s = warp - 9;
       constexpr uint32_t HI = ptx::sdesc_sw128_hi(1024);
       const uint32_t q_lo = ptx::sdesc_sw128_lo(sb + (s ? C::OFF_Q1 : C::OFF_Q0), 16);
@@ -370,32 +303,14 @@ __global__ void __launch_bounds__(384, 1)
       int tcnt = 0;     // tiles of this slot (PFULL phases)
       bool ok = true;
       auto commit = [&](int idx) { ptx::umma_commit_if(leader, bar(idx)); };
-      int2 cnt = pair_raw_counts<SPARSE>(a, blockIdx.x, npairs_h), cnt_next;
-      for (int w = blockIdx.x; ok && w < n_pairs; w += gridDim.x, cnt = cnt_next) {
-        cnt_next = pair_raw_counts<SPARSE>(a, w + gridDim.x, npairs_h);
-        const int h = w / npairs_h;
-        const int p = w - h * npairs_h;
-        const int n0 = slot_list<SPARSE>(a, h, 2 * p, cnt.x).n;
-        const int n1 = slot_list<SPARSE>(a, h, 2 * p + 1, cnt.y).n;
-        const int n = n0 > n1 ? n0 : n1;
-        const int nm = s ? n1 : n0;
-        for (int j = 0; j < n; ++j) {
-          const bool a0 = j < n0, a1 = j < n1;
-          int sk, sv;
-          bool sole;  // the tile's two EMPTY commits both come from this slot
-          if constexpr (SPARSE) {
-            const int base = seq;
-            seq += (a0 ? 2 : 0) + (a1 ? 2 : 0);
-            sk = s ? base + (a0 ? 1 : 0) : base;
-            sv = sk + (a0 ? 1 : 0) + (a1 ? 1 : 0);
-            sole = true;
-          } else {
-            sk = seq;
-            sv = seq + 1;
-            seq += 2;
-            sole = !a1;
-          }
-          if (j >= nm) continue;
+      for (int w = blockIdx.x; ok && w < n_pairs; w += gridDim.x) {
+        const Pair pr = pair_of(a, w, npairs_h);
+        const bool mine = s == 0 || pr.has1;   // slot 1 idles on a pair without a second block
+        const bool sole = !pr.has1;             // slot 0 then gives both commits of each tile
+        for (int j = 0; j < a.nkb; ++j) {
+          const int sk = seq, sv = seq + 1;     // K_j and V_j
+          seq += 2;
+          if (!mine) continue;
           if ((j == 0 && !wait(C::B_QFULL + s, qn++)) || !wait(C::B_FULL + sk % NST, sk / NST)) {
             ok = false;
             break;
@@ -413,7 +328,7 @@ __global__ void __launch_bounds__(384, 1)
           commit(C::B_SFULL + s);
           commit(C::B_EMPTY + sk % NST);
           if (sole) commit(C::B_EMPTY + sk % NST);
-          if (j == nm - 1) commit(C::B_QEMPTY + s);
+          if (j == a.nkb - 1) commit(C::B_QEMPTY + s);
           // O += P V in NPV parts, each issued as soon as the softmax has
           // stored that part of P
           if (!wait(C::B_FULL + sv % NST, sv / NST)) {
@@ -462,48 +377,22 @@ __global__ void __launch_bounds__(384, 1)
     const uint64_t scale2 = ptx::f32x2(sl2, sl2);
     int tcount = 0;  // tiles of this slot so far (SFULL / PVDONE phases)
     bool ok = true;
-    int2 cnt = pair_raw_counts<SPARSE>(a, blockIdx.x, npairs_h), cnt_next;
-    for (int w = blockIdx.x; ok && w < n_pairs; w += gridDim.x, cnt = cnt_next) {
-      cnt_next = pair_raw_counts<SPARSE>(a, w + gridDim.x, npairs_h);
-      const int h = w / npairs_h;
-      const int p = w - h * npairs_h;
-      const int qi = 2 * p + slot;
-      if (qi >= a.nqb) continue;
-      const SlotList<SPARSE> it = slot_list<SPARSE>(a, h, qi, slot ? cnt.y : cnt.x);
+    for (int w = blockIdx.x; ok && w < n_pairs; w += gridDim.x) {
+      const Pair pr = pair_of(a, w, npairs_h);
+      const int h = pr.h;
+      const int qi = pr.q0 + slot;
+      if (slot == 1 && !pr.has1) continue;
       const int grow = qi * a.bq + r;
       const bool row_valid = (r < a.bq) && (grow < a.L);
       uint4* o_dst = reinterpret_cast<uint4*>(a.o + (static_cast<long>(h) * a.L + grow) * D);
-      if (it.n == 0) {
-        if (row_valid) {
-#pragma unroll
-          for (int c = 0; c < D / 8; ++c) o_dst[c] = make_uint4(0, 0, 0, 0);
-          a.lse[static_cast<long>(h) * a.L + grow] = -__int_as_float(0x7f800000);
-        }
-        continue;
-      }
       float m = -__int_as_float(0x7f800000);  // running row max, log2 units (scaled)
       float l = 0.f;                          // running row sum
       // MASS: my row's LSE (log2 units) from the earlier full pass
       float lse2_prev = 0.f;
       if constexpr (MASS)
         lse2_prev = row_valid ? a.lse_prev[static_cast<long>(h) * a.L + grow] * 1.44269504088896340736f : 0.f;
-      // only a list that can hold the ragged last key block needs its entries
-      // here; they are read one tile ahead, off the critical path
-      const bool ragged = SPARSE && (a.Lk % BK) != 0;
-      int blk_next = 0;
-      if (ragged) {
-        const int b0 = it.raw(0);
-        blk_next = (b0 >= 0 && b0 < a.nkb) ? b0 : 0;
-      }
-      for (int jj = 0; jj < it.n; ++jj, ++tcount) {
-        int blk = jj;
-        if (ragged) {
-          blk = blk_next;
-          if (jj + 1 < it.n) {
-            const int bn = it.raw(jj + 1);
-            blk_next = (bn >= 0 && bn < a.nkb) ? bn : 0;
-          }
-        }
+      for (int jj = 0; jj < a.nkb; ++jj, ++tcount) {
+        const int blk = jj;
         if (!ptx::mbar_wait_warp(bar(C::B_SFULL + slot), tcount & 1, abort_flag, a.timeout_ns, kErrTimeout)) {
           ok = false;
           break;

@@ -16,6 +16,7 @@
 
 #include "sparsed.h"
 #include "attn_kernel.cuh"
+#include "attn_list_kernel.cuh"
 #include "select_kernels.cuh"
 #include "column_kernels.cuh"
 #include "losa_kernels.cuh"
@@ -188,11 +189,10 @@ struct Problem {
 // The register split of the kernel (setmaxnreg) must be funded by its launch
 // register count; checked once per kernel before the first launch, so a raise
 // can never wait forever.
-template <int D, int BK, bool SPARSE, bool MASS>
-int launch_attn_t(const Problem& p, const int32_t* kv_idx, const int32_t* kv_count, int kv_stride,
-                  const float* lse_prev, float* mass_part, cudaStream_t st) {
+template <int D, int BK, bool MASS>
+int launch_attn_t(const Problem& p, const float* lse_prev, float* mass_part, cudaStream_t st) {
   using C = AttnCfg<D, BK>;
-  auto kern = attn_fwd_kernel<D, BK, SPARSE, MASS>;
+  auto kern = attn_fwd_kernel<D, BK, MASS>;
   static int regs = -1;
   if (regs < 0) {
     cudaFuncAttributes fa;
@@ -212,9 +212,9 @@ int launch_attn_t(const Problem& p, const int32_t* kv_idx, const int32_t* kv_cou
   a.nqb = p.nqb;
   a.nkb = p.nkb;
   a.scale_log2 = p.scale * 1.44269504088896340736f;
-  a.kv_idx = kv_idx;
-  a.kv_count = kv_count;
-  a.kv_stride = kv_stride;
+  a.kv_idx = nullptr;
+  a.kv_count = nullptr;
+  a.kv_stride = 0;
   a.lse = p.LSE;
   a.o = p.O;
   a.lse_prev = lse_prev;
@@ -232,15 +232,62 @@ int launch_attn_t(const Problem& p, const int32_t* kv_idx, const int32_t* kv_cou
   return SPARSED_OK;
 }
 
-// mass_part != nullptr selects the fused variant (dense only): the pass also
-// writes the block-mass partials, using lse_prev as every row's LSE.
+// Block-sparse passes: the one-tile kernel (each query tile walks its own
+// list), with the same register-split check.
+template <int D, int BK>
+int launch_list_t(const Problem& p, const int32_t* kv_idx, const int32_t* kv_count, int kv_stride,
+                  cudaStream_t st) {
+  using C = ListCfg<D, BK>;
+  auto kern = attn_list_kernel<D, BK>;
+  static int regs = -1;
+  if (regs < 0) {
+    cudaFuncAttributes fa;
+    SP_CUDA(cudaFuncGetAttributes(&fa, kern));
+    regs = fa.numRegs;
+  }
+  if (regs * C::THREADS < C::REGS_SOFTMAX * 256 + C::REGS_OTHER * 128) return SPARSED_ERR_UNSUPPORTED;
+  CUtensorMap tq, tk, tv;
+  SP_TRY(make_map(&tq, p.Q, p.H, p.L, D, 128));
+  SP_TRY(make_map(&tk, p.K, p.H, p.Lk, D, BK));
+  SP_TRY(make_map(&tv, p.V, p.H, p.Lk, D, BK));
+  AttnArgs a;
+  a.H = p.H;
+  a.L = p.L;
+  a.Lk = p.Lk;
+  a.bq = p.bq;
+  a.nqb = p.nqb;
+  a.nkb = p.nkb;
+  a.scale_log2 = p.scale * 1.44269504088896340736f;
+  a.kv_idx = kv_idx;
+  a.kv_count = kv_count;
+  a.kv_stride = kv_stride;
+  a.lse = p.LSE;
+  a.o = p.O;
+  a.lse_prev = nullptr;
+  a.mass_part = nullptr;
+  a.timeout_ns = kWaitTimeoutNs;
+  int sms = 0;
+  SP_TRY(sm_count(&sms));
+  SP_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES));
+  // persistent: one CTA per SM, each walking items blockIdx.x, blockIdx.x + gridDim.x, ...
+  const long items = static_cast<long>(p.H) * p.nqb;
+  const int grid = static_cast<int>(items < sms ? items : sms);
+  kern<<<grid, C::THREADS, C::SMEM_BYTES, st>>>(tq, tk, tv, a);
+  SP_CUDA(cudaGetLastError());
+  return SPARSED_OK;
+}
+
+// Dense passes (and the fused selecting pass) run in the two-tile kernel,
+// block-sparse passes in the one-tile kernel. mass_part != nullptr selects the
+// fused variant (dense only): the pass also writes the block-mass partials,
+// using lse_prev as every row's LSE.
 int launch_attn(const Problem& p, bool sparse, const int32_t* kv_idx, const int32_t* kv_count,
                 int kv_stride, cudaStream_t st, const float* lse_prev = nullptr, float* mass_part = nullptr) {
 #define SP_ATTN(D_, BK_)                                                                                  \
   if (p.d == D_ && p.bk == BK_) {                                                                         \
-    if (sparse) return launch_attn_t<D_, BK_, true, false>(p, kv_idx, kv_count, kv_stride, nullptr, nullptr, st); \
-    if (mass_part) return launch_attn_t<D_, BK_, false, true>(p, nullptr, nullptr, 0, lse_prev, mass_part, st);   \
-    return launch_attn_t<D_, BK_, false, false>(p, nullptr, nullptr, 0, nullptr, nullptr, st);           \
+    if (sparse) return launch_list_t<D_, BK_>(p, kv_idx, kv_count, kv_stride, st);                        \
+    if (mass_part) return launch_attn_t<D_, BK_, true>(p, lse_prev, mass_part, st);                     \
+    return launch_attn_t<D_, BK_, false>(p, nullptr, nullptr, st);                                        \
   }
   SP_ATTN(64, 64)
   SP_ATTN(64, 128)
@@ -1346,7 +1393,7 @@ int sparsed_losa_splits(int H, int B, int bq, int P, int bk, int sm_count, int* 
   if (!splits || H < 1 || B < 1 || P < 1 || sm_count < 1) return SPARSED_ERR_INVALID_ARG;
   if ((bq != 64 && bq != 128) || (bk != 64 && bk != 128)) return SPARSED_ERR_UNSUPPORTED;
   const long per_split = static_cast<long>(H) * cdiv(B, bq);  // work items of one split
-  long s = 2L * sm_count / per_split;  // the attention kernel runs two work items per SM
+  long s = sm_count / per_split;
   if (s < 1) s = 1;
   long s_max = cdiv(cdiv(P, bk), kLosaMinChunk);
   if (s_max > kLosaMaxSplits) s_max = kLosaMaxSplits;

@@ -399,9 +399,8 @@ int sparsed_select_pattern_noalloc(const uint16_t* Q, const uint16_t* K, const u
  * outside a graph capture (it creates that stream and its two events). */
 
 /* Splits for a step of these sizes on a GPU with sm_count SMs: as many as
- * keep two work items per SM at most (the attention kernel runs two query
- * tiles per SM), one split having H*ceil(B/bq) work items
- * (floor(2*sm_count / (H*ceil(B/bq))), at least 1, at most min(32, ceil(nkb/4))). */
+ * keep one split's H*ceil(B/bq) work items per SM at most
+ * (floor(sm_count / (H*ceil(B/bq))), at least 1, at most min(32, ceil(nkb/4))). */
 int sparsed_losa_splits(int H, int B, int bq, int P, int bk, int sm_count, int* splits);
 
 /* Workspace bytes of sparsed_losa_init / _step / _block for these sizes:

@@ -170,9 +170,9 @@ def _losa_splits(H=32, B=64, bq=64, P_=32768, bk=64, sms=148):
 
 
 def test_losa_splits():
-    assert _losa_splits() == (_lib.OK, 9)                      # 2 x 148 work items / 32 per split
-    assert _losa_splits(B=128) == (_lib.OK, 4)                 # two query tiles per split
-    assert _losa_splits(H=400) == (_lib.OK, 1)                 # at least one split
+    assert _losa_splits() == (_lib.OK, 4)                      # 148 SMs / 32 work items per split
+    assert _losa_splits(B=128) == (_lib.OK, 2)                 # two query tiles per split
+    assert _losa_splits(H=200) == (_lib.OK, 1)                 # at least one split
     assert _losa_splits(H=1, P_=100) == (_lib.OK, 1)           # at most ceil(nkb / 4): nkb = 2
     assert _losa_splits(H=1, P_=64 * 40) == (_lib.OK, 10)      # nkb = 40 -> at most 10
     assert _losa_splits(H=1, P_=64 * 1000) == (_lib.OK, 32)    # never more than 32

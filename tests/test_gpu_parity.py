@@ -114,9 +114,13 @@ def test_many_items_per_persistent_cta(d, bq, bk):
 
 
 @pytest.mark.parametrize("d,bk", [(64, 64), (128, 128), (128, 64)])
-def test_keep_all_bitwise_equals_dense(d, bk):
+def test_keep_all_equals_dense(d, bk):
+    """A list that keeps every block in ascending order is dense attention:
+    the block-sparse kernel and the dense kernel (two different kernels, the
+    same sums in a different grouping) agree to fp32 rounding of the row sums
+    and one bf16 rounding of O, and both match the oracle."""
     H, L, bq = 2, 1024 + 64, 128
-    q, k, v, _ = _inputs(H, L, d, seed=5)
+    q, k, v, scale = _inputs(H, L, d, seed=5)
     qc, kc, vc = _cuda(q, k, v)
     nqb, nkb = -(-L // bq), -(-L // bk)
     kv_idx = torch.arange(nkb, dtype=torch.int32, device="cuda").repeat(H, nqb, 1).contiguous()
@@ -124,8 +128,10 @@ def test_keep_all_bitwise_equals_dense(d, bk):
     o1, l1 = sp.dense_attn(qc, kc, vc, bq=bq, bk=bk)
     o2, l2 = sp.block_sparse_attn(qc, kc, vc, kv_idx, kv_count, bq=bq, bk=bk)
     sp.device_check()
-    assert torch.equal(o1.view(torch.int16), o2.view(torch.int16))
-    assert torch.equal(l1, l2)
+    assert (o1.float() - o2.float()).abs().max().item() <= 2 ** -7
+    assert (l1 - l2).abs().max().item() <= 1e-5
+    o_ref, l_ref = oracle_dense_heads(q, k, v, scale)
+    assert_o_lse(o2, l2, o_ref, l_ref, f"keep-all sparse d={d} bk={bk}")
 
 
 def test_determinism():
