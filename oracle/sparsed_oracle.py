@@ -48,6 +48,7 @@ import numpy as np
 
 DENSE, SELECT, SPARSE = 0, 1, 2
 ROUND_EPS = 1e-6  # guards ceil() against products like 0.1*30 = 3.0000000000000004
+DRIFT_AMPLITUDE = 2.0 ** -6  # default size of the per-step query drift (O6b)
 
 # --------------------------------------------------------------------------
 # O1  dense bidirectional attention
@@ -374,15 +375,20 @@ def schedule(T, warmup_frac, refresh_every=0):
 
 
 def run_steps(q, k, v, scale, bq, bk, keep_ratio, budget, T, warmup_frac,
-              refresh_every=0):
-    """The denoising loop over one layer with fixed inputs: each step runs the
-    kind ``schedule`` gives; SELECT refreshes the cached pattern; SPARSE uses
-    the cached pattern. Returns (o, lse, kinds, pattern) of the last step."""
+              refresh_every=0, drift_seed=None, drift_amplitude=DRIFT_AMPLITUDE, patterns=None):
+    """The denoising loop over one layer: each step runs the kind ``schedule``
+    gives; SELECT refreshes the cached pattern; SPARSE uses the cached pattern.
+    With ``drift_seed`` the queries of step t are drift_queries(q, drift_seed,
+    t) (K and V fixed), otherwise q at every step. ``patterns`` (a list), when
+    given, receives every SELECT step's (t, pattern). Returns (o, lse, kinds,
+    pattern) of the last step."""
     kinds = schedule(T, warmup_frac, refresh_every)
     H, L, _ = q.shape
     pattern = None
     o = lse = None
+    q_fixed = q
     for t in range(T):
+        q = q_fixed if drift_seed is None else drift_queries(q_fixed, drift_seed, t, drift_amplitude)
         if kinds[t] == DENSE:
             o = np.empty(q.shape)
             lse = np.empty((H, L))
@@ -391,6 +397,8 @@ def run_steps(q, k, v, scale, bq, bk, keep_ratio, budget, T, warmup_frac,
         elif kinds[t] == SELECT:
             pattern = select_pattern(q, k, v, scale, bq, bk, keep_ratio, budget)
             o, lse = pattern["o"], pattern["lse"]
+            if patterns is not None:
+                patterns.append((t, pattern))
         else:
             o = np.empty(q.shape)
             lse = np.empty((H, L))
@@ -399,6 +407,59 @@ def run_steps(q, k, v, scale, bq, bk, keep_ratio, budget, T, warmup_frac,
                                                 pattern["kv_idx"][h],
                                                 pattern["kv_count"][h], bq, bk)
     return o, lse, kinds, pattern
+
+
+# --------------------------------------------------------------------------
+# O6b  queries that change across the denoising steps
+# --------------------------------------------------------------------------
+
+
+def fmix32(x):
+    """MurmurHash3's 32-bit finalizer (Austin Appleby's published definition):
+    h ^= h >> 16; h *= 0x85ebca6b; h ^= h >> 13; h *= 0xc2b2ae35; h ^= h >> 16,
+    all modulo 2^32. Elementwise on an integer array."""
+    h = np.asarray(x, dtype=np.uint64) & 0xFFFFFFFF
+    h = h ^ (h >> 16)
+    h = (h * 0x85EBCA6B) & 0xFFFFFFFF
+    h = h ^ (h >> 13)
+    h = (h * 0xC2B2AE35) & 0xFFFFFFFF
+    h = h ^ (h >> 16)
+    return h
+
+
+def drift_uniform(seed, t, n):
+    """The counter-based uniforms of step t: for element i of a tensor of n
+    elements, key = fmix32(fmix32(seed) ^ t) and u = (fmix32(i ^ key) >> 8) *
+    2^-23 - 1, on a 2^-23 grid in [-1, 1). Returned in float64 (exact)."""
+    key = int(fmix32(int(fmix32(seed)) ^ (int(t) & 0xFFFFFFFF)))
+    i = np.arange(n, dtype=np.uint64)
+    h = fmix32(i ^ key)
+    return (h >> 8).astype(np.float64) * 2.0 ** -23 - 1.0
+
+
+def bf16_round(x32):
+    """Round float32 values to bf16, nearest even (finite inputs), returned as
+    float64."""
+    b = np.asarray(x32, dtype=np.float32).view(np.uint32).astype(np.uint64)
+    b = (b + 0x7FFF + ((b >> 16) & 1)) >> 16
+    return (b.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+
+
+def drift_queries(q, seed, t, amplitude=DRIFT_AMPLITUDE):
+    """Q of denoising step t: Q_t = bf16(fp32(Q) + fp32(amplitude * u)) elementwise,
+    u = drift_uniform(seed, t, Q.size) in the row-major order of Q [H, L, d].
+
+    The pages give no per-step activations. They say that attention patterns
+    stay similar across steps (SparseD abstract) and are only locally
+    consistent, shifting at some transitions (Step-dLLM abstract). The reading
+    taken: a small seeded perturbation of the queries at every step, the same
+    bits on any machine (integer hash, one fp32 addition and one bf16
+    rounding). ``q`` holds bf16 values (float64 or float32); amplitude a power
+    of two keeps amplitude * u exact in fp32."""
+    q32 = np.asarray(q, dtype=np.float32)
+    u = drift_uniform(seed, t, q32.size).reshape(q32.shape)
+    d32 = (u * float(amplitude)).astype(np.float32)
+    return bf16_round(q32 + d32)
 
 
 # --------------------------------------------------------------------------
