@@ -46,7 +46,7 @@ from ._lib import (BUDGET_ENTROPY, BUDGET_UNIFORM, STEP_DENSE, STEP_SELECT,  # n
                    STEP_SPARSE, SparsedError, check)
 
 __all__ = ["dense_attn", "select_pattern", "block_sparse_attn", "run_steps", "workspace_bytes",
-           "run_steps_workspace_bytes",
+           "run_steps_workspace_bytes", "drift_queries", "DRIFT_AMPLITUDE",
            "uniform_keep", "schedule", "device_check", "version", "SparsedError", "Pattern",
            "RunResult", "default_scale", "column_keep", "column_workspace_bytes", "select_columns",
            "column_sparse_attn", "run_steps_columns", "ColumnPattern", "select_head_entropy",
@@ -214,12 +214,30 @@ class RunResult:
     kv_count: torch.Tensor
 
 
+DRIFT_AMPLITUDE = 2.0 ** -6
+
+
+def drift_queries(q, seed: int, t: int, amplitude: float = DRIFT_AMPLITUDE, out=None, stream=None):
+    """The queries of denoising step t (sparsed_drift_queries): a seeded
+    perturbation of q, the same bits on any machine."""
+    H, L, d = q.shape
+    if q.dtype != torch.bfloat16 or not q.is_cuda or not q.is_contiguous():
+        raise ValueError("q must be a contiguous bfloat16 CUDA tensor [H, L, d]")
+    out = torch.empty_like(q) if out is None else out
+    check(_lib.load().sparsed_drift_queries(_ptr(q), H, L, d, seed & 0xFFFFFFFF, t, amplitude, _ptr(out),
+                                            _stream(stream)), "sparsed_drift_queries")
+    return out
+
+
 def run_steps(q, k, v, T, warmup_frac=0.2, keep=0.1, budget="uniform", refresh_every=0, scale=None,
               bq=128, bk=128, start_step=0, pattern=None, time_steps=False, out=None, lse=None,
-              workspace=None, stream=None, end_step=None) -> RunResult:
+              workspace=None, stream=None, end_step=None, drift_seed=None,
+              drift_amplitude=DRIFT_AMPLITUDE) -> RunResult:
     """The denoising loop over one layer: dense warm-up, pattern selection at
     the switch (and at anchors), block-sparse attention afterwards. With
-    ``end_step`` only steps start_step .. end_step-1 of the T-step schedule run."""
+    ``end_step`` only steps start_step .. end_step-1 of the T-step schedule run.
+    With ``drift_seed`` every step t attends with its own queries,
+    drift_queries(q, drift_seed, t, drift_amplitude) (K and V fixed)."""
     H, L, d = _check_qkv(q, k, v)
     scale = default_scale(d) if scale is None else scale
     mode = {"uniform": BUDGET_UNIFORM, "entropy": BUDGET_ENTROPY}[budget]
@@ -241,7 +259,14 @@ def run_steps(q, k, v, T, warmup_frac=0.2, keep=0.1, budget="uniform", refresh_e
     tail = (_ptr(kv_idx), _ptr(kv_count), kv_idx.shape[2], _ptr(out), _ptr(lse),
             ctypes.cast(kinds, ctypes.c_void_p), None if ms is None else ctypes.cast(ms, ctypes.c_void_p),
             _ptr(ws), ws.numel(), _stream(stream))
-    if end_step is None:
+    if drift_seed is not None:
+        q_step = torch.empty_like(q)
+        rc = _lib.load().sparsed_run_steps_drift(_ptr(q), _ptr(k), _ptr(v), H, L, d, scale, bq, bk, keep, mode,
+                                                 T, warmup_frac, refresh_every, start_step,
+                                                 T if end_step is None else end_step, have,
+                                                 drift_seed & 0xFFFFFFFF, drift_amplitude, _ptr(q_step), *tail)
+        check(rc, "sparsed_run_steps_drift")
+    elif end_step is None:
         rc = _lib.load().sparsed_run_steps(_ptr(q), _ptr(k), _ptr(v), H, L, d, scale, bq, bk, keep, mode, T,
                                            warmup_frac, refresh_every, start_step, have, *tail)
         check(rc, "sparsed_run_steps")

@@ -48,6 +48,9 @@ SIGNATURES = {
     "sparsed_run_steps": (_I, [_P, _P, _P, _I, _I, _I, _F, _I, _I, _F, _I, _I, _F, _I, _I, _I, _P, _P,
                                _I, _P, _P, _P, _P, _P, _SZ, _P]),
     "sparsed_run_steps_workspace_bytes": (_I, [_I, _I, _I, _I, ctypes.POINTER(_SZ)]),
+    "sparsed_drift_queries": (_I, [_P, _I, _I, _I, ctypes.c_uint, _I, _F, _P, _P]),
+    "sparsed_run_steps_drift": (_I, [_P, _P, _P, _I, _I, _I, _F, _I, _I, _F, _I, _I, _F, _I, _I, _I, _I,
+                                     ctypes.c_uint, _F, _P, _P, _P, _I, _P, _P, _P, _P, _P, _SZ, _P]),
     "sparsed_run_steps_span": (_I, [_P, _P, _P, _I, _I, _I, _F, _I, _I, _F, _I, _I, _F, _I, _I, _I, _I, _P,
                                     _P, _I, _P, _P, _P, _P, _P, _SZ, _P]),
     "sparsed_select_head_entropy": (_I, [_P, _P, _P, _I, _I, _I, _F, _I, _I, _P, _P, _P, _P, _SZ, _P]),

@@ -177,6 +177,53 @@ __global__ void wait_timeout_selftest_kernel(unsigned long long timeout_ns) {
   }
 }
 
+// ---- queries that change across the denoising steps
+// Q_t = bf16(fp32(Q) + fp32(amplitude * u)) elementwise, with the counter-based
+// uniform u = (fmix32(i ^ key) >> 8) * 2^-23 - 1 of element i (row-major over
+// [H, L, d]) and key = fmix32(fmix32(seed) ^ t); fmix32 is the MurmurHash3
+// 32-bit finalizer. The product and the sum are rounded once each (no fused
+// multiply-add), so the bits are those of any other implementation of the
+// same definition.
+__host__ __device__ inline uint32_t fmix32(uint32_t h) {
+  h ^= h >> 16;
+  h *= 0x85EBCA6Bu;
+  h ^= h >> 13;
+  h *= 0xC2B2AE35u;
+  h ^= h >> 16;
+  return h;
+}
+
+inline uint32_t drift_key(uint32_t seed, int t) { return fmix32(fmix32(seed) ^ static_cast<uint32_t>(t)); }
+
+__device__ __forceinline__ uint16_t bf16_rne(float x) {
+  const uint32_t b = __float_as_uint(x);
+  return static_cast<uint16_t>((b + 0x7FFFu + ((b >> 16) & 1u)) >> 16);
+}
+
+// Eight elements (16 bytes) per thread; n is a multiple of 8 (d is).
+__global__ void __launch_bounds__(256)
+    drift_queries_kernel(const uint4* __restrict__ q, long n8, uint32_t key, float amplitude,
+                         uint4* __restrict__ q_out) {
+  const long v = static_cast<long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (v >= n8) return;
+  const uint4 in = q[v];
+  const uint32_t w[4] = {in.x, in.y, in.z, in.w};
+  uint32_t o[4];
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    uint16_t r[2];
+#pragma unroll
+    for (int half = 0; half < 2; ++half) {
+      const uint32_t i = static_cast<uint32_t>(v * 8 + e * 2 + half);
+      const float u = __fsub_rn(__fmul_rn(static_cast<float>(fmix32(i ^ key) >> 8), 0x1p-23f), 1.0f);
+      const float qv = __uint_as_float((half ? (w[e] >> 16) : (w[e] & 0xFFFFu)) << 16);
+      r[half] = bf16_rne(__fadd_rn(qv, __fmul_rn(u, amplitude)));
+    }
+    o[e] = static_cast<uint32_t>(r[0]) | (static_cast<uint32_t>(r[1]) << 16);
+  }
+  q_out[v] = make_uint4(o[0], o[1], o[2], o[3]);
+}
+
 struct Problem {
   const uint16_t *Q, *K, *V;
   uint16_t* O;
@@ -542,6 +589,30 @@ int check_select_args(const Problem& p, float keep_ratio, int budget_mode, int32
   return SPARSED_OK;
 }
 
+// Per-step queries of the step driver: seed and amplitude of the drift, and
+// the caller's buffer that receives each step's queries.
+struct Drift {
+  uint32_t seed;
+  float amplitude;
+  uint16_t* q_step;
+};
+
+int launch_drift(const uint16_t* Q, long n, uint32_t seed, int t, float amplitude, uint16_t* Q_out,
+                 cudaStream_t st) {
+  const long n8 = n / 8;
+  drift_queries_kernel<<<static_cast<unsigned>(cdiv(n8, 256)), 256, 0, st>>>(
+      reinterpret_cast<const uint4*>(Q), n8, drift_key(seed, t), amplitude, reinterpret_cast<uint4*>(Q_out));
+  SP_CUDA(cudaGetLastError());
+  return SPARSED_OK;
+}
+
+int run_steps_impl(const uint16_t* Q, const uint16_t* K, const uint16_t* V, int H, int L, int d,
+                   float scale, int bq, int bk, float keep_ratio, int budget_mode, int T,
+                   float warmup_frac, int refresh_every, int start_step, int end_step,
+                   int have_pattern, int32_t* kv_idx, int32_t* kv_count, int kv_stride, uint16_t* O,
+                   float* LSE, int8_t* step_kind, float* step_ms, void* workspace,
+                   size_t workspace_bytes, void* stream, const Drift* drift);
+
 }  // namespace
 
 extern "C" {
@@ -690,6 +761,47 @@ int sparsed_run_steps_span(const uint16_t* Q, const uint16_t* K, const uint16_t*
                            int have_pattern, int32_t* kv_idx, int32_t* kv_count, int kv_stride, uint16_t* O,
                            float* LSE, int8_t* step_kind, float* step_ms, void* workspace,
                            size_t workspace_bytes, void* stream) {
+  return run_steps_impl(Q, K, V, H, L, d, scale, bq, bk, keep_ratio, budget_mode, T, warmup_frac, refresh_every,
+                        start_step, end_step, have_pattern, kv_idx, kv_count, kv_stride, O, LSE, step_kind, step_ms,
+                        workspace, workspace_bytes, stream, nullptr);
+}
+
+int sparsed_run_steps_drift(const uint16_t* Q, const uint16_t* K, const uint16_t* V, int H, int L, int d,
+                            float scale, int bq, int bk, float keep_ratio, int budget_mode, int T,
+                            float warmup_frac, int refresh_every, int start_step, int end_step,
+                            int have_pattern, unsigned int drift_seed, float drift_amplitude, uint16_t* Q_step,
+                            int32_t* kv_idx, int32_t* kv_count, int kv_stride, uint16_t* O, float* LSE,
+                            int8_t* step_kind, float* step_ms, void* workspace, size_t workspace_bytes,
+                            void* stream) {
+  if (!Q_step || !aligned16(Q_step) || !std::isfinite(drift_amplitude)) return SPARSED_ERR_INVALID_ARG;
+  const Drift drift{drift_seed, drift_amplitude, Q_step};
+  return run_steps_impl(Q, K, V, H, L, d, scale, bq, bk, keep_ratio, budget_mode, T, warmup_frac, refresh_every,
+                        start_step, end_step, have_pattern, kv_idx, kv_count, kv_stride, O, LSE, step_kind, step_ms,
+                        workspace, workspace_bytes, stream, &drift);
+}
+
+int sparsed_drift_queries(const uint16_t* Q, int H, int L, int d, unsigned int seed, int t, float amplitude,
+                          uint16_t* Q_out, void* stream) {
+  if (H < 0 || L < 0 || t < 0) return SPARSED_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return SPARSED_ERR_UNSUPPORTED;
+  if (!Q || !Q_out || !aligned16(Q) || !aligned16(Q_out) || !std::isfinite(amplitude))
+    return SPARSED_ERR_INVALID_ARG;
+  if (static_cast<long long>(H) * L * d >= (1ll << 31)) return SPARSED_ERR_UNSUPPORTED;
+  if (static_cast<long>(H) * L == 0) return SPARSED_OK;
+  SP_TRY(require_sm100());
+  return launch_drift(Q, static_cast<long>(H) * L * d, seed, t, amplitude, Q_out, static_cast<cudaStream_t>(stream));
+}
+
+}  // extern "C"
+
+namespace {
+
+int run_steps_impl(const uint16_t* Q, const uint16_t* K, const uint16_t* V, int H, int L, int d,
+                   float scale, int bq, int bk, float keep_ratio, int budget_mode, int T,
+                   float warmup_frac, int refresh_every, int start_step, int end_step,
+                   int have_pattern, int32_t* kv_idx, int32_t* kv_count, int kv_stride, uint16_t* O,
+                   float* LSE, int8_t* step_kind, float* step_ms, void* workspace,
+                   size_t workspace_bytes, void* stream, const Drift* drift) {
   if (T < 0 || start_step < 0 || start_step > end_step || end_step > T) return SPARSED_ERR_INVALID_ARG;
   std::vector<int8_t> kinds(static_cast<size_t>(T) + 1);
   SP_TRY(sparsed_schedule(T, warmup_frac, refresh_every, kinds.data()));
@@ -725,7 +837,11 @@ int sparsed_run_steps_span(const uint16_t* Q, const uint16_t* K, const uint16_t*
     SP_CUDA(cudaEventRecord(ev[0], st));
   }
   int rc = SPARSED_OK;
+  if (drift) p.Q = drift->q_step;  // every step attends with its own queries
   for (int t = start_step; t < end_step && rc == SPARSED_OK; ++t) {
+    if (drift) rc = launch_drift(Q, static_cast<long>(p.H) * p.L * p.d, drift->seed, t, drift->amplitude,
+                                 drift->q_step, st);
+    if (rc != SPARSED_OK) break;
     switch (kinds[t]) {
       case SPARSED_STEP_DENSE:
         rc = launch_attn(p, false, nullptr, nullptr, 0, st);
@@ -773,6 +889,10 @@ int sparsed_run_steps_span(const uint16_t* Q, const uint16_t* K, const uint16_t*
   }
   return rc;
 }
+
+}  // namespace
+
+extern "C" {
 
 // ---- head-sharded entropy budget (the heads of one layer split over ranks)
 

@@ -226,6 +226,52 @@ int sparsed_run_steps_span(const uint16_t* Q, const uint16_t* K, const uint16_t*
                            int8_t* step_kind, float* step_ms,
                            void* workspace, size_t workspace_bytes, void* stream);
 
+/* ---- Queries that change across the denoising steps.
+ *
+ * The pages give no per-step activations; attention patterns stay similar
+ * across steps (SparseD abstract) and are only locally consistent, shifting at
+ * some transitions (Step-dLLM abstract). These entry points give every step t
+ * its own queries, a seeded perturbation of Q with the same bits on any
+ * machine:
+ *   Q_t = bf16(fp32(Q) + fp32(amplitude * u)), elementwise (nearest even),
+ *   u   = (fmix32(i ^ key) >> 8) * 2^-23 - 1, in [-1, 1) on a 2^-23 grid,
+ *   key = fmix32(fmix32(seed) ^ t),
+ * where i is the element's row-major index in [H, L, d] and fmix32 is the
+ * MurmurHash3 32-bit finalizer (h ^= h>>16; h *= 0x85ebca6b; h ^= h>>13;
+ * h *= 0xc2b2ae35; h ^= h>>16). The product and the sum are rounded once
+ * each. */
+
+/* Q_out = Q_t for step t (device pointers, [H, L, d] bf16, 16-byte aligned;
+ * Q_out may not overlap Q). Returns SPARSED_ERR_INVALID_ARG for null or
+ * misaligned pointers, t < 0 or a non-finite amplitude,
+ * SPARSED_ERR_UNSUPPORTED for d not in {64, 128} or H*L*d >= 2^31. Asynchronous
+ * on `stream`. */
+int sparsed_drift_queries(const uint16_t* Q, int H, int L, int d, unsigned int seed, int t,
+                          float amplitude, uint16_t* Q_out, void* stream);
+
+/* sparsed_run_steps_span with per-step queries: before step t the driver
+ * writes Q_t (sparsed_drift_queries with drift_seed, drift_amplitude) into
+ * Q_step (caller memory, [H, L, d] bf16, 16-byte aligned, not overlapping the
+ * other arrays) and runs the step on Q_step, K and V. A SELECT step that uses
+ * the fused block mass (the workspace of sparsed_run_steps_workspace_bytes,
+ * an earlier full pass in the span) weights each row's probabilities with the
+ * LSE of that earlier pass, computed on earlier queries: each row's masses
+ * are then scaled by exp(lse_now - lse_then), so the selection equals the
+ * separate pass's wherever the relative gap between the k-th and (k+1)-th
+ * block mass exceeds 1 - exp(-2 * max |lse_now - lse_then|). Errors as
+ * sparsed_run_steps_span, and SPARSED_ERR_INVALID_ARG for a null or misaligned
+ * Q_step or a non-finite amplitude. */
+int sparsed_run_steps_drift(const uint16_t* Q, const uint16_t* K, const uint16_t* V,
+                            int H, int L, int d, float scale, int bq, int bk,
+                            float keep_ratio, int budget_mode,
+                            int T, float warmup_frac, int refresh_every,
+                            int start_step, int end_step, int have_pattern,
+                            unsigned int drift_seed, float drift_amplitude, uint16_t* Q_step,
+                            int32_t* kv_idx, int32_t* kv_count, int kv_stride,
+                            uint16_t* O, float* LSE,
+                            int8_t* step_kind, float* step_ms,
+                            void* workspace, size_t workspace_bytes, void* stream);
+
 /* ---- Head-sharded selection with the entropy budget (the heads of one
  * layer split over several GPUs: only the per-head entropies cross ranks, one
  * all-gather of H doubles per selection; Step-dLLM abstract: head-adaptive

@@ -303,3 +303,26 @@ def test_losa_init_validation():
     assert _losa_init(ws_bytes=1 << 10) == _lib.ERR_WORKSPACE
     if not GPU:
         assert _losa_init() == _lib.ERR_NO_DEVICE
+
+
+def test_drift_entry_points_validate_on_the_host():
+    f = lib.sparsed_drift_queries
+    assert f(None, 2, 64, 64, 1, 0, 0.0156, P, None) == _lib.ERR_INVALID_ARG
+    assert f(P, 2, 64, 64, 1, 0, 0.0156, None, None) == _lib.ERR_INVALID_ARG
+    assert f(MIS, 2, 64, 64, 1, 0, 0.0156, P, None) == _lib.ERR_INVALID_ARG
+    assert f(P, 2, 64, 64, 1, -1, 0.0156, P, None) == _lib.ERR_INVALID_ARG
+    assert f(P, 2, 64, 64, 1, 0, float("nan"), P, None) == _lib.ERR_INVALID_ARG
+    assert f(P, 2, 64, 96, 1, 0, 0.0156, P, None) == _lib.ERR_UNSUPPORTED
+    assert f(P, 0, 64, 64, 1, 0, 0.0156, P, None) == _lib.OK          # empty: nothing to do
+    if not GPU:
+        assert f(P, 2, 64, 64, 1, 0, 0.0156, P, None) == _lib.ERR_NO_DEVICE
+    g = lib.sparsed_run_steps_drift
+
+    def run(q_step=P, amp=0.0156):
+        return g(P, P, P, 2, 1024, 64, 0.125, 64, 64, 0.25, 0, 4, 0.5, 0, 0, 4, 0, 7, amp, q_step,
+                 P, P, 4, P, P, None, None, P, 1 << 30, None)
+    assert run(q_step=None) == _lib.ERR_INVALID_ARG
+    assert run(q_step=MIS) == _lib.ERR_INVALID_ARG
+    assert run(amp=float("inf")) == _lib.ERR_INVALID_ARG
+    if not GPU:
+        assert run() == _lib.ERR_NO_DEVICE
