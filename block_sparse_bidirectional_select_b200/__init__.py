@@ -51,7 +51,7 @@ __all__ = ["dense_attn", "select_pattern", "block_sparse_attn", "run_steps", "wo
            "RunResult", "default_scale", "column_keep", "column_workspace_bytes", "select_columns",
            "column_sparse_attn", "run_steps_columns", "ColumnPattern", "select_head_entropy",
            "entropy_budget", "select_with_head_k", "select_pattern_sharded", "gather_head_entropies",
-           "run_steps_sharded", "step_segments",
+           "run_steps_sharded",
            "losa_splits", "losa_workspace_bytes", "losa_init", "losa_step", "losa_block", "BlockState",
            "LosaStep", "LosaBlock"]
 
@@ -596,52 +596,73 @@ def losa_block(qs, ks, vs, k_pre, v_pre, n_sel=2, tau=0.01, scale=None, bq=64, b
 
 # ---------------------------------------------------------------- head-sharded denoising loop
 
-def step_segments(kinds):
-    """The schedule cut at its SELECT steps: a list of ("select", t) and
-    ("span", t0, t1) entries in step order, spans holding no SELECT step."""
-    segs, t0 = [], 0
-    for t, kind in enumerate(kinds):
-        if kind == STEP_SELECT:
-            if t > t0:
-                segs.append(("span", t0, t))
-            segs.append(("select", t))
-            t0 = t + 1
-    if t0 < len(kinds):
-        segs.append(("span", t0, len(kinds)))
-    return segs
+_EXCHANGE_FN = ctypes.CFUNCTYPE(ctypes.c_int, ctypes.POINTER(ctypes.c_double), ctypes.c_int,
+                                ctypes.POINTER(ctypes.c_double), ctypes.c_int, ctypes.c_void_p)
 
 
 def run_steps_sharded(q, k, v, T, warmup_frac=0.2, keep=0.1, budget="entropy", refresh_every=0, group=None,
                       scale=None, bq=128, bk=128, out=None, lse=None, workspace=None, stream=None,
-                      gather=None) -> RunResult:
+                      gather=None, rank=None, world=None) -> RunResult:
     """The denoising loop for this rank's heads of a layer whose heads are
-    split evenly over the ranks of ``group`` (rank order = head order).
+    split evenly over the ranks of ``group`` (rank order = head order), run by
+    the C driver sparsed_run_steps_sharded.
 
-    A uniform budget is per head, so the loop is run_steps on the local heads
-    and nothing crosses ranks. The entropy budget spans every head of the
-    layer: each SELECT step is select_pattern_sharded (full pass, per-head
-    entropies, one all-gather of H values, the allocation on every rank, local
-    top-k), and the steps between run through sparsed_run_steps_span with the
-    pattern so far. ``gather`` as in select_pattern_sharded."""
+    A uniform budget is per head, so nothing crosses ranks. The entropy budget
+    spans every head of the layer: at each SELECT step the driver calls back
+    here with the local per-head entropies, which are all-gathered over
+    ``group`` (gather_head_entropies: NCCL for device tensors, other backends
+    host tensors). ``gather`` (optional, with ``rank`` and ``world``) replaces
+    the all-gather: a function from this rank's entropies (a CPU fp64 tensor)
+    to (all entropies in head order as a CPU tensor, this rank's index).
+    Without a group or gather the local heads are the whole layer."""
     H, L, d = _check_qkv(q, k, v)
     scale = default_scale(d) if scale is None else scale
-    if budget == "uniform":
-        return run_steps(q, k, v, T, warmup_frac, keep, "uniform", refresh_every, scale, bq, bk, out=out,
-                         lse=lse, workspace=workspace, stream=stream)
-    if budget != "entropy":
-        raise ValueError(f"unknown budget {budget!r}")
+    mode = {"uniform": BUDGET_UNIFORM, "entropy": BUDGET_ENTROPY}[budget]
+    if group is not None:
+        import torch.distributed as dist
+        rank, world = dist.get_rank(group), dist.get_world_size(group)
+    elif gather is None:
+        rank, world = 0, 1
+    elif rank is None or world is None:
+        raise ValueError("a custom gather needs this rank's index and the number of ranks")
+    nqb, nkb = -(-L // bq), -(-L // bk)
     out, lse = _alloc_out(q, out, lse)
     if workspace is None:
         workspace = torch.empty(run_steps_workspace_bytes(H, L, bq, bk), dtype=torch.uint8, device=q.device)
-    kinds = schedule(T, warmup_frac, refresh_every)
-    kv_idx = kv_count = None
-    for seg in step_segments(kinds):
-        if seg[0] == "select":
-            pat = select_pattern_sharded(q, k, v, keep, group, scale, bq, bk, workspace, stream, out, lse, gather)
-            kv_idx, kv_count = pat.kv_idx, pat.kv_count
-        else:
-            _, t0, t1 = seg
-            run_steps(q, k, v, T, warmup_frac, keep, "entropy", refresh_every, scale, bq, bk, start_step=t0,
-                      pattern=None if kv_idx is None else (kv_idx, kv_count), out=out, lse=lse,
-                      workspace=workspace, stream=stream, end_step=t1)
-    return RunResult(out, lse, kinds, None, kv_idx, kv_count)
+    stride = uniform_keep(L, bk, keep) if (mode == BUDGET_UNIFORM and L > 0) else max(nkb, 1)
+    kv_idx = torch.full((H, nqb, stride), -1, dtype=torch.int32, device=q.device)
+    kv_count = torch.zeros((H, nqb), dtype=torch.int32, device=q.device)
+    kinds = (ctypes.c_int8 * max(T, 1))()
+    errors = []
+
+    def exchange(local_ptr, h_local, all_ptr, h_total, _user):
+        try:
+            local = torch.tensor([local_ptr[i] for i in range(h_local)], dtype=torch.float64)
+            if gather is not None:
+                ent_all, _ = gather(local)
+            elif group is not None:
+                import torch.distributed as dist
+                mine = local.to(q.device) if dist.get_backend(group) == "nccl" else local
+                ent_all, _ = gather_head_entropies(mine, group)
+            else:
+                ent_all = local
+            vals = [float(x) for x in ent_all]
+            if len(vals) != h_total:
+                raise ValueError(f"gathered {len(vals)} head entropies, the layer has {h_total}")
+            for i, x in enumerate(vals):
+                all_ptr[i] = x
+            return 0
+        except Exception as e:  # reported after the C call returns
+            errors.append(e)
+            return 1
+
+    cb = _EXCHANGE_FN(exchange)
+    rc = _lib.load().sparsed_run_steps_sharded(
+        _ptr(q), _ptr(k), _ptr(v), H, L, d, scale, bq, bk, keep, mode, H * world, H * rank, T, warmup_frac,
+        refresh_every, _ptr(kv_idx), _ptr(kv_count), kv_idx.shape[2], _ptr(out), _ptr(lse),
+        ctypes.cast(kinds, ctypes.c_void_p), ctypes.cast(cb, ctypes.c_void_p), None, _ptr(workspace),
+        workspace.numel(), _stream(stream))
+    if errors:
+        raise errors[0]
+    check(rc, "sparsed_run_steps_sharded")
+    return RunResult(out, lse, list(kinds[:T]), None, kv_idx, kv_count)

@@ -19,6 +19,7 @@ ERR_BAD_PATTERN = -4
 ERR_CUDA = -5
 ERR_DEVICE_TIMEOUT = -6
 ERR_NO_DEVICE = -7
+ERR_EXCHANGE = -8
 
 BUDGET_UNIFORM = 0
 BUDGET_ENTROPY = 1
@@ -49,6 +50,8 @@ SIGNATURES = {
                                _I, _P, _P, _P, _P, _P, _SZ, _P]),
     "sparsed_run_steps_workspace_bytes": (_I, [_I, _I, _I, _I, ctypes.POINTER(_SZ)]),
     "sparsed_drift_queries": (_I, [_P, _I, _I, _I, ctypes.c_uint, _I, _F, _P, _P]),
+    "sparsed_run_steps_sharded": (_I, [_P, _P, _P, _I, _I, _I, _F, _I, _I, _F, _I, _I, _I, _I, _F, _I, _P, _P,
+                                       _I, _P, _P, _P, _P, _P, _P, _SZ, _P]),
     "sparsed_run_steps_drift": (_I, [_P, _P, _P, _I, _I, _I, _F, _I, _I, _F, _I, _I, _F, _I, _I, _I, _I,
                                      ctypes.c_uint, _F, _P, _P, _P, _I, _P, _P, _P, _P, _P, _SZ, _P]),
     "sparsed_run_steps_span": (_I, [_P, _P, _P, _I, _I, _I, _F, _I, _I, _F, _I, _I, _F, _I, _I, _I, _I, _P,

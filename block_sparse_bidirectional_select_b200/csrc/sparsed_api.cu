@@ -629,6 +629,7 @@ const char* sparsed_strerror(int status) {
     case SPARSED_ERR_CUDA: return "CUDA runtime error (see sparsed_last_cuda_error)";
     case SPARSED_ERR_DEVICE_TIMEOUT: return "a bounded device-side wait expired";
     case SPARSED_ERR_NO_DEVICE: return "no sm_100 (B200) device is current";
+    case SPARSED_ERR_EXCHANGE: return "the exchange callback of the head-sharded loop failed";
     default: return "unknown status";
   }
 }
@@ -950,6 +951,64 @@ int sparsed_select_with_head_k(int H, int L, int bq, int bk, const int32_t* head
   topk_kernel<<<(rows + 7) / 8, 256, 0, static_cast<cudaStream_t>(stream)>>>(mass, rows, nqb, nkb, 0, head_k,
                                                                               nullptr, kv_idx, kv_count, kv_stride);
   SP_CUDA(cudaGetLastError());
+  return SPARSED_OK;
+}
+
+int sparsed_run_steps_sharded(const uint16_t* Q, const uint16_t* K, const uint16_t* V, int H, int L, int d,
+                              float scale, int bq, int bk, float keep_ratio, int budget_mode, int h_total,
+                              int head_offset, int T, float warmup_frac, int refresh_every, int32_t* kv_idx,
+                              int32_t* kv_count, int kv_stride, uint16_t* O, float* LSE, int8_t* step_kind,
+                              sparsed_exchange_fn exchange, void* user, void* workspace, size_t workspace_bytes,
+                              void* stream) {
+  if (h_total < H || head_offset < 0 || head_offset > h_total - H || T < 0) return SPARSED_ERR_INVALID_ARG;
+  if (budget_mode == SPARSED_BUDGET_UNIFORM)
+    return run_steps_impl(Q, K, V, H, L, d, scale, bq, bk, keep_ratio, budget_mode, T, warmup_frac, refresh_every,
+                          0, T, 0, kv_idx, kv_count, kv_stride, O, LSE, step_kind, nullptr, workspace,
+                          workspace_bytes, stream, nullptr);
+  if (budget_mode != SPARSED_BUDGET_ENTROPY || !exchange) return SPARSED_ERR_INVALID_ARG;
+  if (!(keep_ratio > 0.f && keep_ratio <= 1.f)) return SPARSED_ERR_INVALID_ARG;
+  std::vector<int8_t> kinds(static_cast<size_t>(T) + 1);
+  SP_TRY(sparsed_schedule(T, warmup_frac, refresh_every, kinds.data()));
+  if (step_kind && T > 0) std::memcpy(step_kind, kinds.data(), static_cast<size_t>(T));
+  Problem p;
+  bool empty = false;
+  SP_TRY(prepare(Q, K, V, H, L, d, scale, bq, bk, O, LSE, &p, &empty));
+  if (empty) return SPARSED_OK;
+  SP_TRY(check_select_args(p, keep_ratio, budget_mode, kv_idx, kv_count, kv_stride, workspace, workspace_bytes));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const Workspace w = ws_layout(p.H, p.nqb, p.nkb);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  double* ent_dev = reinterpret_cast<double*>(ws + w.scratch);  // H doubles of the budget scratch
+  int32_t* k_dev = reinterpret_cast<int32_t*>(ws + w.headk);
+  std::vector<double> ent_local(static_cast<size_t>(H)), ent_all(static_cast<size_t>(h_total));
+  std::vector<double> scratch(static_cast<size_t>(h_total) * 3);
+  std::vector<int32_t> k_all(static_cast<size_t>(h_total));
+  bool have_pattern = false;
+  int t0 = 0;
+  for (int t = 0; t <= T; ++t) {
+    if (t < T && kinds[t] != SPARSED_STEP_SELECT) continue;
+    if (t > t0)  // the steps before this SELECT (or the end): no selection among them
+      SP_TRY(run_steps_impl(Q, K, V, H, L, d, scale, bq, bk, keep_ratio, budget_mode, T, warmup_frac,
+                            refresh_every, t0, t, have_pattern ? 1 : 0, kv_idx, kv_count, kv_stride, O, LSE,
+                            nullptr, nullptr, workspace, workspace_bytes, stream, nullptr));
+    if (t == T) break;
+    SP_TRY(sparsed_select_head_entropy(Q, K, V, H, L, d, scale, bq, bk, O, LSE, ent_dev, workspace,
+                                       workspace_bytes, stream));
+    SP_CUDA(cudaMemcpyAsync(ent_local.data(), ent_dev, static_cast<size_t>(H) * sizeof(double),
+                            cudaMemcpyDeviceToHost, st));
+    SP_CUDA(cudaStreamSynchronize(st));
+    if (exchange(ent_local.data(), H, ent_all.data(), h_total, user) != 0) return SPARSED_ERR_EXCHANGE;
+    allocate_budget(ent_all.data(), h_total, p.nkb, keep_ratio, scratch.data(), scratch.data() + h_total,
+                    scratch.data() + 2 * h_total, k_all.data());
+    SP_CUDA(cudaMemcpyAsync(k_dev, k_all.data() + head_offset, static_cast<size_t>(H) * sizeof(int32_t),
+                            cudaMemcpyHostToDevice, st));
+    SP_TRY(sparsed_select_with_head_k(H, L, bq, bk, k_dev, kv_idx, kv_count, kv_stride, workspace, workspace_bytes,
+                                      stream));
+    // k_all is reused at the next selection only after this one's copy has run
+    SP_CUDA(cudaStreamSynchronize(st));
+    have_pattern = true;
+    t0 = t + 1;
+  }
   return SPARSED_OK;
 }
 

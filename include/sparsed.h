@@ -71,7 +71,8 @@ enum {
   SPARSED_ERR_BAD_PATTERN = -4,    /* a pattern entry out of range / not ascending (device) */
   SPARSED_ERR_CUDA = -5,           /* a CUDA runtime call failed; see sparsed_last_cuda_error */
   SPARSED_ERR_DEVICE_TIMEOUT = -6, /* a bounded device-side wait expired */
-  SPARSED_ERR_NO_DEVICE = -7       /* no sm_100 device is current */
+  SPARSED_ERR_NO_DEVICE = -7,      /* no sm_100 device is current */
+  SPARSED_ERR_EXCHANGE = -8        /* the caller's exchange callback returned nonzero */
 };
 
 enum { SPARSED_BUDGET_UNIFORM = 0, SPARSED_BUDGET_ENTROPY = 1 };
@@ -225,6 +226,48 @@ int sparsed_run_steps_span(const uint16_t* Q, const uint16_t* K, const uint16_t*
                            uint16_t* O, float* LSE,
                            int8_t* step_kind, float* step_ms,
                            void* workspace, size_t workspace_bytes, void* stream);
+
+/* The exchange of the head-sharded loop, supplied by the caller (an
+ * all-gather over the ranks that hold the heads of one layer). It is called on
+ * the host at every selecting step with this rank's h_local per-head
+ * entropies (host memory, fp64) and must fill all_entropy with the h_total
+ * entropies of the layer in head order (host memory), then return 0. Any
+ * other return value stops the loop with SPARSED_ERR_EXCHANGE. */
+typedef int (*sparsed_exchange_fn)(const double* local_entropy, int h_local, double* all_entropy, int h_total,
+                                   void* user);
+
+/* The denoising loop for this rank's heads of a layer whose h_total heads are
+ * split over ranks (Step-dLLM abstract: a head-adaptive global budget spans
+ * the heads of a layer). This rank holds heads [head_offset, head_offset + H)
+ * of Q, K, V ([H, L, d], as sparsed_run_steps).
+ *   - budget_mode SPARSED_BUDGET_UNIFORM: every head's budget is its own, so
+ *     the loop is sparsed_run_steps on the local heads; exchange is not
+ *     called and may be null.
+ *   - SPARSED_BUDGET_ENTROPY: the loop is cut at its SELECT steps. Steps
+ *     between them run as sparsed_run_steps_span. Each SELECT step runs as
+ *     follows:
+ *       1. the full pass, the block mass and the mean row entropy of each
+ *          local head (sparsed_select_head_entropy);
+ *       2. the entropies are copied to the host (a stream synchronisation);
+ *       3. exchange(...) gathers all h_total entropies;
+ *       4. the allocation of sparsed_entropy_budget over all heads;
+ *       5. top-k with this rank's k_h (sparsed_select_with_head_k).
+ *     Every rank reaches the same allocation from the same gathered
+ *     entropies.
+ * kv_idx / kv_count: the pattern cache, [H, nqb, kv_stride] / [H, nqb] int32,
+ * kv_stride >= nkb for the entropy budget. step_kind: nullable [T]. The
+ * workspace: sparsed_workspace_bytes(H, L, bq, bk) bytes, 256-byte aligned,
+ * for the entropy budget. Returns the first failing call's status,
+ * SPARSED_ERR_INVALID_ARG for inconsistent head counts or a null exchange with
+ * the entropy budget, SPARSED_ERR_EXCHANGE when the callback fails. */
+int sparsed_run_steps_sharded(const uint16_t* Q, const uint16_t* K, const uint16_t* V,
+                              int H, int L, int d, float scale, int bq, int bk,
+                              float keep_ratio, int budget_mode, int h_total, int head_offset,
+                              int T, float warmup_frac, int refresh_every,
+                              int32_t* kv_idx, int32_t* kv_count, int kv_stride,
+                              uint16_t* O, float* LSE, int8_t* step_kind,
+                              sparsed_exchange_fn exchange, void* user,
+                              void* workspace, size_t workspace_bytes, void* stream);
 
 /* ---- Queries that change across the denoising steps.
  *

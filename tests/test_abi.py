@@ -326,3 +326,20 @@ def test_drift_entry_points_validate_on_the_host():
     assert run(amp=float("inf")) == _lib.ERR_INVALID_ARG
     if not GPU:
         assert run() == _lib.ERR_NO_DEVICE
+
+
+def test_sharded_loop_validates_on_the_host():
+    f = lib.sparsed_run_steps_sharded
+
+    def run(budget=1, h_total=4, offset=2, exchange=P):
+        return f(P, P, P, 2, 1024, 64, 0.125, 64, 64, 0.25, budget, h_total, offset, 8, 0.3, 2,
+                 P, P, 16, P, P, None, exchange, None, P, 1 << 30, None)
+    assert run(h_total=1) == _lib.ERR_INVALID_ARG          # fewer heads in the layer than here
+    assert run(offset=3) == _lib.ERR_INVALID_ARG           # heads past the layer's end
+    assert run(offset=-1) == _lib.ERR_INVALID_ARG
+    assert run(exchange=None) == _lib.ERR_INVALID_ARG      # the entropy budget needs the exchange
+    assert run(budget=5) == _lib.ERR_INVALID_ARG
+    assert lib.sparsed_strerror(_lib.ERR_EXCHANGE).decode().startswith("the exchange callback")
+    if not GPU:
+        assert run() == _lib.ERR_NO_DEVICE
+        assert run(budget=0, exchange=None) == _lib.ERR_NO_DEVICE

@@ -105,22 +105,6 @@ def test_two_shards_on_one_gpu_equal_the_unsharded_selection():
         assert torch.equal(lse, full.lse[s])
 
 
-def test_step_segments_cut_the_schedule_at_select_steps():
-    kinds = sp.schedule(10, 0.3, 3)
-    assert kinds == [0, 0, 1, 2, 2, 1, 2, 2, 1, 2]
-    assert sp.step_segments(kinds) == [("span", 0, 2), ("select", 2), ("span", 3, 5), ("select", 5),
-                                       ("span", 6, 8), ("select", 8), ("span", 9, 10)]
-    assert sp.step_segments(sp.schedule(4, 1.0, 0)) == [("span", 0, 4)]          # all dense, no select
-    assert sp.step_segments(sp.schedule(5, 0.2, 0)) == [("select", 0), ("span", 1, 5)]
-    assert sp.step_segments([]) == []
-    # every step is covered once, in order
-    for T, w, r in [(1, 0.0, 0), (7, 0.5, 1), (256, 0.2, 0), (512, 0.2, 64)]:
-        steps = []
-        for seg in sp.step_segments(sp.schedule(T, w, r)):
-            steps += [seg[1]] if seg[0] == "select" else list(range(seg[1], seg[2]))
-        assert steps == list(range(T))
-
-
 @pytest.mark.gpu
 def test_sharded_denoising_loop_two_shards_in_two_threads():
     """Two ranks emulated by two host threads on one GPU (each its own stream;
@@ -156,7 +140,8 @@ def test_sharded_denoising_loop_two_shards_in_two_threads():
             with torch.cuda.stream(s):
                 sl = shards[rank]
                 res = sp.run_steps_sharded(q[sl].contiguous(), k[sl].contiguous(), v[sl].contiguous(), T, w,
-                                           keep, "entropy", r, stream=s, gather=make_gather(rank))
+                                           keep, "entropy", r, stream=s, gather=make_gather(rank), rank=rank,
+                                           world=2)
                 s.synchronize()
                 results[rank] = res
         except Exception as e:  # reported below; the barrier times out for the other thread
