@@ -315,6 +315,9 @@ def main():
                          "with the column-sparse pattern; losa: block-wise generation over a prefix cache "
                          "with active-token reuse (--block-workload)")
     ap.add_argument("--block-workload", default="losa_32k", choices=sorted(BLOCK_WORKLOADS))
+    ap.add_argument("--warmup-frac", type=float, default=None,
+                    help="override the workload's dense warm-up fraction w (e.g. 0.05: the column or block "
+                         "pattern applied from earlier denoising steps)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     rank = int(os.environ.get("RANK", "0"))
@@ -339,6 +342,8 @@ def main():
         return reduce_max(x, world, dev)
 
     wl = WORKLOADS[args.workload]
+    if args.warmup_frac is not None:
+        wl = wl.scaled(warmup_frac=args.warmup_frac)
     if args.op != "run":
         return time_one_op(args, wl, dev, rank)
     if args.path == "columns":
@@ -685,23 +690,39 @@ def run_losa(args, dev, rank, world, barrier, max_over_ranks):
     n_active = res.active.cpu().numpy().sum(axis=1)
     per_step_bytes = losa_bytes(wl, ucount)
     run_bytes = float(sum(per_step_bytes))
+    # the block run captured once in a CUDA graph (the library's side stream
+    # joins the capture through its fork / join events) and replayed: a later
+    # step is a handful of short dependent kernels, whose launch gaps the
+    # graph removes
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        one_run()
+    graph.replay()
+    torch.cuda.synchronize()
+    sp.device_check()
+
+    def timed(fn):
+        total = 0.0
+        for _ in range(args.steps):
+            flush.zero_()
+            s_ev = torch.cuda.Event(enable_timing=True)
+            e_ev = torch.cuda.Event(enable_timing=True)
+            s_ev.record(stream)
+            fn()
+            e_ev.record(stream)
+            e_ev.synchronize()
+            total += s_ev.elapsed_time(e_ev)
+        return total
+
     torch.cuda.synchronize()
     barrier()
     clocks = ClockSampler(dev.index or 0)
     clocks.start()
-    total = 0.0
-    for _ in range(args.steps):
-        flush.zero_()
-        s_ev = torch.cuda.Event(enable_timing=True)
-        e_ev = torch.cuda.Event(enable_timing=True)
-        s_ev.record(stream)
-        one_run()
-        e_ev.record(stream)
-        e_ev.synchronize()
-        total += s_ev.elapsed_time(e_ev)
+    total = timed(graph.replay)
     barrier()
     clk = clocks.stop()
     total_ms = max_over_ranks(total)
+    eager_ms = max_over_ranks(timed(one_run))
     sp.device_check()
     # the first (dense) step alone: 8 calls back to back (the GPU, not the
     # host, sets the pace: each reads the whole 0.5 GB prefix) between two
@@ -736,6 +757,9 @@ def run_losa(args, dev, rank, world, barrier, max_over_ranks):
                        "parallelism": f"independent blocks x{world}" if world > 1 else "single"},
             "ms_per_denoise_step": total_ms / args.steps / wl.T,
             "first_step_ms": first_ms, "later_step_ms": step_ms,
+            "timing": "block run replayed from a CUDA graph; eager launches beside it",
+            "ms_per_step_eager": eager_ms / args.steps,
+            "later_step_ms_eager": (eager_ms / args.steps - first_ms) / (wl.T - 1) if wl.T > 1 else None,
             "active_tokens_per_step": float(n_active[1:].mean()) if wl.T > 1 else None,
             "union_blocks_per_head": float(ucount[1:].mean()) if wl.T > 1 else None,
             "prefix_density": float(ucount[1:].mean()) / nkb if wl.T > 1 else None,
