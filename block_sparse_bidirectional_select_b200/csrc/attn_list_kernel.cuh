@@ -25,8 +25,10 @@
 //               t%16 and the column half t/16 of every S tile, so the two
 //               halves of a row meet in one warp (row max / sum by shuffle).
 //   warp 8      TMA producer: Q of each item, K_g / V_g into KS- / VS-deep rings
-//   warp 9      TMEM owner; its lane 0 issues the S = Q K^T MMAs
-//   warp 10     lane 0 issues the O += P V MMAs
+//   warp 9      TMEM owner; issues the S = Q K^T MMAs
+//   warp 10     issues the O += P V MMAs
+// (warps 8-10 run warp-uniform code; one elected lane issues each copy, MMA
+// and commit)
 //   warp 11     idle (donates its registers)
 // TMEM (128 lanes): [S0 | S1 | O | P0 | P1] = 2*BK + D + BK fp32 columns. S is
 // double-buffered, so S(g+1) is computed while the softmax works on S(g); P has
@@ -222,11 +224,20 @@ __global__ void __launch_bounds__(384, 1)
 
   if (warp >= 8) {
     setmaxnreg_dec_56();
-    if (warp == 8 && lane == 0) {
+    // The producer and the issuers run warp-uniform code (descriptors and
+    // counters stay in uniform registers); one elected lane issues each copy,
+    // MMA and commit.
+    const uint32_t leader = ptx::elect_one();
+    auto wait = [&](int idx, int parity) -> bool {
+      return ptx::mbar_wait_warp(bar(idx), parity & 1, abort_flag, a.timeout_ns, kErrTimeout);
+    };
+    if (warp == 8) {
       // ============================================================ producer
-      ptx::tma_prefetch_desc(&tm_q);
-      ptx::tma_prefetch_desc(&tm_k);
-      ptx::tma_prefetch_desc(&tm_v);
+      if (leader) {
+        ptx::tma_prefetch_desc(&tm_q);
+        ptx::tma_prefetch_desc(&tm_k);
+        ptx::tma_prefetch_desc(&tm_v);
+      }
       int g = 0, iq = 0;  // tile counter, Q tiles loaded so far
       int issued_k = 0, issued_v = 0;
       bool ok = true;
@@ -235,17 +246,17 @@ __global__ void __launch_bounds__(384, 1)
         n_raw_next = raw_count<SPARSE>(a, w + gridDim.x);
         const int h = w / a.nqb, qi = w - h * a.nqb;
         const ItemList<SPARSE> it = item_list<SPARSE>(a, w, n_raw);
-        if (SPARSE && n_raw != it.n) ptx::record_error(kErrBadPattern);
+        if (SPARSE && leader && n_raw != it.n) ptx::record_error(kErrBadPattern);
         if (it.n == 0) continue;
         // Q of this item once every S MMA of the previous item is complete
-        if (iq > 0 && !ptx::mbar_wait(bar(C::B_QEMPTY), (iq - 1) & 1, abort_flag, a.timeout_ns, kErrTimeout)) {
+        if (iq > 0 && !wait(C::B_QEMPTY, iq - 1)) {
           ok = false;
           break;
         }
-        ptx::mbar_arrive_expect_tx(bar(C::B_QFULL), C::Q_BYTES);
+        ptx::mbar_arrive_expect_tx_if(leader, bar(C::B_QFULL), C::Q_BYTES);
 #pragma unroll
         for (int c = 0; c < C::DCH; ++c)
-          ptx::tma_load_3d(sb + C::OFF_Q + c * C::Q_CHUNK, &tm_q, bar(C::B_QFULL), c * 64, qi * a.bq, h);
+          ptx::tma_load_3d_if(leader, sb + C::OFF_Q + c * C::Q_CHUNK, &tm_q, bar(C::B_QFULL), c * 64, qi * a.bq, h);
         ++iq;
         // list entries are read one tile ahead, off the copy-issue path
         int prev = -1, raw_next = it.raw(0);
@@ -253,33 +264,31 @@ __global__ void __launch_bounds__(384, 1)
           const int raw = raw_next;
           if (jj + 1 < it.n) raw_next = it.raw(jj + 1);
           if constexpr (SPARSE) {
-            if (raw < 0 || raw >= a.nkb || raw <= prev) ptx::record_error(kErrBadPattern);
+            if (leader && (raw < 0 || raw >= a.nkb || raw <= prev)) ptx::record_error(kErrBadPattern);
             prev = raw;
           }
           const int j = (raw >= 0 && raw < a.nkb) ? raw : 0;
           const int ks = g % C::KS;
-          if (g >= C::KS &&
-              !ptx::mbar_wait(bar(C::B_KEMPTY + ks), (g / C::KS - 1) & 1, abort_flag, a.timeout_ns, kErrTimeout)) {
+          if (g >= C::KS && !wait(C::B_KEMPTY + ks, g / C::KS - 1)) {
             ok = false;
             break;
           }
-          ptx::mbar_arrive_expect_tx(bar(C::B_KFULL + ks), C::KV_BYTES);
+          ptx::mbar_arrive_expect_tx_if(leader, bar(C::B_KFULL + ks), C::KV_BYTES);
 #pragma unroll
           for (int c = 0; c < C::DCH; ++c)
-            ptx::tma_load_3d(sb + C::OFF_K + ks * C::KV_BYTES + c * C::KV_CHUNK, &tm_k, bar(C::B_KFULL + ks),
-                             c * 64, j * BK, h);
+            ptx::tma_load_3d_if(leader, sb + C::OFF_K + ks * C::KV_BYTES + c * C::KV_CHUNK, &tm_k,
+                                bar(C::B_KFULL + ks), c * 64, j * BK, h);
           issued_k = g + 1;
           const int vs = g % C::VS;
-          if (g >= C::VS &&
-              !ptx::mbar_wait(bar(C::B_VEMPTY + vs), (g / C::VS - 1) & 1, abort_flag, a.timeout_ns, kErrTimeout)) {
+          if (g >= C::VS && !wait(C::B_VEMPTY + vs, g / C::VS - 1)) {
             ok = false;
             break;
           }
-          ptx::mbar_arrive_expect_tx(bar(C::B_VFULL + vs), C::KV_BYTES);
+          ptx::mbar_arrive_expect_tx_if(leader, bar(C::B_VFULL + vs), C::KV_BYTES);
 #pragma unroll
           for (int c = 0; c < C::DCH; ++c)
-            ptx::tma_load_3d(sb + C::OFF_V + vs * C::KV_BYTES + c * C::KV_CHUNK, &tm_v, bar(C::B_VFULL + vs),
-                             c * 64, j * BK, h);
+            ptx::tma_load_3d_if(leader, sb + C::OFF_V + vs * C::KV_BYTES + c * C::KV_CHUNK, &tm_v,
+                                bar(C::B_VFULL + vs), c * 64, j * BK, h);
           issued_v = g + 1;
         }
       }
@@ -293,8 +302,9 @@ __global__ void __launch_bounds__(384, 1)
           ptx::mbar_wait(bar(C::B_KFULL + u % C::KS), (u / C::KS) & 1, &dummy, short_ns, 0);
         for (int u = (issued_v > C::VS ? issued_v - C::VS : 0); u < issued_v; ++u)
           ptx::mbar_wait(bar(C::B_VFULL + u % C::VS), (u / C::VS) & 1, &dummy, short_ns, 0);
+        __syncwarp();
       }
-    } else if (warp == 9 && lane == 0) {
+    } else if (warp == 9) {
       // ============================================================ S issuer
       constexpr uint32_t HI = ptx::sdesc_sw128_hi(1024);
       const uint32_t qlo = ptx::sdesc_sw128_lo(sb + C::OFF_Q, 16);
@@ -306,16 +316,14 @@ __global__ void __launch_bounds__(384, 1)
         n_raw_next = raw_count<SPARSE>(a, w + gridDim.x);
         const ItemList<SPARSE> it = item_list<SPARSE>(a, w, n_raw);
         if (it.n == 0) continue;
-        if (!ptx::mbar_wait(bar(C::B_QFULL), iq & 1, abort_flag, a.timeout_ns, kErrTimeout)) {
+        if (!wait(C::B_QFULL, iq)) {
           ok = false;
           break;
         }
         for (int jj = 0; jj < it.n; ++jj, ++g) {
           const int b = g & 1;
           const int ks = g % C::KS;
-          if (!ptx::mbar_wait(bar(C::B_KFULL + ks), (g / C::KS) & 1, abort_flag, a.timeout_ns, kErrTimeout) ||
-              (g >= 2 &&
-               !ptx::mbar_wait(bar(C::B_PVDONE + b), ((g - 2) >> 1) & 1, abort_flag, a.timeout_ns, kErrTimeout))) {
+          if (!wait(C::B_KFULL + ks, g / C::KS) || (g >= 2 && !wait(C::B_PVDONE + b, (g - 2) >> 1))) {
             ok = false;
             break;
           }
@@ -326,22 +334,23 @@ __global__ void __launch_bounds__(384, 1)
           for (int kk = 0; kk < D / 16; ++kk) {
             const uint32_t ao = (kk >> 2) * (C::Q_CHUNK >> 4) + (kk & 3) * 2;
             const uint32_t bo = (kk >> 2) * (C::KV_CHUNK >> 4) + (kk & 3) * 2;
-            ptx::umma_ss_lohi(s_tmem, qlo + ao, b0 + bo, HI, C::IDESC_S, kk > 0 ? 1u : 0u);
+            ptx::umma_ss_lohi_if(leader, s_tmem, qlo + ao, b0 + bo, HI, C::IDESC_S, kk > 0 ? 1u : 0u);
           }
-          ptx::umma_commit(bar(C::B_SFULL + b));
-          ptx::umma_commit(bar(C::B_KEMPTY + ks));
+          ptx::umma_commit_if(leader, bar(C::B_SFULL + b));
+          ptx::umma_commit_if(leader, bar(C::B_KEMPTY + ks));
         }
         if (!ok) break;
         // every S MMA of this item read Q: the producer may refill it
-        ptx::umma_commit(bar(C::B_QEMPTY));
+        ptx::umma_commit_if(leader, bar(C::B_QEMPTY));
         ++iq;
       }
       if (!ok) {
-        ptx::umma_commit(bar(C::B_DRAIN));
+        ptx::umma_commit_if(leader, bar(C::B_DRAIN));
         volatile int dummy = 0;
         ptx::mbar_wait(bar(C::B_DRAIN), 0, &dummy, a.timeout_ns / 4, 0);
+        __syncwarp();
       }
-    } else if (warp == 10 && lane == 0) {
+    } else if (warp == 10) {
       // ============================================================ PV issuer
       constexpr uint32_t HI = ptx::sdesc_sw128_hi(1024);
       const uint32_t vlo = ptx::sdesc_sw128_lo(sb + C::OFF_V, C::KV_CHUNK);
@@ -354,8 +363,7 @@ __global__ void __launch_bounds__(384, 1)
         for (int jj = 0; jj < it.n; ++jj, ++g) {
           const int b = g & 1;
           const int vs = g % C::VS;
-          if (!ptx::mbar_wait(bar(C::B_PFULL + b), (g >> 1) & 1, abort_flag, a.timeout_ns, kErrTimeout) ||
-              !ptx::mbar_wait(bar(C::B_VFULL + vs), (g / C::VS) & 1, abort_flag, a.timeout_ns, kErrTimeout)) {
+          if (!wait(C::B_PFULL + b, g >> 1) || !wait(C::B_VFULL + vs, g / C::VS)) {
             ok = false;
             break;
           }
@@ -364,16 +372,17 @@ __global__ void __launch_bounds__(384, 1)
           const uint32_t p_tmem = tmem + (b ? C::TM_P1 : C::TM_P0);
 #pragma unroll
           for (int kk = 0; kk < BK / 16; ++kk)
-            ptx::umma_ts_lohi(tmem + C::TM_O, p_tmem + kk * 8, b0 + kk * (2048 >> 4), HI, C::IDESC_PV,
-                              (jj > 0 || kk > 0) ? 1u : 0u);
-          ptx::umma_commit(bar(C::B_VEMPTY + vs));
-          ptx::umma_commit(bar(C::B_PVDONE + b));
+            ptx::umma_ts_lohi_if(leader, tmem + C::TM_O, p_tmem + kk * 8, b0 + kk * (2048 >> 4), HI, C::IDESC_PV,
+                                 (jj > 0 || kk > 0) ? 1u : 0u);
+          ptx::umma_commit_if(leader, bar(C::B_VEMPTY + vs));
+          ptx::umma_commit_if(leader, bar(C::B_PVDONE + b));
         }
       }
       if (!ok) {
-        ptx::umma_commit(bar(C::B_DRAIN + 1));
+        ptx::umma_commit_if(leader, bar(C::B_DRAIN + 1));
         volatile int dummy = 0;
         ptx::mbar_wait(bar(C::B_DRAIN + 1), 0, &dummy, a.timeout_ns / 4, 0);
+        __syncwarp();
       }
     }
   } else {
