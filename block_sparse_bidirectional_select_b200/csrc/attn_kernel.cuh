@@ -17,10 +17,13 @@
 // softmax has stored that part of P, so it overlaps the rest of the
 // exponentials.
 //
-// Persistent CTAs: the grid holds one CTA per SM and CTA b takes the pairs
-// b, b + G, b + 2G, ... of the flattened (h, p) order (G = grid size), so the
-// CTAs resident at any moment cover consecutive query blocks of one head and
-// share its K/V tiles in L2. The pipelines run on across pair boundaries.
+// Persistent CTAs: the grid holds one CTA per SM and CTA b starts with pair b
+// of the flattened (h, p) order. Its later pairs are b + G, b + 2G, ... (G =
+// grid size) or, given a counter, the next unclaimed pair, so the CTAs
+// resident at any moment cover consecutive query blocks of at most two heads
+// and share their K/V tiles in L2. The producer takes each pair index and
+// publishes it to the other warps through shared memory (B_WFULL / B_WEMPTY).
+// The pipelines run on across pair boundaries.
 //
 // Warp roles (384 threads):
 //   warps 0-3   softmax of slot 0: warp w holds rows 32w..32w+31 of the tile,
@@ -78,6 +81,14 @@ struct AttnArgs {
   const float* lse_prev;
   float* mass_part;
   uint64_t timeout_ns;       // bound of every device-side wait
+  // Pair scheduling (two-tile kernel). sched == nullptr: CTA b takes pairs b,
+  // b + G, b + 2G, ... (G = grid size). Otherwise CTA b takes pair b first and
+  // then claims pair G + atomicAdd(sched, 1) until the pairs run out, so the
+  // pairs in flight stay a window of about G consecutive pairs however
+  // unevenly the CTAs progress. *sched must be 0 at launch; the kernel sets
+  // *sched_reset (nullable) to 0 for the next launch.
+  int* sched;
+  int* sched_reset;
 };
 
 __device__ __forceinline__ void setmaxnreg_inc_224() {
@@ -111,8 +122,11 @@ struct AttnCfg {
   static constexpr int B_PFULL = B_SFULL + 2;   // [2][NPV] 4 warp arrivals
   static constexpr int B_PVDONE = B_PFULL + 2 * NPV;  // [2]
   static constexpr int B_DRAIN = B_PVDONE + 2;  // [2]
-  static constexpr int NUM_BARS = B_DRAIN + 2;
-  static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;  // tmem slot, abort flag
+  static constexpr int B_WFULL = B_DRAIN + 2;   // [2] pair index published
+  static constexpr int B_WEMPTY = B_WFULL + 2;  // [2] pair index read by every consumer warp
+  static constexpr int N_WTAKERS = 10;          // softmax warps 0-7, MMA issuers 9-10
+  static constexpr int NUM_BARS = B_WEMPTY + 2;
+  static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;  // tmem slot, abort flag, pair index [2]
   static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;
   static constexpr int TM_S0 = 0;
   static constexpr int TM_S1 = BK;
@@ -180,11 +194,16 @@ __global__ void __launch_bounds__(384, 1)
   const int n_pairs = a.H * npairs_h;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
+  // the producer publishes each pair index it takes here, double-buffered
+  volatile int* pair_w = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 8);
   auto bar = [&](int idx) -> uint32_t { return sb + C::OFF_BAR + 8 * idx; };
 
   // ---- setup
   if (threadIdx.x == 0) {
+    if (a.sched_reset && blockIdx.x == 0) *a.sched_reset = 0;
     for (int s = 0; s < 2; ++s) {
+      ptx::mbar_init(bar(C::B_WFULL + s), 1);
+      ptx::mbar_init(bar(C::B_WEMPTY + s), C::N_WTAKERS);
       ptx::mbar_init(bar(C::B_QFULL + s), 1);
       ptx::mbar_init(bar(C::B_QEMPTY + s), 1);
       ptx::mbar_init(bar(C::B_SFULL + s), 1);
@@ -251,12 +270,36 @@ __global__ void __launch_bounds__(384, 1)
         else ++qn0;
         return true;
       };
-      for (int w = blockIdx.x; ok && w < n_pairs; w += gridDim.x) {
+      int np = 0;  // pair indices published
+      // publish pair index w (n_pairs: no more pairs) once every consumer
+      // warp has read the index published two before it
+      auto publish = [&](int w) -> bool {
+        const int b = np & 1;
+        if (np >= 2 && !wait(C::B_WEMPTY + b, (np >> 1) - 1)) return false;
+        if (leader) {
+          pair_w[b] = w;
+          ptx::mbar_arrive(bar(C::B_WFULL + b));
+        }
+        __syncwarp();
+        ++np;
+        return true;
+      };
+      int w = blockIdx.x;
+      while (ok) {
+        ok = publish(w < n_pairs ? w : n_pairs);
+        if (!ok || w >= n_pairs) break;
         const Pair pr = pair_of(a, w, npairs_h);
         h = pr.h;
+        // the CTA's next pair: the static stride, or a claim on the counter
+        int w_next = w + static_cast<int>(gridDim.x);
+        if (a.sched) {
+          int claim = 0;
+          if (leader) claim = atomicAdd(a.sched, 1);
+          w_next = static_cast<int>(gridDim.x) + __reduce_max_sync(0xffffffffu, claim);
+        }
         // the next pair's Q rows into L2 while this pair runs
-        if (leader && w + static_cast<int>(gridDim.x) < n_pairs) {
-          const Pair pn = pair_of(a, w + gridDim.x, npairs_h);
+        if (leader && w_next < n_pairs) {
+          const Pair pn = pair_of(a, w_next, npairs_h);
 #pragma unroll
           for (int c = 0; c < C::DCH; ++c) {
             ptx::tma_prefetch_3d(&tm_q, c * 64, pn.q0 * a.bq, pn.h);
@@ -270,6 +313,7 @@ __global__ void __launch_bounds__(384, 1)
           if (ok && pr.has1 && j == 0) ok = load_q(1, pr.q0 + 1);
           if (ok) ok = load_tile(&tm_v, j);
         }
+        w = w_next;
       }
       if (!ok) {
         // let the copies in flight land before the CTA's shared memory goes
@@ -303,7 +347,15 @@ __global__ void __launch_bounds__(384, 1)
       int tcnt = 0;     // tiles of this slot (PFULL phases)
       bool ok = true;
       auto commit = [&](int idx) { ptx::umma_commit_if(leader, bar(idx)); };
-      for (int w = blockIdx.x; ok && w < n_pairs; w += gridDim.x) {
+      for (int np = 0; ok; ++np) {
+        if (!wait(C::B_WFULL + (np & 1), np >> 1)) {
+          ok = false;
+          break;
+        }
+        const int w = pair_w[np & 1];
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive(bar(C::B_WEMPTY + (np & 1)));
+        if (w >= n_pairs) break;
         const Pair pr = pair_of(a, w, npairs_h);
         const bool mine = s == 0 || pr.has1;   // slot 1 idles on a pair without a second block
         const bool sole = !pr.has1;             // slot 0 then gives both commits of each tile
@@ -356,6 +408,7 @@ __global__ void __launch_bounds__(384, 1)
           if (sole) commit(C::B_EMPTY + sv % NST);
           ++tcnt;
         }
+        if (!ok) break;
       }
       if (!ok) {
         commit(C::B_DRAIN + s);
@@ -377,7 +430,15 @@ __global__ void __launch_bounds__(384, 1)
     const uint64_t scale2 = ptx::f32x2(sl2, sl2);
     int tcount = 0;  // tiles of this slot so far (SFULL / PVDONE phases)
     bool ok = true;
-    for (int w = blockIdx.x; ok && w < n_pairs; w += gridDim.x) {
+    for (int np = 0; ok; ++np) {
+      if (!ptx::mbar_wait_warp(bar(C::B_WFULL + (np & 1)), (np >> 1) & 1, abort_flag, a.timeout_ns, kErrTimeout)) {
+        ok = false;
+        break;
+      }
+      const int w = pair_w[np & 1];
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(bar(C::B_WEMPTY + (np & 1)));
+      if (w >= n_pairs) break;
       const Pair pr = pair_of(a, w, npairs_h);
       const int h = pr.h;
       const int qi = pr.q0 + slot;

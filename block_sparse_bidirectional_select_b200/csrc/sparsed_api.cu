@@ -233,11 +233,29 @@ struct Problem {
   float scale;
 };
 
+// Counter slots of the two-tile kernel's pair scheduler, in a caller's
+// workspace. Launch k of a sequence on one stream claims pairs from slot k % 2
+// and clears slot (k + 1) % 2 for launch k + 1; stream order has finished
+// launch k - 1, that slot's last user, by then. One memset clears the first
+// slot when the sequence starts. Without slots (base == nullptr) the kernel
+// takes its pairs by the static stride.
+struct PairSched {
+  int* base = nullptr;
+  int k = 0;
+};
+
+int begin_pair_sched(PairSched* ps, void* slots, cudaStream_t st) {
+  ps->base = static_cast<int*>(slots);
+  ps->k = 0;
+  if (ps->base) SP_CUDA(cudaMemsetAsync(ps->base, 0, 2 * sizeof(int), st));
+  return SPARSED_OK;
+}
+
 // The register split of the kernel (setmaxnreg) must be funded by its launch
 // register count; checked once per kernel before the first launch, so a raise
 // can never wait forever.
 template <int D, int BK, bool MASS>
-int launch_attn_t(const Problem& p, const float* lse_prev, float* mass_part, cudaStream_t st) {
+int launch_attn_t(const Problem& p, const float* lse_prev, float* mass_part, PairSched* ps, cudaStream_t st) {
   using C = AttnCfg<D, BK>;
   auto kern = attn_fwd_kernel<D, BK, MASS>;
   static int regs = -1;
@@ -267,15 +285,19 @@ int launch_attn_t(const Problem& p, const float* lse_prev, float* mass_part, cud
   a.lse_prev = lse_prev;
   a.mass_part = mass_part;
   a.timeout_ns = kWaitTimeoutNs;
+  const bool dyn = ps && ps->base;
+  a.sched = dyn ? ps->base + (ps->k & 1) : nullptr;
+  a.sched_reset = dyn ? ps->base + ((ps->k + 1) & 1) : nullptr;
   int sms = 0;
   SP_TRY(sm_count(&sms));
   SP_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES));
-  // persistent: one CTA per SM (its registers admit one), each walking the
-  // pairs of query blocks blockIdx.x, blockIdx.x + gridDim.x, ...
+  // persistent: one CTA per SM (its registers admit one); CTA b starts with
+  // pair b, then takes pairs by the static stride or from the counter
   const long pairs = static_cast<long>(p.H) * ((p.nqb + 1) / 2);
   const int grid = static_cast<int>(pairs < sms ? pairs : sms);
   kern<<<grid, C::THREADS, C::SMEM_BYTES, st>>>(tq, tk, tv, a);
   SP_CUDA(cudaGetLastError());
+  if (dyn) ++ps->k;
   return SPARSED_OK;
 }
 
@@ -313,6 +335,8 @@ int launch_list_t(const Problem& p, const int32_t* kv_idx, const int32_t* kv_cou
   a.lse_prev = nullptr;
   a.mass_part = nullptr;
   a.timeout_ns = kWaitTimeoutNs;
+  a.sched = nullptr;
+  a.sched_reset = nullptr;
   int sms = 0;
   SP_TRY(sm_count(&sms));
   SP_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES));
@@ -327,14 +351,16 @@ int launch_list_t(const Problem& p, const int32_t* kv_idx, const int32_t* kv_cou
 // Dense passes (and the fused selecting pass) run in the two-tile kernel,
 // block-sparse passes in the one-tile kernel. mass_part != nullptr selects the
 // fused variant (dense only): the pass also writes the block-mass partials,
-// using lse_prev as every row's LSE.
+// using lse_prev as every row's LSE. ps (nullable) gives the dense passes the
+// counter slots of their pair scheduler.
 int launch_attn(const Problem& p, bool sparse, const int32_t* kv_idx, const int32_t* kv_count,
-                int kv_stride, cudaStream_t st, const float* lse_prev = nullptr, float* mass_part = nullptr) {
+                int kv_stride, cudaStream_t st, const float* lse_prev = nullptr, float* mass_part = nullptr,
+                PairSched* ps = nullptr) {
 #define SP_ATTN(D_, BK_)                                                                                  \
   if (p.d == D_ && p.bk == BK_) {                                                                         \
     if (sparse) return launch_list_t<D_, BK_>(p, kv_idx, kv_count, kv_stride, st);                        \
-    if (mass_part) return launch_attn_t<D_, BK_, true>(p, lse_prev, mass_part, st);                     \
-    return launch_attn_t<D_, BK_, false>(p, nullptr, nullptr, st);                                        \
+    if (mass_part) return launch_attn_t<D_, BK_, true>(p, lse_prev, mass_part, ps, st);                 \
+    return launch_attn_t<D_, BK_, false>(p, nullptr, nullptr, ps, st);                                    \
   }
   SP_ATTN(64, 64)
   SP_ATTN(64, 128)
@@ -406,7 +432,7 @@ int launch_col_mass(const Problem& p, float* mass, cudaStream_t st) {
 }
 
 struct ColWorkspace {
-  size_t mass, ksel, vsel, total;
+  size_t mass, ksel, vsel, sched, total;
 };
 
 ColWorkspace col_ws_layout(int H, int L, int d, int kc) {
@@ -414,7 +440,8 @@ ColWorkspace col_ws_layout(int H, int L, int d, int kc) {
   w.mass = 0;
   w.ksel = align256(static_cast<size_t>(H) * L * sizeof(float));
   w.vsel = w.ksel + align256(static_cast<size_t>(H) * kc * d * 2);
-  w.total = w.vsel + align256(static_cast<size_t>(H) * kc * d * 2);
+  w.sched = w.vsel + align256(static_cast<size_t>(H) * kc * d * 2);
+  w.total = w.sched + align256(2 * sizeof(int32_t));  // the pair scheduler's counter slots
   return w;
 }
 
@@ -461,7 +488,7 @@ int column_attn(const Problem& p, const int32_t* cols, int kc, int col_stride, v
 }
 
 struct Workspace {
-  size_t grid, ent, scratch, headk, total;
+  size_t grid, ent, scratch, headk, sched, total;
 };
 
 Workspace ws_layout(int H, int nqb, int nkb) {
@@ -470,8 +497,8 @@ Workspace ws_layout(int H, int nqb, int nkb) {
   w.ent = w.grid + align256(static_cast<size_t>(H) * nqb * nkb * sizeof(float));
   w.scratch = w.ent + align256(static_cast<size_t>(H) * nqb * sizeof(double));
   w.headk = w.scratch + align256(static_cast<size_t>(H) * 4 * sizeof(double));
-  w.total = w.headk + align256(static_cast<size_t>(H) * sizeof(int32_t));
-  if (w.total == 0) w.total = 256;
+  w.sched = w.headk + align256(static_cast<size_t>(H) * sizeof(int32_t));
+  w.total = w.sched + align256(2 * sizeof(int32_t));  // the pair scheduler's counter slots
   return w;
 }
 
@@ -529,12 +556,12 @@ FusedWorkspace fused_ws_layout(int H, int L, int nqb, int nkb) {
 // LSE is taken from lse_prev, the LSE of an earlier full pass of the same
 // inputs (so it equals the LSE this pass computes).
 int fused_select(const Problem& p, float keep_ratio, int budget_mode, int32_t* kv_idx, int32_t* kv_count,
-                 int kv_stride, void* workspace, cudaStream_t st) {
+                 int kv_stride, void* workspace, PairSched* ps, cudaStream_t st) {
   const FusedWorkspace f = fused_ws_layout(p.H, p.L, p.nqb, p.nkb);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   float* part = reinterpret_cast<float*>(ws + f.part);
   const float* lse_prev = reinterpret_cast<const float*>(ws + f.lse_prev);
-  SP_TRY(launch_attn(p, false, nullptr, nullptr, 0, st, lse_prev, part));
+  SP_TRY(launch_attn(p, false, nullptr, nullptr, 0, st, lse_prev, part, ps));
   float* mass = reinterpret_cast<float*>(ws + ws_layout(p.H, p.nqb, p.nkb).grid);
   const long n = static_cast<long>(p.H) * p.nqb * p.nkb;
   mass_from_parts_kernel<<<static_cast<unsigned>(cdiv(n, 256)), 256, 0, st>>>(reinterpret_cast<const float4*>(part),
@@ -831,6 +858,13 @@ int run_steps_impl(const uint16_t* Q, const uint16_t* K, const uint16_t* V, int 
                      workspace_bytes >= fused_ws_layout(p.H, p.L, p.nqb, p.nkb).total &&
                      static_cast<long long>(p.H) * p.nqb * p.nkb * kMassParts < (1ll << 31);
   bool have_lse = false;  // a full pass of this call left its LSE in the workspace
+  // the dense passes take their pairs from counters in the workspace when it
+  // has the room
+  const Workspace wl = ws_layout(p.H, p.nqb, p.nkb);
+  PairSched ps;
+  SP_TRY(begin_pair_sched(&ps, workspace && workspace_bytes >= wl.total ? static_cast<uint8_t*>(workspace) + wl.sched
+                                                                        : nullptr,
+                          st));
   std::vector<cudaEvent_t> ev;
   if (step_ms && start_step < end_step) {
     ev.resize(static_cast<size_t>(end_step - start_step) + 1, nullptr);
@@ -845,7 +879,7 @@ int run_steps_impl(const uint16_t* Q, const uint16_t* K, const uint16_t* V, int 
     if (rc != SPARSED_OK) break;
     switch (kinds[t]) {
       case SPARSED_STEP_DENSE:
-        rc = launch_attn(p, false, nullptr, nullptr, 0, st);
+        rc = launch_attn(p, false, nullptr, nullptr, 0, st, nullptr, nullptr, &ps);
         if (rc == SPARSED_OK && fused && t + 1 < end_step && kinds[t + 1] == SPARSED_STEP_SELECT) {
           rc = save_lse(p, workspace, st);
           have_lse = true;
@@ -853,9 +887,9 @@ int run_steps_impl(const uint16_t* Q, const uint16_t* K, const uint16_t* V, int 
         break;
       case SPARSED_STEP_SELECT:
         if (fused && have_lse) {
-          rc = fused_select(p, keep_ratio, budget_mode, kv_idx, kv_count, kv_stride, workspace, st);
+          rc = fused_select(p, keep_ratio, budget_mode, kv_idx, kv_count, kv_stride, workspace, &ps, st);
         } else {
-          rc = launch_attn(p, false, nullptr, nullptr, 0, st);
+          rc = launch_attn(p, false, nullptr, nullptr, 0, st, nullptr, nullptr, &ps);
           if (rc == SPARSED_OK)
             rc = select_after_dense(p, keep_ratio, budget_mode, kv_idx, kv_count, kv_stride, nullptr,
                                     nullptr, workspace, st);
@@ -1081,6 +1115,10 @@ int sparsed_run_steps_columns(const uint16_t* Q, const uint16_t* K, const uint16
   SP_TRY(require_sm100());
   SP_TRY(get_encoder());
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  // the full passes take their pairs from counters in the workspace
+  PairSched ps;
+  if (start_step < T)
+    SP_TRY(begin_pair_sched(&ps, static_cast<uint8_t*>(workspace) + col_ws_layout(p.H, p.L, p.d, kc).sched, st));
   std::vector<cudaEvent_t> ev;
   if (step_ms && start_step < T) {
     ev.resize(static_cast<size_t>(T - start_step) + 1, nullptr);
@@ -1091,10 +1129,10 @@ int sparsed_run_steps_columns(const uint16_t* Q, const uint16_t* K, const uint16
   for (int t = start_step; t < T && rc == SPARSED_OK; ++t) {
     switch (kinds[t]) {
       case SPARSED_STEP_DENSE:
-        rc = launch_attn(p, false, nullptr, nullptr, 0, st);
+        rc = launch_attn(p, false, nullptr, nullptr, 0, st, nullptr, nullptr, &ps);
         break;
       case SPARSED_STEP_SELECT:
-        rc = launch_attn(p, false, nullptr, nullptr, 0, st);
+        rc = launch_attn(p, false, nullptr, nullptr, 0, st, nullptr, nullptr, &ps);
         if (rc == SPARSED_OK) rc = select_columns_after_dense(p, kc, cols, col_stride, nullptr, workspace, st);
         break;
       default:

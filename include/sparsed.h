@@ -199,7 +199,13 @@ int sparsed_block_sparse_attn(const uint16_t* Q, const uint16_t* K, const uint16
  * pass, which equals this pass's LSE because the loop's inputs are fixed
  * (Step-dLLM abstract: selection cost matters at every anchor). A SELECT step
  * with no earlier full pass in the call, or a smaller workspace, runs the
- * separate block-mass pass of sparsed_select_pattern. */
+ * separate block-mass pass of sparsed_select_pattern. With a workspace of at
+ * least sparsed_workspace_bytes, the loop's full passes take their pairs of
+ * query blocks from counters kept in it (cleared by one memset per call), so
+ * the CTAs in flight stay on neighbouring query blocks and share K/V in L2.
+ * The results are the same bits as with the static order of a call without
+ * a workspace. The workspace must not be in use by another call at the same
+ * time. */
 int sparsed_run_steps(const uint16_t* Q, const uint16_t* K, const uint16_t* V,
                       int H, int L, int d, float scale, int bq, int bk,
                       float keep_ratio, int budget_mode,
@@ -393,7 +399,8 @@ int sparsed_column_sparse_attn(const uint16_t* Q, const uint16_t* K, const uint1
  * sparsed_schedule(T, warmup_frac, refresh_every); DENSE: sparsed_dense_attn;
  * SELECT: sparsed_select_columns into cols (the pattern cache, caller memory);
  * SPARSE: sparsed_column_sparse_attn with the cached columns. Arguments and
- * outputs otherwise as sparsed_run_steps. */
+ * outputs otherwise as sparsed_run_steps; the full passes take their pairs of
+ * query blocks from counters in the workspace as there. */
 int sparsed_run_steps_columns(const uint16_t* Q, const uint16_t* K, const uint16_t* V,
                               int H, int L, int d, float scale, int bq, int bk, float keep_ratio,
                               int T, float warmup_frac, int refresh_every,

@@ -364,3 +364,28 @@ def test_dense_attn_agrees_with_torch_sdpa(d, L):
     assert err.max().item() <= 2e-2 and err.mean().item() <= 2e-3
     s = torch.matmul(qc.float(), kc.float().transpose(1, 2)) * scale
     assert (lse - torch.logsumexp(s, dim=-1)).abs().max().item() <= 1e-3
+
+
+@pytest.mark.parametrize("H,L,d,bq,bk", [(8, 4000, 128, 128, 128), (4, 8200, 64, 64, 64),
+                                         (16, 16384 + 100, 128, 128, 128), (3, 640, 128, 128, 64)])
+def test_counter_scheduled_passes_equal_static(H, L, d, bq, bk):
+    """The step loop's full passes take their pairs of query blocks from a
+    counter in the workspace; a standalone dense_attn takes them by a static
+    stride. A pair's arithmetic does not depend on which CTA runs it, so every
+    pass of a loop of dense steps (the counter slots alternating from launch to
+    launch, and starting over in a second call on the same workspace) gives
+    the bits of the static pass. The cases cover fewer pairs than SMs, an odd
+    number of query blocks (a pair without a second block) and several waves."""
+    q, k, v, scale = _inputs(H, L, d, seed=31 + d + H, structure="band")
+    qc, kc, vc = _cuda(q, k, v)
+    od, ld = sp.dense_attn(qc, kc, vc, bq=bq, bk=bk)
+    ws = torch.empty(sp.run_steps_workspace_bytes(H, L, bq, bk), dtype=torch.uint8, device="cuda")
+    for _ in range(2):
+        r = sp.run_steps(qc, kc, vc, T=5, warmup_frac=1.0, bq=bq, bk=bk, workspace=ws)
+        sp.device_check()
+        assert set(r.kinds) == {sp.STEP_DENSE}
+        assert torch.equal(r.o.view(torch.int16), od.view(torch.int16))
+        assert torch.equal(r.lse, ld)
+    if L <= 4000:
+        o_ref, l_ref = oracle_dense_heads(q, k, v, scale)
+        assert_o_lse(r.o, r.lse, o_ref, l_ref, f"counter-scheduled dense d={d} bq={bq} bk={bk}")
