@@ -43,13 +43,18 @@ struct ColMassCfg {
   static constexpr int TILE_BYTES = 128 * D * 2;
   static constexpr int OFF_K = 0;
   static constexpr int OFF_Q = TILE_BYTES;
-  static constexpr int OFF_LSE = OFF_Q + STAGES * TILE_BYTES;  // float [2][128]
-  static constexpr int OFF_BAR = OFF_LSE + 2 * 128 * 4;
+  static constexpr int G = 4;             // column groups of reducer warps
+  static constexpr int CW = N / G;        // query columns per group and tile
+  static constexpr int RWARPS = 4 * G;    // reducer warps (4 + w)
+  static constexpr int REDUCERS = 32 * RWARPS;
+  static constexpr int OFF_LSE = OFF_Q + STAGES * TILE_BYTES;  // float2 [RWARPS][2][CW/2]: -LSE (log2 units)
+  static constexpr int OFF_TOT = OFF_LSE + RWARPS * CW * 8;    // float [G-1][128]: groups 1.. sums
+  static constexpr int OFF_BAR = OFF_TOT + (G - 1) * 128 * 4;
   static constexpr int B_KFULL = 0;
   static constexpr int B_QFULL = 1;
   static constexpr int B_QEMPTY = B_QFULL + STAGES;
   static constexpr int B_SFULL = B_QEMPTY + STAGES;  // [2]
-  static constexpr int B_SFREE = B_SFULL + 2;        // [2] 128 reducer arrivals
+  static constexpr int B_SFREE = B_SFULL + 2;        // [2] one arrival per reducer thread
   static constexpr int B_DRAIN = B_SFREE + 2;
   static constexpr int NUM_BARS = B_DRAIN + 1;
   static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;  // tmem slot, abort flag
@@ -58,15 +63,25 @@ struct ColMassCfg {
   static constexpr int TM_S1 = N;
   static constexpr int TM_ALLOC = 256;
   static constexpr uint32_t IDESC = ptx::idesc_bf16_f32(M, N, 0, 0);
+  static constexpr int THREADS = 128 + REDUCERS;
+  static_assert(CW % 32 == 0, "whole 32-column TMEM loads per group");
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 };
 
-// Grid (ceil(Lk/128), H), 256 threads: warp 0 loads K once and streams the
-// query tiles, warp 1 owns TMEM and issues S^T_i = K_j Q_i^T, warps 4-7 reduce
-// (thread = key row = TMEM lane). Every query tile's LSE values are staged in
-// shared memory by the reducers, one tile ahead of their use.
+// Grid (ceil(Lk/128), H), 128 + 32 * 4G threads: warp 0 loads K once and streams the
+// query tiles, warp 1 owns TMEM and issues S^T_i = K_j Q_i^T (double-buffered),
+// warps 4 .. 4 + 4G - 1 reduce. A reducer thread is a key row (its TMEM lane,
+// warp % 4 the lane quarter); group g (warps 4 + 4g .. 4 + 4g + 3) takes query
+// columns g*CW .. g*CW + CW - 1 of every tile, so G warps per SM
+// sub-partition keep the exponentials coming. Each thread sums its columns in
+// a fixed order (two packed fp32x2 accumulators, then one running total per
+// group), and the groups' totals are added in a fixed order at the end:
+// bit-reproducible. Each reducer warp stages the -LSE of its CW query columns
+// in its own
+// double-buffered shared-memory slice, loaded one tile ahead, so the warps
+// synchronise only through the S buffers' mbarriers.
 template <int D>
-__global__ void __launch_bounds__(256, 1)
+__global__ void __launch_bounds__(ColMassCfg<D>::THREADS, 1)
     column_mass_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                        const ColMassArgs a) {
   using C = ColMassCfg<D>;
@@ -79,7 +94,6 @@ __global__ void __launch_bounds__(256, 1)
   const int kj = blockIdx.x;
   const int h = blockIdx.y;
   const int n = (a.L + C::N - 1) / C::N;  // query tiles
-  float* lse2s = reinterpret_cast<float*>(smem + C::OFF_LSE);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
   auto bar = [&](int idx) -> uint32_t { return sb + C::OFF_BAR + 8 * idx; };
@@ -92,7 +106,7 @@ __global__ void __launch_bounds__(256, 1)
     }
     for (int b = 0; b < 2; ++b) {
       ptx::mbar_init(bar(C::B_SFULL + b), 1);
-      ptx::mbar_init(bar(C::B_SFREE + b), 128);
+      ptx::mbar_init(bar(C::B_SFREE + b), C::REDUCERS);
     }
     ptx::mbar_init(bar(C::B_DRAIN), 1);
     *abort_flag = 0;
@@ -167,47 +181,78 @@ __global__ void __launch_bounds__(256, 1)
     }
   } else if (warp >= 4) {
     // ================================================================ reducers
+    const int g = (warp - 4) >> 2;  // column group
     const int wq = warp & 3;
-    const int r = wq * 32 + lane;  // key row of this CTA == TMEM lane
+    const int r = wq * 32 + lane;   // key row of this CTA == TMEM lane
     const uint32_t lane_base = tmem + (static_cast<uint32_t>(wq * 32) << 16);
-    const float sl2 = a.scale_log2;
+    const uint64_t sl2 = ptx::f32x2(a.scale_log2, a.scale_log2);
     const float* lse_h = a.lse + static_cast<long>(h) * a.L;
-    const float kInf = __int_as_float(0x7f800000);
-    // LSE of query i*128 + r in log2 units; queries past L weigh nothing
-    auto lse2_of = [&](int i) -> float {
-      const int qrow = i * C::N + r;
-      return qrow < a.L ? lse_h[qrow] * 1.44269504088896340736f : kInf;
+    float* tot = reinterpret_cast<float*>(smem + C::OFF_TOT);
+    const float kNegInf = -__int_as_float(0x7f800000);
+    // -LSE (log2 units) of this warp's query columns 2*lane, 2*lane + 1 of
+    // tile i (lanes below CW/2); queries past L weigh nothing
+    auto neg_lse2_of = [&](int i) -> float2 {
+      const int q = i * C::N + g * C::CW + 2 * lane;
+      float2 v;
+      v.x = q < a.L ? lse_h[q] * -1.44269504088896340736f : kNegInf;
+      v.y = q + 1 < a.L ? lse_h[q + 1] * -1.44269504088896340736f : kNegInf;
+      return v;
     };
-    float nxt = lse2_of(0);
+    float2* wl = reinterpret_cast<float2*>(smem + C::OFF_LSE) + (warp - 4) * C::CW;  // [2][CW/2] float2
+    constexpr int HW = C::CW / 2;
+    float2 nxt = lane < HW ? neg_lse2_of(0) : float2{};
     float total = 0.f;
     for (int i = 0; i < n; ++i) {
       const int b = i & 1;
-      // every reducer takes every named barrier, also after an abort (the
-      // waits below then return at once), so none is left behind
-      lse2s[b * 128 + r] = nxt;
-      ptx::named_bar_sync(1, 128);
-      if (i + 1 < n) nxt = lse2_of(i + 1);
+      // buffer b was last read at tile i - 2, before the __syncwarp of tile i - 1
+      if (lane < HW) wl[b * HW + lane] = nxt;
+      __syncwarp();
+      if (i + 1 < n && lane < HW) nxt = neg_lse2_of(i + 1);
       const bool ok =
           ptx::mbar_wait_warp(bar(C::B_SFULL + b), (i >> 1) & 1, abort_flag, a.timeout_ns, kErrTimeout);
       if (!ok) continue;
       ptx::tc_fence_after();
-      float part[4] = {0.f, 0.f, 0.f, 0.f};
+      constexpr int NC = C::CW / 32;
+      uint32_t raw[NC][32];
+      const uint32_t col0 = (b ? C::TM_S1 : C::TM_S0) + g * C::CW;
 #pragma unroll
-      for (int c = 0; c < C::N / 32; ++c) {
-        uint32_t raw[32];
-        ptx::tmem_ld32(lane_base + (b ? C::TM_S1 : C::TM_S0) + c * 32, raw);
-        ptx::tmem_wait_ld();
-        ptx::reg_fence32(raw);
-#pragma unroll
-        for (int e = 0; e < 32; ++e)
-          part[e & 3] += ptx::ex2(fmaf(__uint_as_float(raw[e]), sl2, -lse2s[b * 128 + c * 32 + e]));
-      }
+      for (int c = 0; c < NC; ++c) ptx::tmem_ld32(lane_base + col0 + c * 32, raw[c]);
+      ptx::tmem_wait_ld();
       ptx::tc_fence_before();
-      ptx::mbar_arrive(bar(C::B_SFREE + b));
-      total += (part[0] + part[1]) + (part[2] + part[3]);
+      ptx::mbar_arrive(bar(C::B_SFREE + b));  // S_b is in registers: the MMA may overwrite it
+      const float2* nl = wl + b * HW;
+      uint64_t acc0 = ptx::f32x2(0.f, 0.f), acc1 = acc0;
+#pragma unroll
+      for (int c = 0; c < NC; ++c) {
+        ptx::reg_fence32(raw[c]);
+#pragma unroll
+        for (int e = 0; e < 32; e += 2) {
+          const float2 l2 = nl[(c * 32 + e) >> 1];
+          float x0, x1;
+          ptx::f32x2_split(ptx::fma_f32x2(ptx::f32x2(__uint_as_float(raw[c][e]), __uint_as_float(raw[c][e + 1])),
+                                          sl2, ptx::f32x2(l2.x, l2.y)),
+                           x0, x1);
+          const uint64_t p2 = ptx::f32x2(ptx::ex2(x0), ptx::ex2(x1));
+          if (e & 2)
+            acc1 = ptx::add_f32x2(acc1, p2);
+          else
+            acc0 = ptx::add_f32x2(acc0, p2);
+        }
+      }
+      float a0, a1, b0, b1;
+      ptx::f32x2_split(acc0, a0, a1);
+      ptx::f32x2_split(acc1, b0, b1);
+      total += (a0 + b0) + (a1 + b1);
     }
+    // the groups' sums of every key row, added in a fixed order
+    if (g > 0) tot[(g - 1) * 128 + r] = total;
+    ptx::named_bar_sync(2, C::REDUCERS);
     const int key = kj * C::M + r;
-    if (key < a.Lk && !*abort_flag) a.mass[static_cast<long>(h) * a.Lk + key] = total;
+    if (g == 0 && key < a.Lk && !*abort_flag) {
+#pragma unroll
+      for (int q = 1; q < C::G; ++q) total += tot[(q - 1) * 128 + r];
+      a.mass[static_cast<long>(h) * a.Lk + key] = total;
+    }
   }
 
   ptx::tc_fence_before();

@@ -420,7 +420,7 @@ int launch_col_mass_t(const Problem& p, float* mass, cudaStream_t st) {
   a.timeout_ns = kWaitTimeoutNs;
   auto kern = column_mass_kernel<D>;
   SP_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES));
-  kern<<<dim3(static_cast<unsigned>(cdiv(p.L, C::M)), p.H), 256, C::SMEM_BYTES, st>>>(tq, tk, a);
+  kern<<<dim3(static_cast<unsigned>(cdiv(p.L, C::M)), p.H), C::THREADS, C::SMEM_BYTES, st>>>(tq, tk, a);
   SP_CUDA(cudaGetLastError());
   return SPARSED_OK;
 }

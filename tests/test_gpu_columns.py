@@ -22,8 +22,11 @@ def _inputs(H, L, d, seed, structure="iid"):
 
 
 @pytest.mark.parametrize("d,L,keep,structure", [(64, 1000, 0.1, "iid"), (128, 2048, 0.05, "band"),
-                                                 (128, 777, 0.3, "key_bias")])
+                                                 (128, 777, 0.3, "key_bias"), (64, 100, 0.2, "iid")])
 def test_select_columns_parity(d, L, keep, structure):
+    """Selection pass, column mass and kept columns against the oracle. The
+    column-mass kernel takes one 128-key block per CTA: L=1000 and L=777 end
+    in a ragged block, L=100 is a single ragged block."""
     H = 3
     q, k, v, scale = _inputs(H, L, d, seed=900 + d + L, structure=structure)
     pat = sp.select_columns(*(t.cuda() for t in (q, k, v)), keep=keep, return_mass=True)
