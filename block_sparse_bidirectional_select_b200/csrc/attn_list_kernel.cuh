@@ -221,6 +221,10 @@ __global__ void __launch_bounds__(384, 1)
   __syncthreads();
   ptx::tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  // As a programmatic dependent (the block-wise steps) the setup above ran
+  // while the previous kernel finished; nothing global is read before here.
+  ptx::grid_dep_wait();
+  ptx::grid_dep_launch();
 
   if (warp >= 8) {
     setmaxnreg_dec_56();

@@ -74,6 +74,7 @@ __global__ void __launch_bounds__(256)
     query_mse_kernel(const uint16_t* __restrict__ q, const uint16_t* __restrict__ q_prev, int H, int B, int d,
                      double tau, int32_t* __restrict__ active) {
   __shared__ double s_part[8];
+  ptx::grid_dep_launch();  // the union-and-lists kernel may launch; it waits for this grid to complete
   const int b = blockIdx.x;
   const int row_u4 = d / 8;
   const int n_u4 = H * row_u4;
@@ -144,6 +145,10 @@ __global__ void __launch_bounds__(256) losa_lists_kernel(const LosaListArgs a) {
   __shared__ int s_scan[8];
   __shared__ int s_warp[8];
   __shared__ int s_u;
+  // a programmatic dependent of the locality score: active[] is complete
+  // past this point (a no-op after an ordinary launch)
+  ptx::grid_dep_wait();
+  ptx::grid_dep_launch();
   const int h = blockIdx.x;
   const int tid = threadIdx.x;
   const int lane = tid & 31, wid = tid >> 5;
@@ -293,6 +298,7 @@ struct LosaMergeArgs {
 template <int D>
 __global__ void __launch_bounds__(256) losa_merge_kernel(const LosaMergeArgs a) {
   constexpr int PER = D / 32;  // contiguous elements per lane
+  ptx::grid_dep_wait();        // a programmatic dependent of the prefix pass
   const int lane = threadIdx.x & 31;
   const long row = static_cast<long>(blockIdx.x) * 8 + (threadIdx.x >> 5);
   if (row >= static_cast<long>(a.H) * a.B) return;

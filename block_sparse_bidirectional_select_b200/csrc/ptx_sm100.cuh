@@ -278,6 +278,13 @@ __device__ __forceinline__ void umma_commit_if(uint32_t leader, uint32_t bar) {
       "r"(leader)
       : "memory");
 }
+// Programmatic dependent launch. grid_dep_wait: the grids this one was
+// launched after (as a programmatic dependent) have completed and their
+// memory is visible; without such a launch it returns at once.
+// grid_dep_launch: this CTA lets the dependents of its grid be launched.
+__device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void grid_dep_launch() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // 1 in exactly one lane of the (fully active) warp, 0 elsewhere.
 __device__ __forceinline__ uint32_t elect_one() {
   uint32_t r;

@@ -301,11 +301,31 @@ int launch_attn_t(const Problem& p, const float* lse_prev, float* mass_part, Pai
   return SPARSED_OK;
 }
 
+// A kernel launch that may start as a programmatic dependent of the previous
+// kernel on the stream (pdl): its CTAs are scheduled while that kernel
+// finishes and wait in the kernel (griddepcontrol.wait) before they read its
+// results. Only kernels that wait before any global access are launched so.
+template <typename... KArgs, typename... Args>
+int launch_k(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st, bool pdl, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[0].val.programmaticStreamSerializationAllowed = pdl ? 1 : 0;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  SP_CUDA(cudaLaunchKernelEx(&cfg, kern, args...));
+  return SPARSED_OK;
+}
+
 // Block-sparse passes: the one-tile kernel (each query tile walks its own
 // list), with the same register-split check.
 template <int D, int BK>
 int launch_list_t(const Problem& p, const int32_t* kv_idx, const int32_t* kv_count, int kv_stride,
-                  cudaStream_t st) {
+                  cudaStream_t st, bool pdl = false) {
   using C = ListCfg<D, BK>;
   auto kern = attn_list_kernel<D, BK>;
   static int regs = -1;
@@ -343,6 +363,7 @@ int launch_list_t(const Problem& p, const int32_t* kv_idx, const int32_t* kv_cou
   // persistent: one CTA per SM, each walking items blockIdx.x, blockIdx.x + gridDim.x, ...
   const long items = static_cast<long>(p.H) * p.nqb;
   const int grid = static_cast<int>(items < sms ? items : sms);
+  if (pdl) return launch_k(kern, dim3(grid), dim3(C::THREADS), C::SMEM_BYTES, st, true, tq, tk, tv, a);
   kern<<<grid, C::THREADS, C::SMEM_BYTES, st>>>(tq, tk, tv, a);
   SP_CUDA(cudaGetLastError());
   return SPARSED_OK;
@@ -352,13 +373,14 @@ int launch_list_t(const Problem& p, const int32_t* kv_idx, const int32_t* kv_cou
 // block-sparse passes in the one-tile kernel. mass_part != nullptr selects the
 // fused variant (dense only): the pass also writes the block-mass partials,
 // using lse_prev as every row's LSE. ps (nullable) gives the dense passes the
-// counter slots of their pair scheduler.
+// counter slots of their pair scheduler; pdl launches a block-sparse pass as a
+// programmatic dependent of the previous kernel on the stream.
 int launch_attn(const Problem& p, bool sparse, const int32_t* kv_idx, const int32_t* kv_count,
                 int kv_stride, cudaStream_t st, const float* lse_prev = nullptr, float* mass_part = nullptr,
-                PairSched* ps = nullptr) {
+                PairSched* ps = nullptr, bool pdl = false) {
 #define SP_ATTN(D_, BK_)                                                                                  \
   if (p.d == D_ && p.bk == BK_) {                                                                         \
-    if (sparse) return launch_list_t<D_, BK_>(p, kv_idx, kv_count, kv_stride, st);                        \
+    if (sparse) return launch_list_t<D_, BK_>(p, kv_idx, kv_count, kv_stride, st, pdl);                   \
     if (mass_part) return launch_attn_t<D_, BK_, true>(p, lse_prev, mass_part, ps, st);                 \
     return launch_attn_t<D_, BK_, false>(p, nullptr, nullptr, ps, st);                                    \
   }
@@ -1453,9 +1475,7 @@ int losa_lists(const LosaDims& g, const int32_t* active, const int32_t* sel, int
   a.kv_idx = reinterpret_cast<int32_t*>(ws + w.kvi);
   a.kv_count = reinterpret_cast<int32_t*>(ws + w.kvc);
   a.q_rep = reinterpret_cast<uint16_t*>(ws + w.qrep);
-  losa_lists_kernel<<<g.H, 256, 0, st>>>(a);
-  SP_CUDA(cudaGetLastError());
-  return SPARSED_OK;
+  return launch_k(losa_lists_kernel, dim3(g.H), dim3(256), 0, st, true, a);
 }
 
 // Prefix pass over the split lists (block-sparse kernel, the replicated
@@ -1480,7 +1500,8 @@ int losa_prefix_and_merge(const LosaDims& g, const uint16_t* Kp, const uint16_t*
   p.Lk = g.P;
   p.scale = scale;
   const int32_t* kvc = reinterpret_cast<const int32_t*>(ws + w.kvc);
-  SP_TRY(launch_attn(p, true, reinterpret_cast<const int32_t*>(ws + w.kvi), kvc, g.stride, st));
+  SP_TRY(launch_attn(p, true, reinterpret_cast<const int32_t*>(ws + w.kvi), kvc, g.stride, st, nullptr, nullptr,
+                     nullptr, true));
   if (suffix_done) SP_CUDA(cudaStreamWaitEvent(st, suffix_done, 0));  // the merge reads the suffix part
   LosaMergeArgs m;
   m.H = g.H;
@@ -1499,12 +1520,7 @@ int losa_prefix_and_merge(const LosaDims& g, const uint16_t* Kp, const uint16_t*
   m.o = O;
   m.lse = LSE;
   const unsigned grid = static_cast<unsigned>(cdiv(static_cast<long>(g.H) * g.B, 8));
-  if (g.d == 64)
-    losa_merge_kernel<64><<<grid, 256, 0, st>>>(m);
-  else
-    losa_merge_kernel<128><<<grid, 256, 0, st>>>(m);
-  SP_CUDA(cudaGetLastError());
-  return SPARSED_OK;
+  return launch_k(g.d == 64 ? losa_merge_kernel<64> : losa_merge_kernel<128>, dim3(grid), dim3(256), 0, st, true, m);
 }
 
 template <int D, int BK>
