@@ -30,18 +30,25 @@
 // (warps 8-10 run warp-uniform code; one elected lane issues each copy, MMA
 // and commit)
 //   warp 11     idle (donates its registers)
-// TMEM (128 lanes): [S0 | S1 | O | P0 | P1] = 2*BK + D + BK fp32 columns. S is
-// double-buffered, so S(g+1) is computed while the softmax works on S(g); P has
-// its own two buffers, so the two issuers never touch the same columns and can
-// run independently (a commit from one thread tracks only its own MMAs):
-//   S issuer : S_b(g) once PV(g-2) is done (which also means the softmax has
-//              read S_b(g-2) and that P_b is free again)       (PVDONE)
-//   softmax  : reads S_b(g), writes P_b(g)                      (SFULL -> PFULL)
+// TMEM (128 lanes): [S0 | S1 | O | Q0 | Q1] = 2*BK + 2*D fp32 columns. S is
+// double-buffered, so S(g+1) is computed while the softmax works on S(g); P(g)
+// is written over the first BK/2 columns of S_b(g) once the softmax has read
+// them. Q sits in TMEM (two buffers, one per item in flight) so that
+// S = Q K^T is a TS MMA: only K comes from shared memory, which leaves shared
+// memory bandwidth for the K/V copies. The two issuers run independently (a
+// commit from one thread tracks only its own MMAs):
+//   S issuer : S_b(g) once PV(g-2) is done (the softmax has read S_b(g-2) and
+//              PV has read the P_b(g-2) written over it)       (PVDONE)
+//              and the item's Q is in TMEM                      (QTFULL)
+//   softmax  : reads S_b(g), writes P_b(g) over it              (SFULL -> PFULL)
+//              copies each item's Q from shared memory into TMEM Q_c, after
+//              every S MMA that read Q_c two items earlier      (QFULL, QTEMPTY
+//                                                                -> QTFULL, QEMPTY)
 //   PV issuer: O += P_b(g) V_g; the first tile of an item overwrites O, which
 //              the softmax warps have read out before they wrote that P
 //                                                               (PFULL -> PVDONE)
-//   producer : Q of the next item once every S MMA of the current one is
-//              complete                                         (QEMPTY)
+//   producer : Q of the next item once the softmax has copied the current
+//              one into TMEM                                    (QEMPTY)
 // The lazy rescale keeps O and the running sum on a stale row max until a
 // row's max grows by more than 2^8; both halves of a row see the same max, so
 // they take the same decision, and each rescales its half of O.
@@ -72,7 +79,7 @@ struct ListCfg {
   static constexpr int OFF_V = OFF_K + KS * KV_BYTES;
   static constexpr int OFF_BAR = OFF_V + VS * KV_BYTES;
   static constexpr int B_QFULL = 0;
-  static constexpr int B_QEMPTY = 1;
+  static constexpr int B_QEMPTY = 1;             // 8 softmax-warp arrivals: Q copied into TMEM
   static constexpr int B_KFULL = 2;
   static constexpr int B_KEMPTY = B_KFULL + KS;
   static constexpr int B_VFULL = B_KEMPTY + KS;
@@ -81,15 +88,17 @@ struct ListCfg {
   static constexpr int B_PFULL = B_SFULL + 2;    // [2] 8 warp arrivals
   static constexpr int B_PVDONE = B_PFULL + 2;   // [2]
   static constexpr int B_DRAIN = B_PVDONE + 2;   // [2] per issuer
-  static constexpr int NUM_BARS = B_DRAIN + 2;
+  static constexpr int B_QTFULL = B_DRAIN + 2;   // [2] Q_c in TMEM: 8 softmax-warp arrivals
+  static constexpr int B_QTEMPTY = B_QTFULL + 2; // [2] every S MMA that read Q_c is complete
+  static constexpr int NUM_BARS = B_QTEMPTY + 2;
   static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;  // tmem slot, abort flag
   static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;
   static constexpr int TM_S0 = 0;
   static constexpr int TM_S1 = BK;
   static constexpr int TM_O = 2 * BK;
-  static constexpr int TM_P0 = 2 * BK + D;
-  static constexpr int TM_P1 = TM_P0 + BK / 2;
-  static constexpr int TM_USED = TM_P1 + BK / 2;
+  static constexpr int TM_Q0 = 2 * BK + D;       // Q as the A operand: D/2 columns of bf16 pairs
+  static constexpr int TM_Q1 = TM_Q0 + D / 2;
+  static constexpr int TM_USED = TM_Q1 + D / 2;
   static constexpr int TM_ALLOC = TM_USED <= 256 ? 256 : 512;
   static constexpr uint32_t IDESC_S = ptx::idesc_bf16_f32(128, BK, 0, 0);
   static constexpr uint32_t IDESC_PV = ptx::idesc_bf16_f32(128, D, 0, 1);
@@ -195,7 +204,11 @@ __global__ void __launch_bounds__(384, 1)
   // ---- setup
   if (threadIdx.x == 0) {
     ptx::mbar_init(bar(C::B_QFULL), 1);
-    ptx::mbar_init(bar(C::B_QEMPTY), 1);
+    ptx::mbar_init(bar(C::B_QEMPTY), 8);  // one arrival per softmax warp
+    for (int c = 0; c < 2; ++c) {
+      ptx::mbar_init(bar(C::B_QTFULL + c), 8);
+      ptx::mbar_init(bar(C::B_QTEMPTY + c), 1);
+    }
     for (int s = 0; s < C::KS; ++s) {
       ptx::mbar_init(bar(C::B_KFULL + s), 1);
       ptx::mbar_init(bar(C::B_KEMPTY + s), 1);
@@ -252,7 +265,7 @@ __global__ void __launch_bounds__(384, 1)
         const ItemList<SPARSE> it = item_list<SPARSE>(a, w, n_raw);
         if (SPARSE && leader && n_raw != it.n) ptx::record_error(kErrBadPattern);
         if (it.n == 0) continue;
-        // Q of this item once every S MMA of the previous item is complete
+        // Q of this item once the softmax has copied the previous one into TMEM
         if (iq > 0 && !wait(C::B_QEMPTY, iq - 1)) {
           ok = false;
           break;
@@ -311,7 +324,6 @@ __global__ void __launch_bounds__(384, 1)
     } else if (warp == 9) {
       // ============================================================ S issuer
       constexpr uint32_t HI = ptx::sdesc_sw128_hi(1024);
-      const uint32_t qlo = ptx::sdesc_sw128_lo(sb + C::OFF_Q, 16);
       const uint32_t klo = ptx::sdesc_sw128_lo(sb + C::OFF_K, 16);
       int g = 0, iq = 0;
       bool ok = true;
@@ -320,10 +332,12 @@ __global__ void __launch_bounds__(384, 1)
         n_raw_next = raw_count<SPARSE>(a, w + gridDim.x);
         const ItemList<SPARSE> it = item_list<SPARSE>(a, w, n_raw);
         if (it.n == 0) continue;
-        if (!wait(C::B_QFULL, iq)) {
+        const int qc = iq & 1;
+        if (!wait(C::B_QTFULL + qc, iq >> 1)) {
           ok = false;
           break;
         }
+        const uint32_t q_tmem = tmem + (qc ? C::TM_Q1 : C::TM_Q0);
         for (int jj = 0; jj < it.n; ++jj, ++g) {
           const int b = g & 1;
           const int ks = g % C::KS;
@@ -336,16 +350,15 @@ __global__ void __launch_bounds__(384, 1)
           const uint32_t s_tmem = tmem + (b ? C::TM_S1 : C::TM_S0);
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t ao = (kk >> 2) * (C::Q_CHUNK >> 4) + (kk & 3) * 2;
             const uint32_t bo = (kk >> 2) * (C::KV_CHUNK >> 4) + (kk & 3) * 2;
-            ptx::umma_ss_lohi_if(leader, s_tmem, qlo + ao, b0 + bo, HI, C::IDESC_S, kk > 0 ? 1u : 0u);
+            ptx::umma_ts_lohi_if(leader, s_tmem, q_tmem + kk * 8, b0 + bo, HI, C::IDESC_S, kk > 0 ? 1u : 0u);
           }
           ptx::umma_commit_if(leader, bar(C::B_SFULL + b));
           ptx::umma_commit_if(leader, bar(C::B_KEMPTY + ks));
         }
         if (!ok) break;
-        // every S MMA of this item read Q: the producer may refill it
-        ptx::umma_commit_if(leader, bar(C::B_QEMPTY));
+        // every S MMA of this item read Q_qc: the softmax may copy a later item's Q there
+        ptx::umma_commit_if(leader, bar(C::B_QTEMPTY + qc));
         ++iq;
       }
       if (!ok) {
@@ -373,7 +386,7 @@ __global__ void __launch_bounds__(384, 1)
           }
           ptx::tc_fence_after();
           const uint32_t b0 = vlo + static_cast<uint32_t>(vs * C::KV_BYTES >> 4);
-          const uint32_t p_tmem = tmem + (b ? C::TM_P1 : C::TM_P0);
+          const uint32_t p_tmem = tmem + (b ? C::TM_S1 : C::TM_S0);  // P_b over S_b
 #pragma unroll
           for (int kk = 0; kk < BK / 16; ++kk)
             ptx::umma_ts_lohi_if(leader, tmem + C::TM_O, p_tmem + kk * 8, b0 + kk * (2048 >> 4), HI, C::IDESC_PV,
@@ -398,6 +411,47 @@ __global__ void __launch_bounds__(384, 1)
     const float sl2 = a.scale_log2;
     const int s_off = half * HALF;  // first S column of my half row
     int g = 0;
+    int iq = 0;  // items with work so far; their Q copies are numbered alike
+    int cq = 0;  // Q copies into TMEM so far
+    // Copy the Q tile in shared memory (that of item cq) into TMEM Q_{cq&1}, as
+    // the A operand of the S MMAs: row r in lane r, elements 2j, 2j+1 in
+    // column j. Warp w copies the 64-element chunk w/4 of rows 32*(w%4) ..
+    // +31 (the 32x32b access); the tile is in the 128-byte swizzle of its
+    // TMA copy (16-byte unit u of row r at unit u ^ (r % 8)).
+    auto copy_q = [&]() -> bool {
+      const int c = cq & 1;
+      if (!ptx::mbar_wait_warp(bar(C::B_QFULL), cq & 1, abort_flag, a.timeout_ns, kErrTimeout)) return false;
+      if (cq >= 2 &&
+          !ptx::mbar_wait_warp(bar(C::B_QTEMPTY + c), ((cq >> 1) - 1) & 1, abort_flag, a.timeout_ns, kErrTimeout))
+        return false;
+      ptx::tc_fence_after();
+      const int chunk = warp >> 2;
+      if (chunk < C::DCH) {
+        const int qr = (warp & 3) * 32 + lane;
+        const uint8_t* src = smem + C::OFF_Q + chunk * C::Q_CHUNK + qr * 128;
+        uint32_t v[32];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const uint4 x = *reinterpret_cast<const uint4*>(src + ((u ^ (qr & 7)) << 4));
+          v[4 * u] = x.x;
+          v[4 * u + 1] = x.y;
+          v[4 * u + 2] = x.z;
+          v[4 * u + 3] = x.w;
+        }
+        ptx::tmem_st32(tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16) + (c ? C::TM_Q1 : C::TM_Q0) +
+                           chunk * 32,
+                       v);
+        ptx::tmem_wait_st();
+      }
+      ptx::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) {
+        ptx::mbar_arrive(bar(C::B_QTFULL + c));
+        ptx::mbar_arrive(bar(C::B_QEMPTY));
+      }
+      ++cq;
+      return true;
+    };
     bool ok = true;
     int n_raw = raw_count<SPARSE>(a, blockIdx.x), n_raw_next = 0;
     for (int w = blockIdx.x; ok && w < n_items; w += gridDim.x, n_raw = n_raw_next) {
@@ -415,6 +469,11 @@ __global__ void __launch_bounds__(384, 1)
           if (half == 0) a.lse[static_cast<long>(h) * a.L + grow] = -__int_as_float(0x7f800000);
         }
         continue;
+      }
+      // this item's Q, unless it was copied ahead at the end of the previous one
+      if (cq == iq && !copy_q()) {
+        ok = false;
+        break;
       }
       float m = -__int_as_float(0x7f800000);  // running row max, log2 units (scaled)
       float l = 0.f;                          // running sum of my half row
@@ -490,8 +549,9 @@ __global__ void __launch_bounds__(384, 1)
           l *= alpha;
           m = m_new;
         }
-        // P_b is free: S_b(g) was issued only after PV(g-2) completed
-        const float ps = softmax_half_exp<HALF>(s, sl2, m, lane_base + (b ? C::TM_P1 : C::TM_P0));
+        // P_b(g) over S_b(g), read out above; PV(g-2), the last reader of
+        // P_b(g-2), completed before S_b(g) was issued
+        const float ps = softmax_half_exp<HALF>(s, sl2, m, lane_base + (b ? C::TM_S1 : C::TM_S0));
         l += ps;
         ptx::tmem_wait_st();
         ptx::tc_fence_before();
@@ -499,6 +559,14 @@ __global__ void __launch_bounds__(384, 1)
         if (lane == 0) ptx::mbar_arrive(bar(C::B_PFULL + b));
       }
       if (!ok) break;
+      ++iq;
+      // the next item's Q into TMEM now, so its S MMAs can start during this
+      // item's epilogue (the next item with work, if it is the next one)
+      const int w_next = w + static_cast<int>(gridDim.x);
+      if (w_next < n_items && item_list<SPARSE>(a, w_next, n_raw_next).n > 0 && !copy_q()) {
+        ok = false;
+        break;
+      }
       // ---- epilogue: every PV of the item is done -> O / l -> bf16 -> global; LSE
       if (!ptx::mbar_wait_warp(bar(C::B_PVDONE + ((g - 1) & 1)), ((g - 1) >> 1) & 1, abort_flag, a.timeout_ns,
                                kErrTimeout)) {
