@@ -764,7 +764,10 @@ def run_losa(args, dev, rank, world, barrier, max_over_ranks):
             "union_blocks_per_head": float(ucount[1:].mean()) if wl.T > 1 else None,
             "prefix_density": float(ucount[1:].mean()) / nkb if wl.T > 1 else None,
             "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm, "unit": "GB/s", "frac": gbs / hbm,
-                         "traffic": None, "peak_source": peak_src},
+                         "traffic": load_traffic(wl.name, "losa_kernels_sha256", LOSA_KERNEL_FILES).get("block_run"),
+                         "traffic_unit": "DRAM bytes of one block run (its launches summed, ncu, caches flushed "
+                                         "before each launch)",
+                         "peak_source": peak_src},
             "later_step_roofline": None if step_ms is None else
             {"bound": "hbm", "achieved": step_bytes / (step_ms * 1e-3) / 1e9, "peak": hbm, "unit": "GB/s",
              "frac": step_bytes / (step_ms * 1e-3) / 1e9 / hbm, "bytes": step_bytes},
@@ -789,29 +792,36 @@ def code_signature(src):
     return "\n".join(lines)
 
 
-def kernel_signature():
-    """sha256 of the two attention kernels' code (comments and blank lines
-    removed): the dense two-tile kernel and the block-sparse one-tile kernel."""
+ATTN_KERNEL_FILES = ("attn_kernel.cuh", "attn_list_kernel.cuh")
+LOSA_KERNEL_FILES = ATTN_KERNEL_FILES + ("losa_kernels.cuh",)
+
+
+def kernel_signature(files=ATTN_KERNEL_FILES):
+    """sha256 of the kernels' code (comments and blank lines removed): by
+    default the dense two-tile kernel and the block-sparse one-tile kernel;
+    with LOSA_KERNEL_FILES also the block-wise path's own kernels."""
     import hashlib
     csrc = os.path.join(ROOT, "block_sparse_bidirectional_select_b200", "csrc")
     parts = []
-    for name in ("attn_kernel.cuh", "attn_list_kernel.cuh"):
+    for name in files:
         with open(os.path.join(csrc, name)) as f:
             parts.append(code_signature(f.read()))
     return hashlib.sha256("\n".join(parts).encode()).hexdigest()
 
 
-def load_traffic(workload):
-    """DRAM bytes per launch from the committed ncu capture (profiles/traffic.json),
-    used only while the attention kernels' source is the one that was captured."""
+def load_traffic(workload, sha_key="attn_kernels_sha256", files=ATTN_KERNEL_FILES):
+    """DRAM bytes from the committed ncu capture (profiles/traffic.json), used
+    only while the kernels' source is the one that was captured: per launch
+    of the attention kernels, or (sha_key "losa_kernels_sha256") per block
+    run of the block-wise path."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     try:
         with open(path) as f:
             t = json.load(f)
-        sha = kernel_signature()
+        sha = kernel_signature(files)
     except (OSError, ValueError):
         return {}
-    if t.get("attn_kernels_sha256") != sha:
+    if t.get(sha_key) != sha:
         return {}
     return t.get(workload, {})
 
