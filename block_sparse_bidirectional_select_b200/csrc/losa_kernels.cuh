@@ -445,7 +445,7 @@ struct TokMassCfg {
   static constexpr int B_KFULL = 1;
   static constexpr int B_KEMPTY = B_KFULL + STAGES;
   static constexpr int B_SFULL = B_KEMPTY + STAGES;  // [2]
-  static constexpr int B_SFREE = B_SFULL + 2;        // [2] 128 reducer arrivals
+  static constexpr int B_SFREE = B_SFULL + 2;        // [2] one arrival per reducer thread
   static constexpr int B_DRAIN = B_SFREE + 2;
   static constexpr int NUM_BARS = B_DRAIN + 1;
   static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;  // tmem slot, abort flag
@@ -457,15 +457,18 @@ struct TokMassCfg {
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 };
 
-// Grid (ceil(ceil(P/128) / tiles_per_cta), H, ceil(B/128)), 256 threads. CTA
-// (x, h, z) holds the query tile z (block tokens z*128 ..) and streams the
-// prefix key tiles x*tiles_per_cta .. through a 3-deep ring: warp 0 issues the
-// copies, warp 1 owns TMEM and issues S = Q K^T per tile (double-buffered in
-// TMEM), warps 4-7 reduce. Thread r of the reducers is token z*128 + r (TMEM
-// lane r): per tile it sums 2^(s*scale*log2e - LSE*log2e) over the tile's keys
-// below P, one sum per BK-key block, in a fixed order, and writes M[h, b, j].
+// Grid (ceil(ceil(P/128) / tiles_per_cta), H, ceil(B/128)), 128 + 128 * 128/BK
+// threads. CTA (x, h, z) holds the query tile z (block tokens z*128 ..) and
+// streams the prefix key tiles x*tiles_per_cta .. through a 3-deep ring: warp 0
+// issues the copies, warp 1 owns TMEM and issues S = Q K^T per tile
+// (double-buffered in TMEM), warps 4 .. reduce in 128/BK groups of four, group
+// g taking key block g of every tile (two warps per SM sub-partition at
+// BK = 64). Thread r of a group is token z*128 + r (TMEM lane r, warp % 4 the
+// lane quarter): per tile it sums 2^(s*scale*log2e - LSE*log2e) over its key
+// block's keys below P in a fixed order (packed fp32x2 accumulators) and
+// writes M[h, b, j].
 template <int D, int BK>
-__global__ void __launch_bounds__(256, 1)
+__global__ void __launch_bounds__(384, 1)
     token_block_mass_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                             const TokMassArgs a) {
   using C = TokMassCfg<D>;
@@ -494,7 +497,7 @@ __global__ void __launch_bounds__(256, 1)
     }
     for (int b = 0; b < 2; ++b) {
       ptx::mbar_init(bar(C::B_SFULL + b), 1);
-      ptx::mbar_init(bar(C::B_SFREE + b), 128);
+      ptx::mbar_init(bar(C::B_SFREE + b), 128 * (C::N / BK));
     }
     ptx::mbar_init(bar(C::B_DRAIN), 1);
     *abort_flag = 0;
@@ -569,46 +572,55 @@ __global__ void __launch_bounds__(256, 1)
     }
   } else if (n > 0 && warp >= 4) {
     // ================================================================ reducers
+    constexpr int G = C::N / BK;     // key blocks per tile, one reducer group each
+    const int g = (warp - 4) >> 2;   // my key block within the tile
     const int wq = warp & 3;
-    const int r = wq * 32 + lane;  // token of this CTA == TMEM lane
+    const int r = wq * 32 + lane;    // token of this CTA == TMEM lane
     const int tok = qt * C::M + r;
     const bool valid = tok < a.B;
     const uint32_t lane_base = tmem + (static_cast<uint32_t>(wq * 32) << 16);
-    const float sl2 = a.scale_log2;
-    const float lse2 = valid ? a.lse[static_cast<long>(h) * a.B + tok] * 1.44269504088896340736f : 0.f;
+    const uint64_t sl2 = ptx::f32x2(a.scale_log2, a.scale_log2);
+    const float nl = valid ? a.lse[static_cast<long>(h) * a.B + tok] * -1.44269504088896340736f : 0.f;
+    const uint64_t nl2 = ptx::f32x2(nl, nl);
     float* out = a.mass + (static_cast<long>(h) * a.B + (valid ? tok : 0)) * a.nkb;
     for (int i = 0; i < n; ++i) {
       const int b = i & 1;
       if (!ptx::mbar_wait_warp(bar(C::B_SFULL + b), (i >> 1) & 1, abort_flag, a.timeout_ns, kErrTimeout)) break;
       ptx::tc_fence_after();
-      const int key0 = (t0 + i) * C::N;
-      float part[4];
+      uint32_t raw[BK / 32][32];
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        uint32_t raw[32];
-        ptx::tmem_ld32(lane_base + (b ? C::TM_S1 : C::TM_S0) + c * 32, raw);
-        ptx::tmem_wait_ld();
-        ptx::reg_fence32(raw);
-        float acc = 0.f;
-        const int nvalid = a.P - (key0 + c * 32);  // keys of this chunk below P
-        if (valid) {
-#pragma unroll
-          for (int e = 0; e < 32; ++e)
-            if (e < nvalid) acc += ptx::ex2(fmaf(__uint_as_float(raw[e]), sl2, -lse2));
-        }
-        part[c] = acc;
-      }
+      for (int c = 0; c < BK / 32; ++c)
+        ptx::tmem_ld32(lane_base + (b ? C::TM_S1 : C::TM_S0) + g * BK + c * 32, raw[c]);
+      ptx::tmem_wait_ld();
       ptx::tc_fence_before();
-      ptx::mbar_arrive(bar(C::B_SFREE + b));
-      if (valid) {
-        const int tile = t0 + i;
-        if constexpr (BK == 128) {
-          out[tile] = (part[0] + part[1]) + (part[2] + part[3]);
-        } else {
-          out[2 * tile] = part[0] + part[1];
-          if (2 * tile + 1 < a.nkb) out[2 * tile + 1] = part[2] + part[3];
+      ptx::mbar_arrive(bar(C::B_SFREE + b));  // S_b is in registers: the MMA may overwrite it
+      const int blk = (t0 + i) * G + g;
+      const int nvalid = a.P - blk * BK;      // keys of my block below P
+      uint64_t acc0 = ptx::f32x2(0.f, 0.f), acc1 = acc0;
+#pragma unroll
+      for (int c = 0; c < BK / 32; ++c) {
+        ptx::reg_fence32(raw[c]);
+#pragma unroll
+        for (int e = 0; e < 32; e += 2) {
+          float x0, x1;
+          ptx::f32x2_split(ptx::fma_f32x2(ptx::f32x2(__uint_as_float(raw[c][e]), __uint_as_float(raw[c][e + 1])), sl2,
+                                          nl2),
+                           x0, x1);
+          float p0 = ptx::ex2(x0), p1 = ptx::ex2(x1);
+          if (nvalid < BK) {  // the ragged end of the prefix
+            p0 = c * 32 + e < nvalid ? p0 : 0.f;
+            p1 = c * 32 + e + 1 < nvalid ? p1 : 0.f;
+          }
+          if (e & 2)
+            acc1 = ptx::add_f32x2(acc1, ptx::f32x2(p0, p1));
+          else
+            acc0 = ptx::add_f32x2(acc0, ptx::f32x2(p0, p1));
         }
       }
+      float a0, a1, b0, b1;
+      ptx::f32x2_split(acc0, a0, a1);
+      ptx::f32x2_split(acc1, b0, b1);
+      if (valid && blk < a.nkb) out[blk] = (a0 + b0) + (a1 + b1);
     }
   }
 

@@ -1545,7 +1545,7 @@ int launch_tok_mass_t(const LosaDims& g, const uint16_t* Q, const uint16_t* Kp, 
   const long ntiles = cdiv(g.P, C::N);
   const dim3 grid(static_cast<unsigned>(cdiv(ntiles, a.tiles_per_cta)), static_cast<unsigned>(g.H),
                   static_cast<unsigned>(cdiv(g.B, C::M)));
-  kern<<<grid, 256, C::SMEM_BYTES, st>>>(tq, tk, a);
+  kern<<<grid, 128 + 128 * (C::N / BK), C::SMEM_BYTES, st>>>(tq, tk, a);
   SP_CUDA(cudaGetLastError());
   return SPARSED_OK;
 }

@@ -294,3 +294,29 @@ def test_full_size_block_sampled():
         o_s, l_s = O.softmax_attention(q, f64(ks[t][h]), f64(vs[t][h]), wl.scale)
         o_r, l_r = O.merge_partials(o_p, l_p, o_s, l_s)
         assert_o_lse(ot[h, rows], lt[h, rows], o_r, l_r, f"full size step {t} h={h}")
+
+
+def test_block_run_replayed_from_a_cuda_graph_gives_the_eager_bits():
+    """The block run captured in a CUDA graph: the side stream joins the
+    capture through its fork and join events, and the list, prefix and merge
+    kernels enter it as programmatic dependents of the kernel before them.
+    Every replay gives the bits of the eager run."""
+    wl, (k_pre, v_pre, qs, ks, vs) = _case(2, 2048, 64, 128, 64, 64, 3, T=5, seed=23)
+    kp, vp, qg, kg, vg = _cuda(k_pre, v_pre, qs, ks, vs)
+    eager = sp.losa_block(qg, kg, vg, kp, vp, n_sel=3, tau=wl.tau)
+    sp.device_check()
+    out = torch.empty_like(qg)
+    lse = torch.empty_like(eager.lse)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        cap = sp.losa_block(qg, kg, vg, kp, vp, n_sel=3, tau=wl.tau, splits=eager.state.splits, out=out, lse=lse)
+    for _ in range(2):
+        out.zero_()
+        lse.zero_()
+        graph.replay()
+        torch.cuda.synchronize()
+        sp.device_check()
+        assert torch.equal(out.view(torch.int16), eager.o.view(torch.int16))
+        assert torch.equal(lse, eager.lse)
+        assert torch.equal(cap.active, eager.active) and torch.equal(cap.union_count, eager.union_count)
+    assert (eager.active[1:].sum(dim=1) > 0).any()  # later steps with active tokens took the sparse path
