@@ -133,10 +133,11 @@ struct LosaListArgs {
 //   1. the active tokens in ascending order (warp ballots), and pos[] (head 0)
 //   2. the union as a bitmask over prefix blocks (shared-memory atomics)
 //   3. the ascending union list: each thread expands a contiguous run of words
-//      at the offset of an exclusive scan of the runs' bit counts
+//      at the offset of an exclusive scan of the runs' bit counts, and writes
+//      each entry straight into the split lists as well
 //   4. split s holds union entries [s*chunk, (s+1)*chunk), chunk =
 //      max(kLosaMinChunk, ceil(u / S)); work item (s, t) of query tile t gets
-//      that chunk when the tile holds an active token, else nothing
+//      that chunk when the tile holds an active token, else nothing (counts)
 //   5. row s*R + a of q_rep is the a-th active token's query (zero past the
 //      active count) for every split and tile that have work
 __global__ void __launch_bounds__(256) losa_lists_kernel(const LosaListArgs a) {
@@ -226,39 +227,36 @@ __global__ void __launch_bounds__(256) losa_lists_kernel(const LosaListArgs a) {
   }
   __syncthreads();
   int32_t* ulist = a.union_idx + static_cast<long>(h) * a.nkb;
+  const int u = s_u;
+  const int items = a.S * a.tiles;
+  int chunk = (u + a.S - 1) / a.S;
+  if (chunk < kLosaMinChunk) chunk = kLosaMinChunk;
+  const long item0 = static_cast<long>(h) * items;
   int outp = s_scan[wid] + incl - cnt;
   for (int w = w0; w < w1; ++w) {
     uint32_t m = s_bits[w];
     while (m) {
-      ulist[outp++] = (w << 5) + (__ffs(m) - 1);
+      const int j = (w << 5) + (__ffs(m) - 1);
+      ulist[outp] = j;
+      // entry outp of the union is entry jj of split s, for every tile with work
+      const int s = outp / chunk, jj = outp - s * chunk;
+      for (int t = 0; t < a.tiles && t * a.bq < na; ++t) a.kv_idx[(item0 + s * a.tiles + t) * a.kv_stride + jj] = j;
+      ++outp;
       m &= m - 1u;
     }
   }
-  const int u = s_u;
   if (tid == 0) a.union_count[h] = u;
-  __syncthreads();  // the union list (global, this CTA's writes) is complete
 
-  // 4. split lists
-  const int items = a.S * a.tiles;
-  int chunk = (u + a.S - 1) / a.S;
-  if (chunk < kLosaMinChunk) chunk = kLosaMinChunk;
+  // 4. split list lengths
   auto split_len = [&](int s) -> int {
     if (na == 0) return 0;
     const int left = u - s * chunk;
     return left <= 0 ? 0 : (left < chunk ? left : chunk);
   };
-  const long item0 = static_cast<long>(h) * items;
   for (int it = tid; it < items; it += 256) {
     const int s = it / a.tiles;
     const int t = it - s * a.tiles;
     a.kv_count[item0 + it] = (t * a.bq < na) ? split_len(s) : 0;
-  }
-  for (long e = tid; e < static_cast<long>(items) * a.kv_stride; e += 256) {
-    const int it = static_cast<int>(e / a.kv_stride);
-    const int jj = static_cast<int>(e - static_cast<long>(it) * a.kv_stride);
-    const int s = it / a.tiles;
-    const int t = it - s * a.tiles;
-    if (t * a.bq < na && jj < split_len(s)) a.kv_idx[(item0 + it) * a.kv_stride + jj] = ulist[s * chunk + jj];
   }
 
   // 5. replicated queries of the tiles that have work: each 16-byte piece of
@@ -267,12 +265,24 @@ __global__ void __launch_bounds__(256) losa_lists_kernel(const LosaListArgs a) {
   const uint4* qsrc = reinterpret_cast<const uint4*>(a.q) + static_cast<long>(h) * a.B * row_u4;
   uint4* qdst = reinterpret_cast<uint4*>(a.q_rep) + static_cast<long>(h) * a.S * a.R * row_u4;
   const int rows = ((na + a.bq - 1) / a.bq) * a.bq;  // rows of the tiles with work (<= R)
-  for (int e = tid; e < rows * row_u4; e += 256) {
-    const int r = e / row_u4;
-    const int c = e - r * row_u4;
-    const uint4 val = r < na ? qsrc[static_cast<long>(s_act[r]) * row_u4 + c] : make_uint4(0u, 0u, 0u, 0u);
-    for (int s = 0; s < a.S; ++s)
-      if (split_len(s) > 0) qdst[(static_cast<long>(s) * a.R + r) * row_u4 + c] = val;
+  const int total = rows * row_u4;
+  for (int e0 = tid; e0 < total; e0 += 4 * 256) {
+    uint4 val[4];  // four pieces' loads in flight before their stores
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const int e = e0 + k * 256;
+      const int r = e / row_u4;
+      val[k] = (e < total && r < na) ? qsrc[static_cast<long>(s_act[r]) * row_u4 + (e - r * row_u4)]
+                                     : make_uint4(0u, 0u, 0u, 0u);
+    }
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const int e = e0 + k * 256;
+      if (e >= total) break;
+      const int r = e / row_u4;
+      for (int s = 0; s < a.S; ++s)
+        if (split_len(s) > 0) qdst[(static_cast<long>(s) * a.R + r) * row_u4 + (e - r * row_u4)] = val[k];
+    }
   }
 }
 
@@ -318,9 +328,11 @@ __global__ void __launch_bounds__(256) losa_merge_kernel(const LosaMergeArgs a) 
   if (ap >= 0) {
     const int t = ap / a.bq;
     const long rep0 = static_cast<long>(h) * a.S * a.R + ap;
-    float l_s = kNegInf;
-    if (lane < a.S && a.kv_count[static_cast<long>(h) * a.S * a.tiles + lane * a.tiles + t] > 0)
-      l_s = a.lse_rep[rep0 + static_cast<long>(lane) * a.R];
+    // both loads at once: every split's rows are written by the prefix pass
+    // (LSE -inf for a split without work), so the LSE read never waits on the count
+    const int kc = lane < a.S ? a.kv_count[static_cast<long>(h) * a.S * a.tiles + lane * a.tiles + t] : 0;
+    const float lr = lane < a.S ? a.lse_rep[rep0 + static_cast<long>(lane) * a.R] : kNegInf;
+    const float l_s = kc > 0 ? lr : kNegInf;
     float m = l_s;
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
