@@ -8,7 +8,10 @@
 //                                  exp(scale*<q_r,k_c> - LSE_r)
 //                       recomputes S = Q K^T on tcgen05 (fp32 in TMEM) and
 //                       reduces every 128 x BK tile to one fp32 scalar in a
-//                       fixed order (bit-reproducible).
+//                       fixed order (bit-reproducible): BK/32 groups of four
+//                       reducer warps, each warp 32 columns of every tile, its
+//                       partial handed to one combining warp through shared
+//                       memory (mbarriers, no barrier across the reducers).
 //   row_entropy_kernel  entropy of each row M[h,i,:] / sum_j M[h,i,j] (fp64)
 //   budget_kernel       per-head k_h from the mean row entropy (fp64, one thread)
 //   topk_kernel         per (h,i): the k_h largest masses, ties to the lower
@@ -45,9 +48,14 @@ struct MassCfg {
   static constexpr int B_SFULL = B_KEMPTY + STAGES;
   static constexpr int B_SFREE = B_SFULL + 2;
   static constexpr int B_DRAIN = B_SFREE + 2;
-  static constexpr int NUM_BARS = B_DRAIN + 1;
-  static constexpr int OFF_RED = OFF_BAR + NUM_BARS * 8;     // float red[2][4]
-  static constexpr int OFF_MISC = OFF_RED + 2 * 4 * 4;       // tmem slot, abort flag
+  static constexpr int B_REDFULL = B_DRAIN + 1;    // [2] one arrival per reducer warp
+  static constexpr int B_REDEMPTY = B_REDFULL + 2; // [2] the combining warp has read red[b]
+  static constexpr int NUM_BARS = B_REDEMPTY + 2;
+  static constexpr int G = BK / 32;                // reducer groups: 32 columns of every tile each
+  static constexpr int RWARPS = 4 * G;             // reducer warps (warps 4 ..)
+  static constexpr int THREADS = 128 + 32 * RWARPS;
+  static constexpr int OFF_RED = OFF_BAR + NUM_BARS * 8;     // float red[2][RWARPS]
+  static constexpr int OFF_MISC = OFF_RED + 2 * RWARPS * 4;  // tmem slot, abort flag
   static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;
   static constexpr int TM_S0 = 0;
   static constexpr int TM_S1 = BK;
@@ -57,7 +65,7 @@ struct MassCfg {
 };
 
 template <int D, int BK>
-__global__ void __launch_bounds__(256, 1)
+__global__ void __launch_bounds__(MassCfg<D, BK>::THREADS, 1)
     block_mass_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                       const MassArgs a) {
   using C = MassCfg<D, BK>;
@@ -83,7 +91,9 @@ __global__ void __launch_bounds__(256, 1)
     }
     for (int b = 0; b < 2; ++b) {
       ptx::mbar_init(bar(C::B_SFULL + b), 1);
-      ptx::mbar_init(bar(C::B_SFREE + b), 128);
+      ptx::mbar_init(bar(C::B_SFREE + b), 32 * C::RWARPS);
+      ptx::mbar_init(bar(C::B_REDFULL + b), C::RWARPS);
+      ptx::mbar_init(bar(C::B_REDEMPTY + b), 1);
     }
     ptx::mbar_init(bar(C::B_DRAIN), 1);
     *abort_flag = 0;
@@ -160,47 +170,76 @@ __global__ void __launch_bounds__(256, 1)
       volatile int dummy = 0;
       ptx::mbar_wait(bar(C::B_DRAIN), 0, &dummy, a.timeout_ns / 4, 0);
     }
+  } else if (warp == 2) {
+    // ================================================================ combiner
+    // tile j's mass: the reducer warps' partials in warp order
+    float* out = a.mass + (static_cast<long>(h) * a.nqb + qi) * a.nkb;
+    for (int j = 0; j < n; ++j) {
+      const int b = j & 1;
+      if (!ptx::mbar_wait_warp(bar(C::B_REDFULL + b), (j >> 1) & 1, abort_flag, a.timeout_ns, kErrTimeout)) break;
+      if (lane == 0) {
+        float t = 0.f;
+#pragma unroll
+        for (int w = 0; w < C::RWARPS; ++w) t += red[b * C::RWARPS + w];
+        if (!*abort_flag) out[j] = t;
+        ptx::mbar_arrive(bar(C::B_REDEMPTY + b));
+      }
+      __syncwarp();
+    }
   } else if (warp >= 4) {
     // ================================================================ reducers
-    const int wq = warp & 3;
+    const int rw = warp - 4;    // reducer warp
+    const int g = rw >> 2;      // columns 32g .. 32g + 31 of every tile
+    const int wq = warp & 3;    // TMEM lane quarter
     const int r = wq * 32 + lane;
     const uint32_t lane_base = tmem + (static_cast<uint32_t>(wq * 32) << 16);
     const int grow = qi * a.bq + r;
     const bool row_valid = (r < a.bq) && (grow < a.L);
-    const float lse2 = row_valid ? a.lse[static_cast<long>(h) * a.L + grow] * 1.44269504088896340736f : 0.f;
-    const float sl2 = a.scale_log2;
-    float* out = a.mass + (static_cast<long>(h) * a.nqb + qi) * a.nkb;
+    const float nl = row_valid ? a.lse[static_cast<long>(h) * a.L + grow] * -1.44269504088896340736f : 0.f;
+    const uint64_t nl2 = ptx::f32x2(nl, nl);
+    const uint64_t sl2 = ptx::f32x2(a.scale_log2, a.scale_log2);
     for (int j = 0; j < n; ++j) {
       const int b = j & 1;
-      // after an abort every wait returns at once; the loop still runs to the
-      // end so all 128 reducers take every named barrier
-      const bool ok =
-          ptx::mbar_wait_warp(bar(C::B_SFULL + b), (j >> 1) & 1, abort_flag, a.timeout_ns, kErrTimeout);
-      float acc = 0.f;
-      if (ok) {
-        ptx::tc_fence_after();
-        const int valid = a.L - j * BK < BK ? a.L - j * BK : BK;
-        float part[4] = {0.f, 0.f, 0.f, 0.f};
+      if (!ptx::mbar_wait_warp(bar(C::B_SFULL + b), (j >> 1) & 1, abort_flag, a.timeout_ns, kErrTimeout)) break;
+      ptx::tc_fence_after();
+      uint32_t raw[32];
+      ptx::tmem_ld32(lane_base + (b ? C::TM_S1 : C::TM_S0) + g * 32, raw);
+      ptx::tmem_wait_ld();
+      ptx::tc_fence_before();
+      ptx::mbar_arrive(bar(C::B_SFREE + b));  // S_b is in registers: the MMA may overwrite it
+      ptx::reg_fence32(raw);
+      const int valid = (a.L - j * BK < BK ? a.L - j * BK : BK) - g * 32;  // key columns of mine below L
+      uint64_t acc0 = ptx::f32x2(0.f, 0.f), acc1 = acc0;
 #pragma unroll
-        for (int c = 0; c < BK / 32; ++c) {
-          uint32_t raw[32];
-          ptx::tmem_ld32(lane_base + (b ? C::TM_S1 : C::TM_S0) + c * 32, raw);
-          ptx::tmem_wait_ld();
-#pragma unroll
-          for (int e = 0; e < 32; ++e) {
-            const float p = ptx::ex2(fmaf(__uint_as_float(raw[e]), sl2, -lse2));
-            part[e & 3] += (c * 32 + e < valid) ? p : 0.f;
-          }
+      for (int e = 0; e < 32; e += 2) {
+        float x0, x1;
+        ptx::f32x2_split(ptx::fma_f32x2(ptx::f32x2(__uint_as_float(raw[e]), __uint_as_float(raw[e + 1])), sl2, nl2),
+                         x0, x1);
+        float p0 = ptx::ex2(x0), p1 = ptx::ex2(x1);
+        if (valid < 32) {  // the ragged last key block
+          p0 = e < valid ? p0 : 0.f;
+          p1 = e + 1 < valid ? p1 : 0.f;
         }
-        ptx::tc_fence_before();
-        ptx::mbar_arrive(bar(C::B_SFREE + b));
-        acc = row_valid ? (part[0] + part[1]) + (part[2] + part[3]) : 0.f;
+        if (e & 2)
+          acc1 = ptx::add_f32x2(acc1, ptx::f32x2(p0, p1));
+        else
+          acc0 = ptx::add_f32x2(acc0, ptx::f32x2(p0, p1));
       }
+      float a0, a1, b0, b1;
+      ptx::f32x2_split(acc0, a0, a1);
+      ptx::f32x2_split(acc1, b0, b1);
+      float acc = row_valid ? (a0 + b0) + (a1 + b1) : 0.f;
 #pragma unroll
       for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-      if (lane == 0) red[b * 4 + wq] = acc;
-      ptx::named_bar_sync(1, 128);
-      if (r == 0 && !*abort_flag) out[j] = (red[b * 4 + 0] + red[b * 4 + 1]) + (red[b * 4 + 2] + red[b * 4 + 3]);
+      // red[b] was last read for tile j - 2
+      if (j >= 2 && !ptx::mbar_wait_warp(bar(C::B_REDEMPTY + b), ((j >> 1) - 1) & 1, abort_flag, a.timeout_ns,
+                                         kErrTimeout))
+        break;
+      if (lane == 0) {
+        red[b * C::RWARPS + rw] = acc;
+        ptx::mbar_arrive(bar(C::B_REDFULL + b));
+      }
+      __syncwarp();
     }
   }
 

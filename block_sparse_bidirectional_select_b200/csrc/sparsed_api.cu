@@ -410,7 +410,7 @@ int launch_mass_t(const Problem& p, float* mass, cudaStream_t st) {
   a.timeout_ns = kWaitTimeoutNs;
   auto kern = block_mass_kernel<D, BK>;
   SP_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES));
-  kern<<<dim3(p.nqb, p.H), 256, C::SMEM_BYTES, st>>>(tq, tk, a);
+  kern<<<dim3(p.nqb, p.H), C::THREADS, C::SMEM_BYTES, st>>>(tq, tk, a);
   SP_CUDA(cudaGetLastError());
   return SPARSED_OK;
 }
