@@ -392,6 +392,13 @@ int launch_attn(const Problem& p, bool sparse, const int32_t* kv_idx, const int3
   return SPARSED_ERR_UNSUPPORTED;
 }
 
+// One dense pass whose pairs come from the counter slots in a call's workspace.
+int dense_pass_counted(const Problem& p, void* slots, cudaStream_t st) {
+  PairSched ps;
+  SP_TRY(begin_pair_sched(&ps, slots, st));
+  return launch_attn(p, false, nullptr, nullptr, 0, st, nullptr, nullptr, &ps);
+}
+
 template <int D, int BK>
 int launch_mass_t(const Problem& p, float* mass, cudaStream_t st) {
   using C = MassCfg<D, BK>;
@@ -775,7 +782,7 @@ int sparsed_select_pattern(const uint16_t* Q, const uint16_t* K, const uint16_t*
   SP_TRY(require_sm100());
   SP_TRY(get_encoder());
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  SP_TRY(launch_attn(p, false, nullptr, nullptr, 0, st));
+  SP_TRY(dense_pass_counted(p, static_cast<uint8_t*>(workspace) + ws_layout(p.H, p.nqb, p.nkb).sched, st));
   return select_after_dense(p, keep_ratio, budget_mode, kv_idx, kv_count, kv_stride, block_mass, head_k,
                             workspace, st);
 }
@@ -980,7 +987,7 @@ int sparsed_select_head_entropy(const uint16_t* Q, const uint16_t* K, const uint
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   float* mass = reinterpret_cast<float*>(ws + w.grid);
   double* ent = reinterpret_cast<double*>(ws + w.ent);
-  SP_TRY(launch_attn(p, false, nullptr, nullptr, 0, st));
+  SP_TRY(dense_pass_counted(p, ws + w.sched, st));
   SP_TRY(launch_mass(p, mass, st));
   const int rows = p.H * p.nqb;
   row_entropy_kernel<<<(rows + 7) / 8, 256, 0, st>>>(mass, rows, p.nkb, ent);
@@ -1094,7 +1101,7 @@ int sparsed_select_columns(const uint16_t* Q, const uint16_t* K, const uint16_t*
   SP_TRY(require_sm100());
   SP_TRY(get_encoder());
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  SP_TRY(launch_attn(p, false, nullptr, nullptr, 0, st));
+  SP_TRY(dense_pass_counted(p, static_cast<uint8_t*>(workspace) + col_ws_layout(p.H, p.L, p.d, kc).sched, st));
   return select_columns_after_dense(p, kc, cols, col_stride, col_mass, workspace, st);
 }
 

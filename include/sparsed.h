@@ -150,7 +150,9 @@ int sparsed_dense_attn(const uint16_t* Q, const uint16_t* K, const uint16_t* V,
  *      index), written ascending to kv_idx, and kv_count[h*nqb+i] = k_h.
  * kv_stride >= k (UNIFORM) or >= nkb (ENTROPY). workspace: device memory of at
  * least sparsed_workspace_bytes(H, L, bq, bk) bytes, 256-byte aligned, owned by
- * the caller; contents on entry are ignored. */
+ * the caller; contents on entry are ignored. The full pass takes its pairs of
+ * query blocks from counters kept in the workspace (cleared by the call), so
+ * one workspace must not serve two calls at the same time. */
 int sparsed_select_pattern(const uint16_t* Q, const uint16_t* K, const uint16_t* V,
                            int H, int L, int d, float scale, int bq, int bk,
                            float keep_ratio, int budget_mode,
@@ -332,7 +334,9 @@ int sparsed_run_steps_drift(const uint16_t* Q, const uint16_t* K, const uint16_t
 /* Steps 1-2 of sparsed_select_pattern for this rank's H heads, then the mean
  * row entropy E_h of every head (as in the ENTROPY budget) into head_entropy
  * (DEVICE [H] fp64). The block mass stays in the workspace (at least
- * sparsed_workspace_bytes(H, L, bq, bk) bytes) for sparsed_select_with_head_k. */
+ * sparsed_workspace_bytes(H, L, bq, bk) bytes) for sparsed_select_with_head_k.
+ * The full pass takes its pairs from counters in the workspace, as in
+ * sparsed_select_pattern. */
 int sparsed_select_head_entropy(const uint16_t* Q, const uint16_t* K, const uint16_t* V,
                                 int H, int L, int d, float scale, int bq, int bk,
                                 uint16_t* O, float* LSE, double* head_entropy,
@@ -364,8 +368,9 @@ int sparsed_select_with_head_k(int H, int L, int bq, int bk, const int32_t* head
 int sparsed_column_keep(int L, float keep_ratio, int* kc);
 
 /* Workspace bytes of the column path for H heads, L tokens, head dim d and kc
- * kept columns: the column-mass array [H, L] fp32 and the gathered K and V
- * columns [H, kc, d] bf16 each, every part 256-byte aligned. */
+ * kept columns: the column-mass array [H, L] fp32, the gathered K and V
+ * columns [H, kc, d] bf16 each and the full passes' pair counters, every part
+ * 256-byte aligned. */
 int sparsed_column_workspace_bytes(int H, int L, int d, int kc, size_t* bytes);
 
 /* One full-attention pass that also selects the column pattern:
@@ -376,7 +381,8 @@ int sparsed_column_workspace_bytes(int H, int L, int d, int kc, size_t* bytes);
  *      written ascending to cols [H, col_stride], col_stride >= kc.
  * workspace: device memory of at least sparsed_column_workspace_bytes(H, L, d,
  * kc) bytes, 256-byte aligned, owned by the caller; contents on entry are
- * ignored. */
+ * ignored. The full pass takes its pairs from counters in the workspace, as in
+ * sparsed_select_pattern. */
 int sparsed_select_columns(const uint16_t* Q, const uint16_t* K, const uint16_t* V,
                            int H, int L, int d, float scale, int bq, int bk, float keep_ratio,
                            uint16_t* O, float* LSE, int32_t* cols, int col_stride,
