@@ -61,8 +61,7 @@ def test_bf16_round_matches_torch():
 
 
 def test_drift_queries_against_torch_arithmetic():
-    rng = np.random.default_rng(2)
-    q = torch.randn(3, 40, 16).to(torch.bfloat16)
+    q = torch.randn(3, 40, 16, generator=torch.Generator().manual_seed(2)).to(torch.bfloat16)
     q64 = q.to(torch.float64).numpy()
     for seed, t in [(0, 0), (17, 5), (2 ** 31 + 3, 1000)]:
         got = O.drift_queries(q64, seed, t)
@@ -70,12 +69,12 @@ def test_drift_queries_against_torch_arithmetic():
         d = torch.from_numpy(u * O.DRIFT_AMPLITUDE).to(torch.float32)
         ref = (q.to(torch.float32) + d).to(torch.bfloat16).to(torch.float64).numpy()
         assert np.array_equal(got, ref)
-        # a perturbation of at most the amplitude plus half a bf16 step
-        bound = O.DRIFT_AMPLITUDE + np.abs(q64 + O.DRIFT_AMPLITUDE) * 2.0 ** -8
+        # a perturbation of at most the amplitude plus half a bf16 step of the
+        # sum: half an ulp of x is at most |x| * 2^-8, and |q + u*amp| <= |q| + amp
+        bound = O.DRIFT_AMPLITUDE + (np.abs(q64) + O.DRIFT_AMPLITUDE) * 2.0 ** -8
         assert np.all(np.abs(got - q64) <= bound)
     assert np.array_equal(O.drift_queries(q64, 9, 3, amplitude=0.0), q64)
     assert not np.array_equal(O.drift_queries(q64, 9, 3), O.drift_queries(q64, 9, 4))
-    _ = rng
 
 
 def _bf16(x):
