@@ -343,3 +343,41 @@ def test_sharded_loop_validates_on_the_host():
     if not GPU:
         assert run() == _lib.ERR_NO_DEVICE
         assert run(budget=0, exchange=None) == _lib.ERR_NO_DEVICE
+
+
+def _c_kind(decl):
+    """Kind of a C parameter or return type: 'ptr' (any pointer, the exchange
+    callback), 'int', 'float', 'u64' (size_t, uint64_t), 'u32' (uint32_t)."""
+    t = decl.strip()
+    if "*" in t or "sparsed_exchange_fn" in t:
+        return "ptr"
+    t = re.sub(r"\bconst\b", "", t).split()
+    base = " ".join(t[:-1]) if len(t) > 1 else t[0]
+    return {"int": "int", "float": "float", "size_t": "u64", "uint64_t": "u64", "unsigned long long": "u64",
+            "uint32_t": "u32", "unsigned": "u32", "unsigned int": "u32"}[base]
+
+
+def _ctypes_kind(tp):
+    if tp in (ctypes.c_void_p, ctypes.c_char_p) or isinstance(tp, type) and issubclass(tp, ctypes._Pointer):
+        return "ptr"
+    return {ctypes.c_int: "int", ctypes.c_float: "float", ctypes.c_size_t: "u64", ctypes.c_ulonglong: "u64",
+            ctypes.c_uint: "u32"}[tp]
+
+
+def test_binding_prototypes_match_the_header():
+    """Every declaration of sparsed.h against the binding's ctypes prototype:
+    the same number of parameters, each of the same kind, and the same return
+    kind, so a float passed where the ABI takes an int (or a dropped argument)
+    fails here rather than on a device."""
+    text = re.sub(r"/\*.*?\*/", "", open(HEADER).read(), flags=re.S)
+    decls = re.findall(r"([A-Za-z_][\w \t\*]*?)\s*\b(sparsed_\w+)\s*\(([^;]*?)\)\s*;", text, flags=re.S)
+    seen = set()
+    for ret, name, params in decls:
+        params = " ".join(params.split())
+        c_args = [] if params in ("", "void") else [_c_kind(p) for p in params.split(",")]
+        restype, argtypes = _lib.SIGNATURES[name]
+        assert [_ctypes_kind(a) for a in argtypes] == c_args, name
+        ret_kind = "ptr" if "*" in ret else _c_kind(ret + " r")
+        assert _ctypes_kind(restype) == ret_kind, name
+        seen.add(name)
+    assert seen == set(_lib.SIGNATURES)
